@@ -1,0 +1,427 @@
+#!/usr/bin/env python
+"""Benchmark of the packed ternary-weight decode GEMV on B200.
+
+Default workload: the BitNet b1.58-2B decode layer set -- 30 layers x 7
+projections (q/o 2560x2560, k/v 640x2560, gate/up 6912x2560, down
+2560x6912), batch 1, single ternary plane with a per-tensor scale, int8
+per-token absmax activations, fp32 output, each GEMV with its own seeded
+weights and activations. One step = per-token quantisation of each GEMV's bf16
+activation followed by the GEMV, for all 210 GEMVs in layer order (521 MB of
+packed weights, so every step streams from HBM: inputs larger than L2).
+
+Metric: achieved HBM GB/s over the step (algorithmic bytes: packed weights,
+activations read and written, outputs) and its fraction of the measured copy
+bandwidth; per-shape figures are reported alongside.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  torchrun --nproc-per-node N bench.py --gpus N ...   (independent replicas)
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from packed_ternary_weight_b200 import synth  # noqa: E402
+
+METRIC = "decode GEMV achieved HBM GB/s and % of B200 roofline per layer shape, 1 GPU"
+WORKLOAD = ("BitNet b1.58-2B decode layer set: 30 layers x 7 projections (q,o 2560x2560; k,v 640x2560; "
+            "gate,up 6912x2560; down 2560x6912), batch 1, single ternary plane, per-tensor scale 0.02, "
+            "int8 per-token absmax activations, fp32 out, distinct seeds")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--layers", type=int, default=synth.BITNET_2B_LAYERS)
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, enabled: bool):
+        self.proc = None
+        self.gpu = gpu_index
+        if not enabled:
+            return
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], 0.0, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- our impl
+def run_ours(args, rank, world):
+    import torch
+    import torch.distributed as dist
+
+    from packed_ternary_weight_b200 import tern
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream()
+    layers = []           # per GEMV: dict with desc, packed, offsets
+    x_host = []
+    k_tot = n_tot = 0
+    for lay in synth.bitnet_layer_set(args.layers):
+        d, buf = tern.pack_layer(lay, flags=tern.F_PDL)
+        x = synth.draw_x_bf16(lay.seed, 1, lay.k)[0]
+        layers.append(dict(name=lay.name.split(".", 1)[1], n=lay.n, k=lay.k, desc=d,
+                           packed=torch.from_numpy(buf).to(dev), wbytes=len(buf) - 256,
+                           xoff=k_tot, yoff=n_tot))
+        x_host.append(x)
+        k_tot += lay.k
+        n_tot += lay.n
+        del lay
+    x_all_host = torch.from_numpy(np.concatenate(x_host).view(np.int16)).pin_memory()
+    y_all_host = torch.empty(n_tot, dtype=torch.float32).pin_memory()
+    x_all = x_all_host.to(dev)
+    xq_all = torch.empty(k_tot, dtype=torch.int8, device=dev)
+    sx_all = torch.empty(len(layers), dtype=torch.float32, device=dev)
+    y_all = torch.empty(n_tot, dtype=torch.float32, device=dev)
+    ws_bytes = max(tern.workspace_size(L["desc"], 1) for L in layers)
+    ws = torch.zeros(max(16, ws_bytes), dtype=torch.uint8, device=dev)
+
+    def quant(i, L):
+        tern.quantize_act(x_all[L["xoff"]:L["xoff"] + L["k"]].view(1, L["k"]),
+                          xq_all[L["xoff"]:L["xoff"] + L["k"]], sx_all[i:i + 1], stream)
+
+    def gemv(i, L):
+        tern.gemv(L["desc"], L["packed"], tern.ACT_INT8, xq_all[L["xoff"]:L["xoff"] + L["k"]], sx_all[i:i + 1],
+                  tern.OUT_F32, y_all[L["yoff"]:L["yoff"] + L["n"]], ws, stream)
+
+    def step():
+        for i, L in enumerate(layers):
+            quant(i, L)
+            gemv(i, L)
+
+    def gemv_only(sel=None):
+        for i, L in enumerate(layers):
+            if sel is None or L["name"] == sel:
+                gemv(i, L)
+
+    # bytes that must move per step (algorithmic): packed weights, the bf16
+    # activation read and int8 activation written by the quantiser, the int8
+    # activation and scale read by the GEMV, the fp32 output written
+    gemv_bytes = sum(L["wbytes"] + L["k"] + 4 + 4 * L["n"] for L in layers)
+    quant_bytes = sum(2 * L["k"] + L["k"] + 4 for L in layers)
+    step_bytes = gemv_bytes + quant_bytes
+
+    with torch.cuda.stream(stream):
+        step()                      # eager warm-up, sets kernel attributes
+        torch.cuda.synchronize()
+        assert tern.device_error(stream) == tern.OK
+        g_step = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step, stream=stream):
+            step()
+        g_gemv = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_gemv, stream=stream):
+            gemv_only()
+        shape_graphs = {}
+        for name, _, _ in synth.BITNET_2B_SHAPES:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                gemv_only(name)
+            shape_graphs[name] = g
+    torch.cuda.synchronize()
+
+    # parity spot check of the captured step (first GEMV) against the oracle
+    parity = None
+    if rank == 0:
+        import oracle
+        g_step.replay()
+        torch.cuda.synchronize()
+        lay0 = next(iter(synth.bitnet_layer_set(1)))
+        x0 = synth.draw_x_bf16(lay0.seed, 1, lay0.k)
+        q, s = oracle.quantize_act(x0)
+        yref = oracle.gemv_bitnet_int8(lay0.trits, q, s, lay0.tensor_scale)[0]
+        got = y_all[:lay0.n].cpu().numpy()
+        parity = bool(np.array_equal(got.view(np.uint32), yref.view(np.uint32)))
+        del lay0
+
+    def timed(graph, reps):
+        with torch.cuda.stream(stream):
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                graph.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1)
+            if world > 1:
+                t = torch.tensor([ms], device=dev)
+                dist.all_reduce(t, op=dist.ReduceOp.MAX)
+                ms = float(t.item())
+                dist.barrier()
+        return ms
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            g_step.replay()
+        torch.cuda.synchronize()
+    clocks = ClockSampler(dev.index, not args.no_clocks and rank == 0)
+    # soak so that the clock samples see the GPU under this load
+    t_end = time.time() + 1.0
+    with torch.cuda.stream(stream):
+        while time.time() < t_end:
+            for _ in range(20):
+                g_step.replay()
+            torch.cuda.synchronize()
+    ms_total = timed(g_step, args.steps)
+    clk = clocks.stop()
+    ms_step = ms_total / args.steps
+
+    # dominant kernel: the GEMV, timed alone over the same launches
+    reps_g = max(3, min(args.steps, 200))
+    ms_gemv = timed(g_gemv, reps_g) / reps_g
+    per_shape = []
+    for name, n, k in synth.BITNET_2B_SHAPES:
+        Ls = [L for L in layers if L["name"] == name]
+        b = sum(L["wbytes"] + L["k"] + 4 + 4 * L["n"] for L in Ls)
+        ms = timed(shape_graphs[name], reps_g) / reps_g
+        per_shape.append(dict(shape=f"{name} {n}x{k}", launches=len(Ls), us_per_launch=round(ms * 1e3 / len(Ls), 3),
+                              gbs=round(b / (ms * 1e-3) / 1e9, 1)))
+
+    # end to end through the public API: pinned H2D of the step's activations,
+    # the captured step, D2H of the step's outputs
+    h2d = x_all_host.numel() * 2
+    d2h = y_all_host.numel() * 4
+
+    def e2e_graph_step():
+        x_all.copy_(x_all_host, non_blocking=True)
+        g_step.replay()
+        y_all_host.copy_(y_all, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            e2e_graph_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        reps_e = max(3, min(args.steps, 200))
+        e0.record(stream)
+        for _ in range(reps_e):
+            e2e_graph_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_e2e = e0.elapsed_time(e1) / reps_e
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    assert tern.device_error(stream) == tern.OK
+
+    peak, peak_kind = measured_peaks()
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    achieved = gemv_bytes / (ms_gemv * 1e-3) / 1e9
+    out = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "int8",
+        "data": "synthetic (seeded ternary weights P(-1)=P(+1)=0.3, bf16 N(0,1) activations)",
+        "config": {"workload": WORKLOAD, "layers": args.layers, "gemv_launches_per_step": len(layers),
+                   "l2": "inputs larger than L2 (packed weights per step %.1f MB vs 126 MB L2)" % (
+                       sum(L["wbytes"] for L in layers) / 1e6),
+                   "launch": "CUDA graph of the step, programmatic dependent launch between kernels",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": committed_traffic(gemv_bytes / len(layers)),
+                     "kernel": "gemv2_kernel<int8,P=1,per-tensor scale,M=1>", "peak_kind": peak_kind,
+                     "achieved_basis": "algorithmic bytes of the 210 GEMVs / their launch durations"},
+        "per_shape": per_shape,
+        "e2e": {"value": round(world * step_bytes / (ms_e2e * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * 2 * len(layers),
+        "parity_first_gemv_bit_exact": parity,
+    }
+    if clk is not None:
+        out["clocks"] = clk
+    if rank == 0 and world == 1:
+        out["cpu_baseline"] = cpu_baseline(budget_s=12.0)
+    return out
+
+
+def committed_traffic(algo_bytes_per_launch):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "gemv2_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "packed_ternary_weight_b200", "csrc", "tern_gemv2.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if d.get("source_sha256_16") != h:
+        return None
+    return d.get("dram_bytes_per_launch_scaled")
+
+
+# ---------------------------------------------------------- CPU baseline
+def cpu_baseline(budget_s: float):
+    """The oracle as it stands on a bounded sample of the same workload."""
+    import oracle
+    from packed_ternary_weight_b200 import tern
+    from threadpoolctl import threadpool_limits
+    done_bytes, t_used, gemvs = 0, 0.0, 0
+    with threadpool_limits(limits=1):
+        for lay in synth.bitnet_layer_set():
+            _, buf = tern.pack_layer(lay)
+            x = synth.draw_x_bf16(lay.seed, 1, lay.k)
+            t0 = time.perf_counter()
+            u = oracle.unpack(buf)
+            q, s = oracle.quantize_act(x)
+            oracle.gemv_bitnet_int8(u["trits"], q, s, u["tensor_scale"])
+            t_used += time.perf_counter() - t0
+            done_bytes += (len(buf) - 256) + lay.k + 4 + 4 * lay.n + 3 * lay.k + 4
+            gemvs += 1
+            if t_used > budget_s:
+                break
+    return {"value": round(done_bytes / t_used / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {gemvs} GEMVs of the layer set in layer order (unpack + quantise + exact "
+                      f"integer GEMV, numpy, one thread), {t_used:.1f} s"}
+
+
+# ------------------------------------------------------ reference arm
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: bounded samples of the workload on host cores."""
+    if rank != 0:
+        return None
+    import oracle
+    from packed_ternary_weight_b200 import tern
+    from threadpoolctl import threadpool_limits
+    threadpool_limits(limits=1)
+    total_steps = args.steps + args.warmup
+    budget = 90.0
+    lay = synth.bitnet_layer(2560, 6912, synth.bitnet_layer_set_seed(0, 6))   # down_proj of layer 0
+    _, buf = tern.pack_layer(lay)
+    x = synth.draw_x_bf16(lay.seed, 1, lay.k)
+    # rows per step so that all steps fit the budget (one 32-row tile minimum)
+    t0 = time.perf_counter()
+    u = oracle.unpack(buf)
+    q, s = oracle.quantize_act(x)
+    oracle.gemv_bitnet_int8(u["trits"], q, s, u["tensor_scale"])
+    full = time.perf_counter() - t0
+    frac = min(1.0, budget / total_steps / full)
+    rows = max(32, int(lay.n * frac) // 32 * 32)
+    tiles = rows // 32
+    hdr = oracle.parse_header(buf)
+    cols = hdr["cols"]
+    tile_bytes = cols * 512
+    sub = np.concatenate([buf[:256], buf[256:256 + tiles * tile_bytes]])
+    hd = sub[:256].copy().view("<u4")
+    hd[3] = rows                     # N of the sub-buffer (whole row tiles)
+    hd[8] = tiles
+    sub[:256] = hd.view(np.uint8)
+    sub[48:56] = np.frombuffer(np.uint64(tiles * tile_bytes).tobytes(), np.uint8)
+    sub[56:64] = np.frombuffer(np.uint64(256 + tiles * tile_bytes).tobytes(), np.uint8)
+    step_bytes = tiles * tile_bytes + lay.k + 4 + 4 * rows + 3 * lay.k + 4
+
+    def one():
+        uu = oracle.unpack(sub)
+        qq, ss = oracle.quantize_act(x)
+        oracle.gemv_bitnet_int8(uu["trits"], qq, ss, uu["tensor_scale"])
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    dt = time.perf_counter() - t0
+    v = step_bytes * args.steps / dt / 1e9
+    sample = f"{rows} of 2560 rows of down_proj 2560x6912 per step (unpack + quantise + exact integer GEMV, numpy, 1 thread)"
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "reference": "CPU oracle"},
+            "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    out = run_reference(args, rank, world) if args.impl == "reference" else run_ours(args, rank, world)
+    if rank == 0 and out is not None:
+        print(json.dumps(out))
+    if world > 1 and args.impl == "ours":
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

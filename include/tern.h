@@ -1,0 +1,163 @@
+/*
+ * tern.h -- C ABI of the packed ternary-weight GEMV library (libtern.so).
+ *
+ * The library computes, for a weight matrix W of N rows (outputs) by K
+ * columns (inputs) stored as packed trit planes t in {-1, 0, +1},
+ *
+ *     y[m][n] = sum_p sum_groups s[p][n][grp] * sum_{k in grp} t[p][n][k] * x[m][k]
+ *
+ * in three weight formats:
+ *   TERN_FMT_BITNET  one plane, 2 bits per weight, 4 weights per byte, one
+ *                    per-tensor scale applied once at the end ("Ternary GEMV
+ *                    (No Multiplication)", QORA-LLM-2B model page);
+ *   TERN_FMT_TQ      K additive trit planes ("TQ{K}P"), one fp16 scale per
+ *                    plane per group of g weights along the input dimension
+ *                    (sasori README, "K and g - the quality dials" and
+ *                    "How it works");
+ *   TERN_FMT_BT3     balanced ternary of depth 3 (27 levels): weight =
+ *                    cb[idx] * (9 t2 + 3 t1 + t0), trits base-3 packed five
+ *                    per byte, group 16, 27-entry log-spaced scale codebook
+ *                    with the index stored as three trits (Entrit
+ *                    Llama-3.1-8B-trit-uniform-d3 card, "Quantization details").
+ *
+ * Conventions for every call:
+ *   - All pointers named d_* are device pointers; the others are host
+ *     pointers. The caller owns every buffer; the library allocates no memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Device work is enqueued asynchronously on it.
+ *   - Argument errors are detected on the host and returned before anything
+ *     is enqueued. A launch failure returns TERN_ECUDA.
+ *   - Device-side failures (a bounded wait that expired inside a kernel) are
+ *     recorded in a device error word; tern_device_error() reads and clears it.
+ *   - Activations and outputs are row-major [M][K] and [M][N]. bf16 values
+ *     are passed as their 16-bit patterns.
+ *
+ * The packed buffer layout is fixed by tern_pack(); it is documented in the
+ * repository's design notes and decoded independently by the test oracle.
+ */
+#ifndef TERN_H_
+#define TERN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TERN_ABI_VERSION 1
+
+typedef enum {
+  TERN_OK = 0,
+  TERN_EINVAL = 1,       /* bad argument: NULL pointer, size, unsupported value */
+  TERN_EFORMAT = 2,      /* bad data: a trit outside {-1,0,1}, an index above 26,
+                            a non-finite scale, or a packed header that does not
+                            match the descriptor */
+  TERN_EALIGN = 3,       /* a device pointer is not 16-byte aligned */
+  TERN_ENOSPACE = 4,     /* output buffer or workspace smaller than required */
+  TERN_EUNSUPPORTED = 5, /* valid request this build has no kernel for */
+  TERN_ECUDA = 6,        /* a CUDA runtime call failed */
+  TERN_ETIMEOUT = 7      /* a bounded wait inside a kernel expired */
+} tern_status;
+
+typedef enum { TERN_FMT_BITNET = 1, TERN_FMT_TQ = 2, TERN_FMT_BT3 = 3 } tern_format;
+
+/* TERN_ACT_INT8: x is int8 [M][K] with one fp32 scale per token (x = xq * sx);
+ *   the sums are exact integers and y is fp32, bit-identical to the oracle.
+ * TERN_ACT_BF16: x is bf16 [M][K]; y is accurate to fp32 accumulation. */
+typedef enum { TERN_ACT_INT8 = 1, TERN_ACT_BF16 = 2 } tern_act;
+typedef enum { TERN_OUT_F32 = 1, TERN_OUT_BF16 = 2 } tern_out;
+
+/* Descriptor flags. */
+#define TERN_F_PDL 1u /* launch with programmatic dependent launch: the kernel may
+                         read the packed weights before the preceding kernel on
+                         the stream has finished (it still waits for that kernel
+                         before it reads x or writes y or the workspace). Set it
+                         only when no preceding kernel writes the packed buffer. */
+
+typedef struct tern_desc {
+  int32_t fmt;          /* tern_format */
+  int32_t n;            /* output rows N >= 1 */
+  int32_t k;            /* input columns K >= 1 */
+  int32_t planes;       /* BITNET: 1; TQ: 1..4; BT3: 3 (the depth) */
+  int32_t group;        /* BITNET: ignored (whole row); TQ: g, a multiple of 16
+                           in {16,32,64,128,256} dividing K; BT3: 16 */
+  float tensor_scale;   /* BITNET: the per-tensor scale s_w; else ignored */
+  uint32_t flags;       /* TERN_F_* */
+} tern_desc;
+
+/* Human-readable name of a status code (static string). */
+const char* tern_status_string(tern_status s);
+
+/* Size in bytes of the packed buffer for `desc` (256-byte header + streams). */
+tern_status tern_packed_size(const tern_desc* desc, size_t* bytes);
+
+/*
+ * Pack logical weights into the library's layout (host only, no device work).
+ *   trits       int8 [planes][N][K], values -1, 0, +1 (TERN_EFORMAT otherwise).
+ *               BT3: plane p holds t_p, the trit of weight 3^p.
+ *   scales_fp16 TQ: fp16 bit patterns [planes][N][K/group], finite; else NULL.
+ *   scale_idx   BT3: uint8 [N][K/16], values 0..26 (codebook index); else NULL.
+ *   codebook    BT3: float [27], finite; stored in the header; else NULL.
+ *   out         host buffer of out_cap bytes (TERN_ENOSPACE if too small);
+ *               *out_used receives the packed size.
+ * TQ scales are also checked against the exactness bound of the int8 path
+ * (the exact group-scaled sum must fit in 62 bits; TERN_EFORMAT otherwise).
+ */
+tern_status tern_pack(const tern_desc* desc, const int8_t* trits, const uint16_t* scales_fp16,
+                      const uint8_t* scale_idx, const float* codebook, void* out, size_t out_cap,
+                      size_t* out_used);
+
+/*
+ * Workspace needed by tern_gemv / tern_gemm_batched for `m` tokens (may be 0).
+ * The workspace must be zero-filled before its first use; every call leaves
+ * it zero-filled again. Calls that may run at the same time need separate
+ * workspaces.
+ */
+tern_status tern_workspace_size(const tern_desc* desc, int32_t m, size_t* bytes);
+
+/*
+ * Per-token absmax int8 quantisation of bf16 activations (a reading of the
+ * single-GEMV workload's "per-token absmax"; the pages give no rounding rule):
+ *   a = max |x|, inv = fl32(127 / a), xq = clamp(rint(fl32(x * inv)), -127, 127)
+ *   (round half to even), sx = fl32(a / 127); an all-zero token gives xq = 0, sx = 0.
+ *   d_x_bf16 [m][k] bf16 bits; d_xq int8 [m][k]; d_xscale float [m].
+ */
+tern_status tern_quantize_act(const uint16_t* d_x_bf16, int32_t m, int32_t k, int8_t* d_xq,
+                              float* d_xscale, void* stream);
+
+/*
+ * y = W x for one token (M = 1); same as tern_gemm_batched with m = 1.
+ *   d_packed  the bytes produced by tern_pack, copied to the device,
+ *             16-byte aligned.
+ *   act       TERN_ACT_INT8: d_x int8 [K], d_xscale float [1];
+ *             TERN_ACT_BF16: d_x bf16 [K], d_xscale NULL.
+ *   out       TERN_OUT_F32 (float [N]) or TERN_OUT_BF16 (bf16 bits [N]).
+ *   d_ws      workspace of ws_bytes (see tern_workspace_size); NULL with
+ *             ws_bytes 0 runs without splitting K across blocks.
+ */
+tern_status tern_gemv(const tern_desc* desc, const void* d_packed, tern_act act, const void* d_x,
+                      const float* d_xscale, tern_out out, void* d_y, void* d_ws, size_t ws_bytes,
+                      void* stream);
+
+/*
+ * Y = X W^T for m tokens (m >= 1), the weights read once for all tokens.
+ *   d_x [m][K] (int8 or bf16 bits), d_xscale float [m] for TERN_ACT_INT8,
+ *   d_y [m][N]. For TERN_ACT_INT8 the result is bit-identical to the oracle.
+ */
+tern_status tern_gemm_batched(const tern_desc* desc, const void* d_packed, int32_t m, tern_act act,
+                              const void* d_x, const float* d_xscale, tern_out out, void* d_y,
+                              void* d_ws, size_t ws_bytes, void* stream);
+
+/*
+ * Read and clear the device error word (synchronises `stream`).
+ * Returns TERN_OK if no kernel reported a failure, TERN_ETIMEOUT if a bounded
+ * wait expired, TERN_ECUDA if the read failed.
+ */
+tern_status tern_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TERN_H_ */

@@ -60,13 +60,13 @@ def rng(seed: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(int(seed)))
 
 
+_TRIT_OF_DRAW = np.array([-1, -1, -1, 0, 0, 0, 0, 1, 1, 1], dtype=np.int8)
+
+
 def draw_trits(gen: np.random.Generator, shape) -> np.ndarray:
     """Trits in {-1, 0, +1} as int8 with P(-1)=P(+1)=0.3, P(0)=0.4."""
     u = gen.integers(0, 10, size=shape, dtype=np.int8)
-    t = np.zeros(shape, dtype=np.int8)
-    t[u <= 2] = -1
-    t[u >= 7] = 1
-    return t
+    return _TRIT_OF_DRAW[u]
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:

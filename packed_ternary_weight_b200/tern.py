@@ -1,0 +1,146 @@
+"""ctypes binding of libtern.so: argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels (or, for
+packing, its host C++ code). Importing this module fails loudly if the shared
+library has not been built; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtern.so")
+
+OK, EINVAL, EFORMAT, EALIGN, ENOSPACE, EUNSUPPORTED, ECUDA, ETIMEOUT = range(8)
+FMT = {"bitnet": 1, "tq": 2, "bt3": 3}
+ACT_INT8, ACT_BF16 = 1, 2
+OUT_F32, OUT_BF16 = 1, 2
+F_PDL = 1
+
+
+class TernError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"libtern.so not built ({_LIB_PATH}); run python -m packed_ternary_weight_b200.build")
+    return ctypes.CDLL(_LIB_PATH)
+
+
+lib = _load()
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("n", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("planes", ctypes.c_int32), ("group", ctypes.c_int32), ("tensor_scale", ctypes.c_float),
+                ("flags", ctypes.c_uint32)]
+
+
+_vp, _sz = ctypes.c_void_p, ctypes.c_size_t
+lib.tern_status_string.restype = ctypes.c_char_p
+lib.tern_status_string.argtypes = [ctypes.c_int]
+lib.tern_packed_size.argtypes = [ctypes.POINTER(Desc), ctypes.POINTER(_sz)]
+lib.tern_pack.argtypes = [ctypes.POINTER(Desc), _vp, _vp, _vp, _vp, _vp, _sz, ctypes.POINTER(_sz)]
+lib.tern_workspace_size.argtypes = [ctypes.POINTER(Desc), ctypes.c_int32, ctypes.POINTER(_sz)]
+lib.tern_quantize_act.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp]
+lib.tern_gemv.argtypes = [ctypes.POINTER(Desc), _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp, _vp, _sz, _vp]
+lib.tern_gemm_batched.argtypes = [ctypes.POINTER(Desc), _vp, ctypes.c_int32, ctypes.c_int, _vp, _vp, ctypes.c_int,
+                                  _vp, _vp, _sz, _vp]
+lib.tern_device_error.argtypes = [_vp]
+for _f in (lib.tern_packed_size, lib.tern_pack, lib.tern_workspace_size, lib.tern_quantize_act, lib.tern_gemv,
+           lib.tern_gemm_batched, lib.tern_device_error):
+    _f.restype = ctypes.c_int
+
+
+def status_string(code: int) -> str:
+    return lib.tern_status_string(code).decode()
+
+
+def _check(code: int, what: str):
+    if code != OK:
+        raise TernError(code, what)
+
+
+def make_desc(fmt: str, n: int, k: int, planes: int = 1, group: int = 0, tensor_scale: float = 0.0,
+              flags: int = 0) -> Desc:
+    return Desc(FMT[fmt], n, k, planes, group, tensor_scale, flags)
+
+
+def desc_of(layer, flags: int = 0) -> Desc:
+    """Descriptor of a synth.Layer (or anything with the same fields)."""
+    return make_desc(layer.fmt, layer.n, layer.k, layer.planes, layer.group, layer.tensor_scale, flags)
+
+
+def packed_size(desc: Desc) -> int:
+    out = _sz()
+    _check(lib.tern_packed_size(ctypes.byref(desc), ctypes.byref(out)), "tern_packed_size")
+    return out.value
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    if hasattr(a, "data_ptr"):
+        return ctypes.c_void_p(a.data_ptr())
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def pack(desc: Desc, trits, scales_fp16=None, scale_idx=None, codebook=None) -> np.ndarray:
+    """Pack logical weights (host numpy arrays) into a uint8 numpy buffer."""
+    t = np.ascontiguousarray(trits, dtype=np.int8)
+    s = None if scales_fp16 is None else np.ascontiguousarray(scales_fp16, dtype=np.float16).view(np.uint16)
+    i = None if scale_idx is None else np.ascontiguousarray(scale_idx, dtype=np.uint8)
+    c = None if codebook is None else np.ascontiguousarray(codebook, dtype=np.float32)
+    size = packed_size(desc)
+    out = np.empty(size, dtype=np.uint8)
+    used = _sz()
+    _check(lib.tern_pack(ctypes.byref(desc), _ptr(t), _ptr(s), _ptr(i), _ptr(c), _ptr(out), size,
+                         ctypes.byref(used)), "tern_pack")
+    return out
+
+
+def pack_layer(layer, flags: int = 0):
+    d = desc_of(layer, flags)
+    return d, pack(d, layer.trits, layer.scales, layer.idx, layer.codebook)
+
+
+def workspace_size(desc: Desc, m: int = 1) -> int:
+    out = _sz()
+    _check(lib.tern_workspace_size(ctypes.byref(desc), m, ctypes.byref(out)), "tern_workspace_size")
+    return out.value
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def quantize_act(x_bf16, xq, xscale, stream=None):
+    """x_bf16: device tensor [m][k] of bf16 (or int16/uint16 bits); xq int8 [m][k]; xscale float [m]."""
+    m, k = x_bf16.shape
+    _check(lib.tern_quantize_act(_ptr(x_bf16), m, k, _ptr(xq), _ptr(xscale), _stream(stream)), "tern_quantize_act")
+
+
+def gemm_batched(desc: Desc, packed, m: int, act: int, x, xscale, out: int, y, ws=None, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib.tern_gemm_batched(ctypes.byref(desc), _ptr(packed), m, act, _ptr(x), _ptr(xscale), out, _ptr(y),
+                                 _ptr(ws), ws_bytes, _stream(stream)), "tern_gemm_batched")
+
+
+def gemv(desc: Desc, packed, act: int, x, xscale, out: int, y, ws=None, stream=None):
+    ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib.tern_gemv(ctypes.byref(desc), _ptr(packed), act, _ptr(x), _ptr(xscale), out, _ptr(y), _ptr(ws),
+                         ws_bytes, _stream(stream)), "tern_gemv")
+
+
+def device_error(stream=None) -> int:
+    return lib.tern_device_error(_stream(stream))

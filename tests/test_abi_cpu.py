@@ -1,0 +1,204 @@
+"""Host-side checks of the C-ABI library (no device calls).
+
+* every function declared in include/tern.h is exported by libtern.so;
+* the packer writes the documented layout: its output decodes, with the
+  oracle's independent decoder, to exactly the logical inputs, and a few bytes
+  are checked against values worked out by hand from the format definition;
+* packed sizes follow the closed forms; bad inputs return the documented codes.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from packed_ternary_weight_b200 import synth
+from packed_ternary_weight_b200 import tern
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    txt = open(os.path.join(ROOT, "include", "tern.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:tern_status|const char\*)\s+(tern_\w+)\s*\(", txt, re.M)))
+
+
+def test_all_declared_symbols_exported():
+    names = header_functions()
+    assert len(names) >= 8
+    for n in names:
+        assert hasattr(tern.lib, n), n
+        assert ctypes.cast(getattr(tern.lib, n), ctypes.c_void_p).value
+
+
+def test_status_strings():
+    for c in range(8):
+        assert tern.status_string(c)
+    assert tern.status_string(0) == "ok"
+
+
+# ------------------------------------------------------------ round trips
+def roundtrip(layer):
+    d, buf = tern.pack_layer(layer)
+    u = oracle.unpack(buf)
+    assert u["n"] == layer.n and u["k"] == layer.k and u["planes"] == layer.planes
+    assert np.array_equal(u["trits"], layer.trits)
+    if layer.fmt == "tq":
+        assert np.array_equal(u["scales"].view(np.uint16), layer.scales.view(np.uint16))
+    if layer.fmt == "bt3":
+        assert np.array_equal(u["idx"], layer.idx)
+        assert np.array_equal(u["codebook"], layer.codebook)
+    if layer.fmt == "bitnet":
+        assert u["tensor_scale"] == np.float32(layer.tensor_scale)
+    return buf
+
+
+@pytest.mark.parametrize("n,k", [(1, 1), (37, 100), (32, 64), (64, 1024), (511, 130)])
+def test_roundtrip_bitnet(n, k):
+    roundtrip(synth.bitnet_layer(n, k, seed=n * 1000 + k))
+
+
+@pytest.mark.parametrize("planes", [1, 2, 3, 4])
+@pytest.mark.parametrize("group", [16, 32, 64, 128, 256])
+def test_roundtrip_tq(planes, group):
+    roundtrip(synth.tq_layer(45, 512, planes, group, seed=planes * 10 + group))
+
+
+@pytest.mark.parametrize("n,k", [(1, 16), (45, 96), (32, 160), (70, 4096)])
+def test_roundtrip_bt3(n, k):
+    roundtrip(synth.bt3_layer(n, k, seed=n + k))
+
+
+def test_no_invalid_codes_or_bytes():
+    lay = synth.tq_layer(33, 256, 3, 64, seed=5)
+    buf = roundtrip(lay)
+    h = oracle.parse_header(buf)
+    words = buf[h["trit_offset"]:h["trit_offset"] + h["trit_bytes"]]
+    codes = np.unpackbits(words[:, None], axis=1, bitorder="little").reshape(-1, 2)
+    assert not np.any(codes.all(axis=1))            # no 11 code
+    b3 = roundtrip(synth.bt3_layer(33, 160, seed=6))
+    h = oracle.parse_header(b3)
+    assert b3[h["trit_offset"]:].max() <= 242
+
+
+# --------------------------------------------------- hand-worked byte pins
+def test_bitnet_bytes_by_hand():
+    # one row, K = 64: t[5] = +1 (code 01), t[17] = -1 (code 10), t[63] = +1.
+    # trit j of word w sits at bit 8*(j%4) + 2*(j//4):
+    #   k=5  -> word 0, j=5  -> bit 10 (code 01 -> bit 10 set)
+    #   k=17 -> word 1, j=1  -> bit 8  (code 10 -> bit 9 set)
+    #   k=63 -> word 3, j=15 -> bit 30 (code 01 -> bit 30 set)
+    t = np.zeros((1, 1, 64), np.int8)
+    t[0, 0, 5], t[0, 0, 17], t[0, 0, 63] = 1, -1, 1
+    d = tern.make_desc("bitnet", 1, 64, 1, 64, 0.5)
+    buf = tern.pack(d, t)
+    assert len(buf) == 256 + 512                     # one 32-row tile, one column
+    words = buf[256:256 + 16].view("<u4")
+    assert words.tolist() == [1 << 10, 1 << 9, 0, 1 << 30]
+    assert not buf[256 + 16:].any()                  # rows 1..31 are padding
+    assert oracle.unpack(buf)["trits"].tolist() == t.tolist()
+
+
+def test_bt3_bytes_by_hand():
+    # one row, K = 16 (one group): t0[3] = +1 (digit 2), everything else 0
+    # (digit 1). Byte i holds k = 16 j + i as digit j, so byte 3 of plane 0 is
+    # 2 + 3 + 9 + 27 + 81 = 122 and every other byte is 1+3+9+27+81 = 121.
+    # The group's index 14 = 2 + 1*3 + 1*9: index byte d holds digit d of it as
+    # digit 0 and 0 (padding groups) elsewhere -> 2, 1, 1.
+    t = np.zeros((3, 1, 16), np.int8)
+    t[0, 0, 3] = 1
+    idx = np.array([[14]], np.uint8)
+    cb = synth.codebook27()
+    d = tern.make_desc("bt3", 1, 16, 3, 16)
+    buf = tern.pack(d, t, scale_idx=idx, codebook=cb)
+    assert len(buf) == 256 + 1632
+    col = buf[256:]
+    assert col[3] == 122 and col[0] == 121 and col[15] == 121
+    assert col[512] == 121 and col[1024 + 7] == 121
+    assert col[1536] == 2 and col[1536 + 32] == 1 and col[1536 + 64] == 1
+    assert np.array_equal(buf[128:128 + 108].view("<f4"), cb)
+    u = oracle.unpack(buf)
+    assert np.array_equal(u["trits"], t) and u["idx"].tolist() == [[14]]
+
+
+# ------------------------------------------------------------------ sizes
+def test_packed_size_closed_forms():
+    cases = [
+        (tern.make_desc("bitnet", 2560, 2560, 1, 2560, 0.02), 256 + 80 * 40 * 512),
+        (tern.make_desc("bitnet", 640, 2560, 1, 2560, 0.02), 256 + 20 * 40 * 512),
+        (tern.make_desc("bitnet", 2560, 6912, 1, 6912, 0.02), 256 + 80 * 108 * 512),
+        (tern.make_desc("tq", 4096, 4096, 3, 256), 256 + 128 * 64 * 3 * 512 + 128 * 16 * 3 * 64),
+        (tern.make_desc("tq", 14336, 4096, 2, 32), 256 + 448 * 64 * 2 * 512 + 448 * 128 * 2 * 64),
+        (tern.make_desc("bt3", 4096, 4096, 3, 16), 256 + 128 * 52 * 1632),
+        (tern.make_desc("bt3", 4096, 14336, 3, 16), 256 + 128 * 180 * 1632),
+    ]
+    for d, size in cases:
+        assert tern.packed_size(d) == size
+    # physical bits per weight match the pages' accounting (2K + 16K/g) exactly
+    # when the shape fills whole tiles
+    for planes, g in ((1, 256), (2, 256), (3, 256), (4, 256), (2, 64), (2, 32)):
+        d = tern.make_desc("tq", 4096, 4096, planes, g)
+        bpw = (tern.packed_size(d) - 256) * 8 / (4096 * 4096)
+        assert bpw == oracle.bits_per_weight("tq", planes, g)
+    # balanced ternary: five trits per byte -> (48 + 3) / 5 * 8 / 16 = 5.1 bits
+    # per weight when K fills whole 80-k columns (information content 5.05)
+    d = tern.make_desc("bt3", 32, 4000, 3, 16)
+    assert (tern.packed_size(d) - 256) * 8 / (32 * 4000) == pytest.approx(5.1)
+
+
+def test_c1_layer_set_total_bytes():
+    total = 0
+    for name, n, k in synth.BITNET_2B_SHAPES:
+        total += tern.packed_size(tern.make_desc("bitnet", n, k, 1, k, 0.02)) - 256
+    assert total * synth.BITNET_2B_LAYERS == 30 * (2 * 1638400 + 2 * 409600 + 3 * 4423680)
+
+
+# ------------------------------------------------------------------ errors
+def expect(code, fn):
+    with pytest.raises(tern.TernError) as ei:
+        fn()
+    assert ei.value.code == code
+
+
+def test_error_paths():
+    lay = synth.tq_layer(8, 64, 2, 32, seed=1)
+    d = tern.desc_of(lay)
+    bad = lay.trits.copy()
+    bad[1, 3, 7] = 2
+    expect(tern.EFORMAT, lambda: tern.pack(d, bad, lay.scales))
+    s = lay.scales.copy()
+    s[0, 0, 0] = np.float16(np.inf)
+    expect(tern.EFORMAT, lambda: tern.pack(d, lay.trits, s))
+    expect(tern.EINVAL, lambda: tern.pack(d, lay.trits, None))
+    expect(tern.EINVAL, lambda: tern.packed_size(tern.make_desc("tq", 8, 64, 2, 48)))
+    expect(tern.EINVAL, lambda: tern.packed_size(tern.make_desc("tq", 8, 96, 2, 64)))
+    expect(tern.EINVAL, lambda: tern.packed_size(tern.make_desc("tq", 8, 64, 5, 32)))
+    expect(tern.EINVAL, lambda: tern.packed_size(tern.make_desc("bitnet", 0, 64, 1, 64)))
+    expect(tern.EINVAL, lambda: tern.packed_size(tern.make_desc("bt3", 8, 40, 3, 16)))
+    b3 = synth.bt3_layer(8, 32, seed=2)
+    idx = b3.idx.copy()
+    idx[0, 0] = 27
+    expect(tern.EFORMAT, lambda: tern.pack(tern.desc_of(b3), b3.trits, scale_idx=idx, codebook=b3.codebook))
+    cb = b3.codebook.copy()
+    cb[4] = np.nan
+    expect(tern.EFORMAT, lambda: tern.pack(tern.desc_of(b3), b3.trits, scale_idx=b3.idx, codebook=cb))
+    # output capacity too small
+    out = np.empty(100, np.uint8)
+    used = ctypes.c_size_t()
+    t = np.ascontiguousarray(lay.trits)
+    sc = np.ascontiguousarray(lay.scales).view(np.uint16)
+    rc = tern.lib.tern_pack(ctypes.byref(d), t.ctypes.data_as(ctypes.c_void_p), sc.ctypes.data_as(ctypes.c_void_p),
+                            None, None, out.ctypes.data_as(ctypes.c_void_p), 100, ctypes.byref(used))
+    assert rc == tern.ENOSPACE and used.value == tern.packed_size(d)
+    # exactness bound of the int8 path: huge scales are refused
+    big_lay = synth.tq_layer(8, 65536, 4, 16, seed=3)
+    big = np.full_like(big_lay.scales, np.float16(60000.0))
+    expect(tern.EFORMAT, lambda: tern.pack(tern.desc_of(big_lay), big_lay.trits, big))
+
+
+def test_workspace_size_host_only():
+    d = tern.make_desc("bitnet", 640, 2560, 1, 2560, 0.02)
+    assert tern.workspace_size(d, 1) >= 0
+    assert tern.workspace_size(tern.make_desc("tq", 1024, 4096, 2, 32), 16) > 0

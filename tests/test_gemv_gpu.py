@@ -1,0 +1,211 @@
+"""GPU parity of the C-ABI kernels against the CPU oracle (B200, sm_100a).
+
+int8 activations: bit-exact. bf16 activations: the fp32 result is within
+1e-3 of the fp64 reference relative to max(|y_ref|, 1e-2 * rms(y_ref)); the
+bf16 output is exactly bf16_rn of the same kernel's fp32 result. Inputs come
+from the seeded generators; expected values from the oracle only.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from packed_ternary_weight_b200 import synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+BF16_TOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def tern():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from packed_ternary_weight_b200 import tern as t
+    return t
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def x_dev(xbits):
+    return dev(np.ascontiguousarray(xbits).view(np.int16))
+
+
+def run_int8(tern, layer, xbits, use_ws=True, out=1, pdl=False):
+    """Quantise x on the GPU, run the GEMV/batched GEMV; returns (y, xq, sx)."""
+    d, buf = tern.pack_layer(layer, flags=tern.F_PDL if pdl else 0)
+    m, k = xbits.shape
+    pk = dev(buf)
+    xd = x_dev(xbits)
+    xq = torch.empty((m, k), dtype=torch.int8, device="cuda")
+    sx = torch.empty((m,), dtype=torch.float32, device="cuda")
+    tern.quantize_act(xd, xq, sx)
+    y = torch.empty((m, layer.n), dtype=torch.float32 if out == tern.OUT_F32 else torch.int16, device="cuda")
+    ws = None
+    if use_ws:
+        ws = torch.zeros(max(16, tern.workspace_size(d, m)), dtype=torch.uint8, device="cuda")
+    tern.gemm_batched(d, pk, m, tern.ACT_INT8, xq, sx, out, y, ws)
+    torch.cuda.synchronize()
+    if ws is not None:
+        assert not ws.any().item(), "workspace must be left zero-filled"
+    assert tern.device_error() == tern.OK
+    return y.cpu().numpy(), xq.cpu().numpy(), sx.cpu().numpy()
+
+
+def run_bf16(tern, layer, xbits, out, use_ws=True):
+    d, buf = tern.pack_layer(layer)
+    pk = dev(buf)
+    xd = x_dev(xbits)
+    m = xbits.shape[0]
+    y = torch.empty((m, layer.n), dtype=torch.float32 if out == tern.OUT_F32 else torch.int16, device="cuda")
+    ws = torch.zeros(max(16, tern.workspace_size(d, m)), dtype=torch.uint8, device="cuda") if use_ws else None
+    tern.gemm_batched(d, pk, m, tern.ACT_BF16, xd, None, out, y, ws)
+    torch.cuda.synchronize()
+    assert tern.device_error() == tern.OK
+    return y.cpu().numpy()
+
+
+def check_bf16(y32, yref):
+    floor = 1e-2 * np.sqrt(np.mean(yref ** 2))
+    err = np.abs(y32.astype(np.float64) - yref) / np.maximum(np.abs(yref), floor)
+    assert err.max() <= BF16_TOL, f"max rel err {err.max():.3g}"
+    return err.max()
+
+
+# ---------------------------------------------------------------- quantiser
+@pytest.mark.parametrize("m,k", [(1, 1024), (3, 2560), (5, 6912), (2, 7)])
+def test_quantize_bit_exact(tern, m, k):
+    x = synth.draw_x_bf16(77 + k, m, k)
+    if m >= 3:
+        x[1] = 0                                    # all-zero token
+        x[2, :4] = synth.f32_to_bf16_bits(np.array([2.0, 1.0, -1.0, 0.5], np.float32))
+        x[2, 4:] = 0                                # exact .5 ties after scaling
+    xd = x_dev(x)
+    xq = torch.empty((m, k), dtype=torch.int8, device="cuda")
+    sx = torch.empty((m,), dtype=torch.float32, device="cuda")
+    tern.quantize_act(xd, xq, sx)
+    q_ref, s_ref = oracle.quantize_act(x)
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+
+
+# ---------------------------------------------------------- BitNet int8 path
+def bitnet_check(tern, layer, m=1, **kw):
+    x = synth.draw_x_bf16(layer.seed, m, layer.k)
+    y, xq, sx = run_int8(tern, layer, x, **kw)
+    q_ref, s_ref = oracle.quantize_act(x)
+    assert np.array_equal(xq, q_ref) and np.array_equal(sx, s_ref)
+    y_ref = oracle.gemv_bitnet_int8(layer.trits, q_ref, s_ref, layer.tensor_scale)
+    assert np.array_equal(y.view(np.uint32), y_ref.view(np.uint32)), \
+        f"mismatch at {np.argwhere(y != y_ref)[:5]}"
+
+
+def test_single_gemv_512x1024_bit_exact(tern):
+    bitnet_check(tern, synth.single_gemv_layer())
+    bitnet_check(tern, synth.single_gemv_layer(), use_ws=False)
+
+
+@pytest.mark.parametrize("shape", synth.BITNET_2B_SHAPES, ids=[s[0] for s in synth.BITNET_2B_SHAPES])
+def test_bitnet_2b_layer_shapes_bit_exact(tern, shape):
+    name, n, k = shape
+    layer = synth.bitnet_layer(n, k, synth.bitnet_layer_set_seed(0, [s[0] for s in synth.BITNET_2B_SHAPES].index(name)))
+    bitnet_check(tern, layer)
+    bitnet_check(tern, layer, pdl=True)
+
+
+@pytest.mark.parametrize("n,k", [(1, 1), (37, 100), (33, 64), (300, 1000), (31, 6912), (4097, 129)])
+def test_bitnet_ragged_shapes(tern, n, k):
+    lay = synth.bitnet_layer(n, k, seed=n * 7 + k)
+    bitnet_check(tern, lay)
+    bitnet_check(tern, lay, use_ws=False)
+
+
+@pytest.mark.parametrize("m", [2, 4, 5, 16, 21])
+def test_bitnet_batched_bit_exact(tern, m):
+    bitnet_check(tern, synth.bitnet_layer(640, 2560, seed=9), m=m)
+
+
+def test_bitnet_zero_activation(tern):
+    lay = synth.bitnet_layer(96, 256, seed=4)
+    x = np.zeros((1, 256), np.uint16)
+    y, _, _ = run_int8(tern, lay, x)
+    assert not y.any() and not np.signbit(y).any()
+
+
+def test_bitnet_deterministic(tern):
+    lay = synth.bitnet_layer(2560, 6912, seed=12)
+    x = synth.draw_x_bf16(12, 1, 6912)
+    y1, _, _ = run_int8(tern, lay, x)
+    y2, _, _ = run_int8(tern, lay, x)
+    assert np.array_equal(y1.view(np.uint32), y2.view(np.uint32))
+
+
+# ------------------------------------------------------------- TQ int8 path
+def tq_int8_check(tern, layer, m, rows=None):
+    x = synth.draw_x_bf16(layer.seed, m, layer.k)
+    y, xq, sx = run_int8(tern, layer, x)
+    q_ref, s_ref = oracle.quantize_act(x)
+    assert np.array_equal(xq, q_ref)
+    r = slice(None) if rows is None else rows
+    y_ref = oracle.gemv_tq_int8(layer.trits[:, r], layer.scales[:, r], layer.group, q_ref, s_ref)
+    assert np.array_equal(y[:, r].view(np.uint32), y_ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("m", [1, 4, 16, 3])
+def test_tq2p_g32_int8_bit_exact(tern, m):
+    tq_int8_check(tern, synth.tq_layer(300, 1024, 2, 32, seed=40 + m), m)
+
+
+@pytest.mark.parametrize("shape", synth.PREFILL_SHAPES, ids=[s[0] for s in synth.PREFILL_SHAPES])
+@pytest.mark.parametrize("m", [1, 4])
+def test_tq2p_prefill_shapes_gemv_bit_exact(tern, shape, m):
+    name, n, k = shape
+    lay = synth.tq_layer(n, k, 2, 32, seed=400 + [s[0] for s in synth.PREFILL_SHAPES].index(name))
+    rows = np.sort(np.random.default_rng(0).choice(n, 512, replace=False))
+    tq_int8_check(tern, lay, m, rows=rows)
+
+
+def test_tq3p_g256_int8_bit_exact(tern):
+    tq_int8_check(tern, synth.tq_layer(1024, 4096, 3, 256, seed=7), 1)
+
+
+# ------------------------------------------------------------- TQ bf16 path
+def tq_bf16_check(tern, layer, rows=None, use_ws=True):
+    x = synth.draw_x_bf16(layer.seed, 1, layer.k)
+    y32 = run_bf16(tern, layer, x, tern.OUT_F32, use_ws)
+    y16 = run_bf16(tern, layer, x, tern.OUT_BF16, use_ws)
+    r = slice(None) if rows is None else rows
+    w = oracle.dequantize("tq", layer.trits[:, r], layer.group, scales=layer.scales[:, r])
+    yref = oracle.gemv_bf16(w, x)[0]
+    err = check_bf16(y32[0, r], yref)
+    # bf16 output = round-to-nearest-even of the fp32 result of the same kernel
+    assert np.array_equal(y16.view(np.uint16), synth.f32_to_bf16_bits(y32))
+    return err
+
+
+@pytest.mark.parametrize("shape", synth.LLAMA_8B_SHAPES, ids=[s[0] for s in synth.LLAMA_8B_SHAPES])
+def test_tq3p_llama_shapes_bf16(tern, shape):
+    name, n, k = shape
+    lay = synth.tq_layer(n, k, 3, 256, seed=200 + [s[0] for s in synth.LLAMA_8B_SHAPES].index(name))
+    rows = np.sort(np.random.default_rng(1).choice(n, min(n, 384), replace=False))
+    tq_bf16_check(tern, lay, rows=rows)
+
+
+@pytest.mark.parametrize("planes,group", [(1, 256), (2, 256), (4, 256), (2, 32), (3, 64)])
+def test_tq_bf16_variants(tern, planes, group):
+    lay = synth.tq_layer(200, 1024, planes, group, seed=planes * 100 + group)
+    tq_bf16_check(tern, lay)
+    tq_bf16_check(tern, lay, use_ws=False)
+
+
+def test_tq_bf16_wide_dynamic_range(tern):
+    lay = synth.tq_layer(64, 512, 3, 256, seed=3)
+    x = synth.draw_x_bf16(3, 1, 512).copy()
+    xf = synth.bf16_bits_to_f32(x)
+    xf[0, :256] *= 1e-3                    # one group much smaller than the other
+    xf[0, 300] = 40.0                      # one outlier
+    x = synth.f32_to_bf16_bits(xf)
+    y32 = run_bf16(tern, lay, x, tern.OUT_F32)
+    yref = oracle.gemv_bf16(oracle.dequantize("tq", lay.trits, 256, scales=lay.scales), x)[0]
+    check_bf16(y32[0], yref)
