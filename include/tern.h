@@ -64,7 +64,9 @@ typedef enum { TERN_FMT_BITNET = 1, TERN_FMT_TQ = 2, TERN_FMT_BT3 = 3 } tern_for
 
 /* TERN_ACT_INT8: x is int8 [M][K] with one fp32 scale per token (x = xq * sx);
  *   the sums are exact integers and y is fp32, bit-identical to the oracle.
- * TERN_ACT_BF16: x is bf16 [M][K]; y is accurate to fp32 accumulation. */
+ * TERN_ACT_BF16: x is bf16 [M][K]; y is accurate to fp32 accumulation (each
+ *   group's sum is exact for every activation within 2^15 of the group's
+ *   largest, then rounded once to fp32 and accumulated in fp32). */
 typedef enum { TERN_ACT_INT8 = 1, TERN_ACT_BF16 = 2 } tern_act;
 typedef enum { TERN_OUT_F32 = 1, TERN_OUT_BF16 = 2 } tern_out;
 
@@ -110,9 +112,10 @@ tern_status tern_pack(const tern_desc* desc, const int8_t* trits, const uint16_t
 
 /*
  * Workspace needed by tern_gemv / tern_gemm_batched for `m` tokens (may be 0).
- * The workspace must be zero-filled before its first use; every call leaves
- * it zero-filled again. Calls that may run at the same time need separate
- * workspaces.
+ * The workspace holds per-block arrival counters and split partial sums. It
+ * must be zero-filled before its first use; every call resets the counters
+ * to zero, so the workspace can be reused by later calls without clearing.
+ * Calls that may run at the same time need separate workspaces.
  */
 tern_status tern_workspace_size(const tern_desc* desc, int32_t m, size_t* bytes);
 

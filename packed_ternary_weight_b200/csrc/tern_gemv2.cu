@@ -27,12 +27,12 @@
 //    GEMV (No Multiplication)"); TQ folds each fp16 group scale into an exact
 //    int64 count of 2^-24 (every fp16 value is an integer multiple of 2^-24),
 //    so the result is the exactly rounded group-scaled sum in any order.
-//  * bf16: each group of x is written exactly as q * 2^(E-14) with q a 16-bit
-//    integer (E = exponent of the group's largest |x|; bf16 carries 8
-//    significant bits, so every element within 2^7 of the group maximum is
-//    exact and smaller ones round by at most 2^(E-15)), split into a signed
-//    high byte and an unsigned low byte; integer group sums are exact and are
-//    scaled and accumulated once per group in fp32.
+//  * bf16: each group of x is written as q * 2^(E-22) with q a 24-bit integer
+//    (E = exponent of the group's largest |x|; bf16 carries 8 significant
+//    bits, so every element within 2^15 of the group maximum is exact and
+//    smaller ones round by at most 2^(E-23)), split into a signed high byte and
+//    unsigned middle and low bytes; integer group sums are exact, and each is
+//    rounded once to fp32, scaled and accumulated once per group in fp32.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -49,7 +49,7 @@ constexpr uint32_t kM03 = 0x03030303u;
 constexpr uint32_t kM30 = 0x30303030u;
 
 struct SmemPlan {
-  size_t bars, ring, xa, xb, gsum, gmult, flag, total;
+  size_t bars, ring, xa, xb, xc, gsum, gmult, flag, total;
   int stage_bytes;
 };
 
@@ -69,13 +69,15 @@ __host__ __device__ inline SmemPlan smem_plan(const Gemv2Params& p, int xmode, i
   off = align_up(off + (size_t)p.wpc * p.nstage * 8, 128);
   s.ring = off;
   off += (size_t)p.wpc * p.nstage * s.stage_bytes;
-  s.xa = off;  // int8 x [mt][kr] or bf16 high bytes [kr]
+  s.xa = off;  // int8 x [mt][kr], or the signed high byte of the bf16 image [kr]
   off = align_up(off + (size_t)(xmode == kXInt8 ? mt : 1) * kr, 128);
-  s.xb = off;  // bf16 low bytes [kr]
+  s.xb = off;  // bf16 image: middle byte [kr]
   off = align_up(off + (xmode == kXBf16 ? (size_t)kr : 0), 128);
-  s.gsum = off;  // int32 [mt][gr]: sum x (int8) or sum q (bf16)
-  off = align_up(off + (size_t)mt * gr * 4, 16);
-  s.gmult = off;  // float [gr]: 2^(E-14) (bf16)
+  s.xc = off;  // bf16 image: low byte [kr]
+  off = align_up(off + (xmode == kXBf16 ? (size_t)kr : 0), 128);
+  s.gsum = off;  // int32 [mt][gr]: sum x (int8); int64 [gr]: sum q (bf16)
+  off = align_up(off + (size_t)mt * gr * (xmode == kXBf16 ? 8 : 4), 16);
+  s.gmult = off;  // float [gr]: 2^(E-22) (bf16)
   off = align_up(off + (xmode == kXBf16 ? (size_t)gr * 4 : 0), 16);
   s.flag = off;
   off += 16;
@@ -110,8 +112,9 @@ __device__ void stage_x_int8(const Gemv2Params& p, const SmemPlan& sp, uint8_t* 
 
 __device__ void stage_x_bf16(const Gemv2Params& p, const SmemPlan& sp, uint8_t* smem, int k0, int kr) {
   int8_t* xh = reinterpret_cast<int8_t*>(smem + sp.xa);
-  uint8_t* xl = smem + sp.xb;
-  int* gs = reinterpret_cast<int*>(smem + sp.gsum);
+  uint8_t* xm = smem + sp.xb;
+  uint8_t* xl = smem + sp.xc;
+  long long* gs = reinterpret_cast<long long*>(smem + sp.gsum);
   float* gm = reinterpret_cast<float*>(smem + sp.gmult);
   const uint16_t* x = static_cast<const uint16_t*>(p.x);
   const int g = p.group, gr = kr / g;
@@ -127,23 +130,24 @@ __device__ void stage_x_bf16(const Gemv2Params& p, const SmemPlan& sp, uint8_t* 
 #pragma unroll
     for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const int e = amax > 0.f ? ilogbf(amax) : 0;
-    // multiply by 2^(14-e) in at most two exact power-of-two steps
-    const int sh = 14 - e;
+    // multiply by 2^(22-e) in at most two exact power-of-two steps
+    const int sh = 22 - e;
     const float up1 = ldexpf(1.0f, sh > 100 ? 100 : sh), up2 = ldexpf(1.0f, sh > 100 ? sh - 100 : 0);
-    int s = 0;
+    long long s = 0;
     for (int kk = kb + lane; kk < kb + g; kk += 32) {
       const int k = k0 + kk;
       const float v = k < p.k ? __uint_as_float((uint32_t)x[k] << 16) : 0.f;
-      const int q = __float2int_rn(__fmul_rn(__fmul_rn(v, up1), up2));  // |q| < 2^15
+      const int q = __float2int_rn(__fmul_rn(__fmul_rn(v, up1), up2));  // |q| < 2^23
       s += q;
-      xh[kk] = (int8_t)(q >> 8);
+      xh[kk] = (int8_t)(q >> 16);
+      xm[kk] = (uint8_t)((q >> 8) & 0xFF);
       xl[kk] = (uint8_t)(q & 0xFF);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if (lane == 0) {
       gs[grp] = s;
-      gm[grp] = amax > 0.f ? ldexpf(1.0f, e - 14) : 0.f;
+      gm[grp] = amax > 0.f ? ldexpf(1.0f, e - 22) : 0.f;
     }
   }
 }
@@ -220,14 +224,17 @@ __global__ void __launch_bounds__(256) gemv2_kernel(const Gemv2Params p) {
   __syncthreads();
 
   const int8_t* xs = reinterpret_cast<const int8_t*>(smem + sp.xa);
-  const uint8_t* xl = smem + sp.xb;
+  const uint8_t* xmid = smem + sp.xb;
+  const uint8_t* xl = smem + sp.xc;
   const int* gsum = reinterpret_cast<const int*>(smem + sp.gsum);
+  const long long* gsum64 = reinterpret_cast<const long long*>(smem + sp.gsum);
   const float* gmul = reinterpret_cast<const float*>(smem + sp.gmult);
   const int gr = kTQ ? kr / p.group : 1;
   const int m = p.m;
 
   // accumulators: a = fields 0,1 (weight 1), b = fields 2,3 (weight 16)
   int a[P][MT], b[P][MT];     // int8 x   (or high bytes for bf16)
+  unsigned ma[P], mb[P];      // bf16 middle bytes
   unsigned la[P], lb[P];      // bf16 low bytes
   long long acc64[MT];        // TQ int8
   float yacc = 0.f;           // bf16
@@ -235,7 +242,7 @@ __global__ void __launch_bounds__(256) gemv2_kernel(const Gemv2Params p) {
   for (int q = 0; q < P; ++q) {
 #pragma unroll
     for (int t = 0; t < MT; ++t) a[q][t] = b[q][t] = 0;
-    la[q] = lb[q] = 0;
+    la[q] = lb[q] = ma[q] = mb[q] = 0;
   }
 #pragma unroll
   for (int t = 0; t < MT; ++t) acc64[t] = 0;
@@ -285,6 +292,7 @@ __global__ void __launch_bounds__(256) gemv2_kernel(const Gemv2Params p) {
             }
           } else {
             const int4 hv = *reinterpret_cast<const int4*>(xs + kx + wi * 16);
+            const uint4 mv = *reinterpret_cast<const uint4*>(xmid + kx + wi * 16);
             const uint4 lv = *reinterpret_cast<const uint4*>(xl + kx + wi * 16);
 #pragma unroll
             for (int q = 0; q < P; ++q) {
@@ -292,6 +300,10 @@ __global__ void __launch_bounds__(256) gemv2_kernel(const Gemv2Params p) {
               a[q][0] = dp4a_ss((int)(F2[q] & kM03), hv.y, a[q][0]);
               b[q][0] = dp4a_ss((int)(F[q] & kM30), hv.z, b[q][0]);
               b[q][0] = dp4a_ss((int)(F2[q] & kM30), hv.w, b[q][0]);
+              ma[q] = dp4a_uu(F[q] & kM03, mv.x, ma[q]);
+              ma[q] = dp4a_uu(F2[q] & kM03, mv.y, ma[q]);
+              mb[q] = dp4a_uu(F[q] & kM30, mv.z, mb[q]);
+              mb[q] = dp4a_uu(F2[q] & kM30, mv.w, mb[q]);
               la[q] = dp4a_uu(F[q] & kM03, lv.x, la[q]);
               la[q] = dp4a_uu(F2[q] & kM03, lv.y, la[q]);
               lb[q] = dp4a_uu(F[q] & kM30, lv.z, lb[q]);
@@ -318,11 +330,12 @@ __global__ void __launch_bounds__(256) gemv2_kernel(const Gemv2Params p) {
                   }
                 } else {
                   const int H = a[q][0] + (b[q][0] >> 4);
+                  const int Mi = (int)(ma[q] + (mb[q] >> 4));
                   const int L = (int)(la[q] + (lb[q] >> 4));
-                  const int S = gsum[gl] - (H * 256 + L);
-                  yacc = fmaf(__half2float(__ushort_as_half(h)) * gmul[gl], (float)S, yacc);
+                  const long long S = gsum64[gl] - ((long long)H * 65536 + (long long)Mi * 256 + L);
+                  yacc = fmaf(__half2float(__ushort_as_half(h)) * gmul[gl], __ll2float_rn(S), yacc);
                   a[q][0] = b[q][0] = 0;
-                  la[q] = lb[q] = 0;
+                  la[q] = lb[q] = ma[q] = mb[q] = 0;
                 }
               }
             }

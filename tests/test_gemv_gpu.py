@@ -47,10 +47,15 @@ def run_int8(tern, layer, xbits, use_ws=True, out=1, pdl=False):
         ws = torch.zeros(max(16, tern.workspace_size(d, m)), dtype=torch.uint8, device="cuda")
     tern.gemm_batched(d, pk, m, tern.ACT_INT8, xq, sx, out, y, ws)
     torch.cuda.synchronize()
+    y1 = y.cpu().numpy()
     if ws is not None:
-        assert not ws.any().item(), "workspace must be left zero-filled"
+        # the same workspace again: its arrival counters must have been reset
+        y.fill_(0)
+        tern.gemm_batched(d, pk, m, tern.ACT_INT8, xq, sx, out, y, ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(y.cpu().numpy().view(np.uint32), y1.view(np.uint32))
     assert tern.device_error() == tern.OK
-    return y.cpu().numpy(), xq.cpu().numpy(), sx.cpu().numpy()
+    return y1, xq.cpu().numpy(), sx.cpu().numpy()
 
 
 def run_bf16(tern, layer, xbits, out, use_ws=True):
