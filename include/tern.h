@@ -153,6 +153,26 @@ tern_status tern_gemm_batched(const tern_desc* desc, const void* d_packed, int32
                               void* d_ws, size_t ws_bytes, void* stream);
 
 /*
+ * tern_gemv without a caller-provided workspace, for callers that cannot
+ * allocate device memory (code running where cudaMalloc is not permitted, or
+ * inside a framework that owns every device allocation). The paper has no
+ * counterpart; this is a deployment convenience of this library.
+ *   Arguments as tern_gemv (one token), minus d_ws / ws_bytes.
+ *   Scratch: a fixed 1 MiB array in device memory owned by the library; every
+ *   GPU that loads the library holds it until the process exits. A layer whose
+ *   workspace (tern_workspace_size with m = 1) exceeds 1 MiB is rejected with
+ *   TERN_ENOSPACE before anything is enqueued.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any stream
+ *   capture. Each call clears the part of the scratch it uses on `stream`
+ *   (cudaMemsetAsync) and never allocates or frees memory.
+ *   All calls on a device share the same scratch: calls that may overlap on
+ *   the GPU (different streams without ordering between them) race.
+ */
+tern_status tern_gemv_noalloc(const tern_desc* desc, const void* d_packed, tern_act act, const void* d_x,
+                              const float* d_xscale, tern_out out, void* d_y, void* stream);
+
+/*
  * Read and clear the device error word (synchronises `stream`).
  * Returns TERN_OK if no kernel reported a failure, TERN_ETIMEOUT if a bounded
  * wait expired, TERN_ECUDA if the read failed.

@@ -52,8 +52,9 @@ lib.tern_gemv.argtypes = [ctypes.POINTER(Desc), _vp, ctypes.c_int, _vp, _vp, cty
 lib.tern_gemm_batched.argtypes = [ctypes.POINTER(Desc), _vp, ctypes.c_int32, ctypes.c_int, _vp, _vp, ctypes.c_int,
                                   _vp, _vp, _sz, _vp]
 lib.tern_device_error.argtypes = [_vp]
+lib.tern_gemv_noalloc.argtypes = [ctypes.POINTER(Desc), _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp, _vp]
 for _f in (lib.tern_packed_size, lib.tern_pack, lib.tern_workspace_size, lib.tern_quantize_act, lib.tern_gemv,
-           lib.tern_gemm_batched, lib.tern_device_error):
+           lib.tern_gemm_batched, lib.tern_device_error, lib.tern_gemv_noalloc):
     _f.restype = ctypes.c_int
 
 
@@ -140,6 +141,12 @@ def gemv(desc: Desc, packed, act: int, x, xscale, out: int, y, ws=None, stream=N
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib.tern_gemv(ctypes.byref(desc), _ptr(packed), act, _ptr(x), _ptr(xscale), out, _ptr(y), _ptr(ws),
                          ws_bytes, _stream(stream)), "tern_gemv")
+
+
+def gemv_noalloc(desc: Desc, packed, act: int, x, xscale, out: int, y, stream=None):
+    """tern_gemv with the library's fixed device scratch instead of a caller workspace."""
+    _check(lib.tern_gemv_noalloc(ctypes.byref(desc), _ptr(packed), act, _ptr(x), _ptr(xscale), out, _ptr(y),
+                                 _stream(stream)), "tern_gemv_noalloc")
 
 
 def device_error(stream=None) -> int:
