@@ -66,8 +66,12 @@ typedef enum { TERN_FMT_BITNET = 1, TERN_FMT_TQ = 2, TERN_FMT_BT3 = 3 } tern_for
  *   the sums are exact integers and y is fp32, bit-identical to the oracle.
  * TERN_ACT_BF16: x is bf16 [M][K]; y is accurate to fp32 accumulation (each
  *   group's sum is exact for every activation within 2^15 of the group's
- *   largest, then rounded once to fp32 and accumulated in fp32). */
-typedef enum { TERN_ACT_INT8 = 1, TERN_ACT_BF16 = 2 } tern_act;
+ *   largest, then rounded once to fp32 and accumulated in fp32).
+ * TERN_ACT_BF16_Q8: x is bf16 [M][K]; each token is quantised to int8 inside
+ *   the GEMV by the rule of tern_quantize_act, then the int8 path runs; the
+ *   result is bit-identical to tern_quantize_act followed by TERN_ACT_INT8
+ *   (d_xscale is ignored). BITNET and TQ only. */
+typedef enum { TERN_ACT_INT8 = 1, TERN_ACT_BF16 = 2, TERN_ACT_BF16_Q8 = 3 } tern_act;
 typedef enum { TERN_OUT_F32 = 1, TERN_OUT_BF16 = 2 } tern_out;
 
 /* Descriptor flags. */
@@ -111,7 +115,9 @@ tern_status tern_pack(const tern_desc* desc, const int8_t* trits, const uint16_t
                       size_t* out_used);
 
 /*
- * Workspace needed by tern_gemv / tern_gemm_batched for `m` tokens (may be 0).
+ * Workspace needed by tern_gemv / tern_gemm_batched for `m` tokens (0 for
+ * most layers: K-splits normally reduce inside a thread-block cluster; only a
+ * very long K needs more splits than a cluster holds and a workspace).
  * The workspace holds per-block arrival counters and split partial sums. It
  * must be zero-filled before its first use; every call resets the counters
  * to zero, so the workspace can be reused by later calls without clearing.
@@ -136,8 +142,8 @@ tern_status tern_quantize_act(const uint16_t* d_x_bf16, int32_t m, int32_t k, in
  *   act       TERN_ACT_INT8: d_x int8 [K], d_xscale float [1];
  *             TERN_ACT_BF16: d_x bf16 [K], d_xscale NULL.
  *   out       TERN_OUT_F32 (float [N]) or TERN_OUT_BF16 (bf16 bits [N]).
- *   d_ws      workspace of ws_bytes (see tern_workspace_size); NULL with
- *             ws_bytes 0 runs without splitting K across blocks.
+ *   d_ws      workspace of ws_bytes (see tern_workspace_size); may be NULL when
+ *             tern_workspace_size reports 0, otherwise TERN_ENOSPACE.
  */
 tern_status tern_gemv(const tern_desc* desc, const void* d_packed, tern_act act, const void* d_x,
                       const float* d_xscale, tern_out out, void* d_y, void* d_ws, size_t ws_bytes,
@@ -151,6 +157,22 @@ tern_status tern_gemv(const tern_desc* desc, const void* d_packed, tern_act act,
 tern_status tern_gemm_batched(const tern_desc* desc, const void* d_packed, int32_t m, tern_act act,
                               const void* d_x, const float* d_xscale, tern_out out, void* d_y,
                               void* d_ws, size_t ws_bytes, void* stream);
+
+/*
+ * Several independent single-token GEMVs in one launch (for example the q, k
+ * and v projections of a decode step, or gate and up). The pages state one
+ * GEMV per projection (QORA-LLM-2B, "SubLN Pattern"); running independent
+ * ones together is a launch-level choice of this library.
+ *   count       1..32 problems; descs[i] must share fmt, k, planes, group and
+ *               flags (n may differ).
+ *   d_packed[i], d_x[i] ([K]), d_xscale[i] (TERN_ACT_INT8, else ignored and may
+ *               be NULL), d_y[i] ([n_i]): as tern_gemv, one per problem.
+ * Needs no workspace. Returns TERN_EUNSUPPORTED if K is too large to split
+ * within one thread-block cluster.
+ */
+tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, const void* const* d_packed, tern_act act,
+                              const void* const* d_x, const float* const* d_xscale, tern_out out, void* const* d_y,
+                              void* stream);
 
 /*
  * tern_gemv without a caller-provided workspace, for callers that cannot

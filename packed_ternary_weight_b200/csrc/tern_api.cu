@@ -9,8 +9,6 @@
 namespace tern {
 namespace {
 
-constexpr int kMaxGemvTokens = 16;  // tokens per pass of the GEMV kernels
-
 int device_sms() {
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) {
@@ -26,54 +24,98 @@ int device_sms() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+int xmode_of(tern_act act) {
+  return act == TERN_ACT_INT8 ? kXInt8 : act == TERN_ACT_BF16 ? kXBf16 : kXBf16Q8;
+}
+
 struct Plan2 {
-  int ks, cps, wpc, stage_cols, nstage, grid_x;
+  int ks, cps, wpc, stage_cols, nstage, cluster, grid_x;
   size_t ws_cnt_bytes, ws_part_bytes;
+  bool ok;
 };
 
-// Launch plan of the 2-bit GEMV for m tokens in one pass.
-//  * K is split into `ks` ranges of whole scale groups so that about four warps
-//    per SM have work (small layers are latency-bound; splitting K spreads
-//    their bytes over all SMs);
+// Launch plan of the 2-bit GEMV for problems that share K and format.
+//  * K is split into `ks` ranges of whole scale groups so that about four
+//    warps per SM have work (small layers are latency-bound; splitting K
+//    spreads their bytes over all SMs), and so that the staged activations of
+//    one split fit in shared memory;
+//  * up to 16 splits reduce through a thread-block cluster; beyond that (huge
+//    K only) a single problem reduces through the caller's workspace;
 //  * each warp streams its range in stages of about 8 KB, up to 4 in flight.
-Plan2 plan_gemv2(const Layout& L, int m, int xmode, int sms, bool allow_split) {
+Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xmode, int sms, bool ws_ok) {
   Plan2 pl{};
   const bool tq = L.fmt == TERN_FMT_TQ;
   const int gc = (tq && L.group >= 64) ? L.group / 64 : 1;  // columns per group
   const int units = (L.cols + gc - 1) / gc;
   const int P = L.planes;
+  const int mt = gemv2_mt(xmode, m);
+  int rt_total = 0;
+  for (int i = 0; i < nprob; ++i) rt_total += row_tiles[i];
   pl.wpc = 4;
-  int sc_target = std::max(gc, (8192 / (P * kPlaneColBytes)) / gc * gc);
-  int ks = 1;
-  if (allow_split) {
-    const int target_warps = 4 * sms;
-    ks = std::min(units, std::max(1, (target_warps + L.row_tiles - 1) / L.row_tiles));
+  const int sc_target = std::max(gc, (8192 / (P * kPlaneColBytes)) / gc * gc);
+  const int ks_par = std::min(units, std::max(1, (4 * sms + rt_total - 1) / rt_total));
+  const int bpk = xmode == kXInt8 ? mt : xmode == kXBf16Q8 ? 3 * mt : 3;  // staged bytes per k
+  int ks_x = 1;
+  while (ks_x < units && (size_t)((units + ks_x - 1) / ks_x) * gc * kColK2 * bpk > 96 * 1024) ++ks_x;
+  int ks = std::max(ks_par, ks_x);
+  const size_t elem = (xmode != kXBf16 && tq) ? 8 : 4;
+  if (ks > kMaxCluster && ks_x <= kMaxCluster) ks = kMaxCluster;
+  pl.cluster = 0;
+  if (ks > 1 && ks <= kMaxCluster) {
+    while ((size_t)ks * mt * pl.wpc * 32 * elem > 32 * 1024 && pl.wpc > 1) pl.wpc /= 2;
+    if ((size_t)ks * mt * pl.wpc * 32 * elem <= 32 * 1024) pl.cluster = 1;
   }
-  // x staging must fit: m tokens x k-range bytes (int8) or 2 bytes (bf16) <= 96 KB
-  const int mt = xmode == kXBf16 ? 1 : (m <= 1 ? 1 : m <= 4 ? 4 : 16);
-  const int per_k = xmode == kXBf16 ? 2 : mt;
-  while (ks < units && (size_t)((units + ks - 1) / ks) * gc * kColK2 * per_k > 96 * 1024) ++ks;
-  int cps_units = (units + ks - 1) / ks;
-  pl.cps = cps_units * gc;
+  if (ks > 1 && !pl.cluster && (!ws_ok || nprob != 1 || xmode == kXBf16Q8)) {
+    pl.ok = false;
+    return pl;
+  }
+  pl.cps = ((units + ks - 1) / ks) * gc;
   pl.ks = (L.cols + pl.cps - 1) / pl.cps;
+  if (pl.ks == 1) pl.cluster = 0;
   pl.stage_cols = std::min(sc_target, pl.cps);
   pl.nstage = std::min(4, (pl.cps + pl.stage_cols - 1) / pl.stage_cols);
-  pl.grid_x = (L.row_tiles + pl.wpc - 1) / pl.wpc;
-  if (pl.ks > 1) {
-    const size_t elem = (xmode == kXInt8 && tq) ? 8 : 4;
-    pl.ws_cnt_bytes = ((size_t)pl.grid_x * 4 + 255) / 256 * 256;
-    pl.ws_part_bytes = (size_t)pl.ks * m * L.row_tiles * kTileRows * elem;
+  // fit shared memory: fewer stages in flight, then fewer warps per CTA
+  for (;;) {
+    Gemv2Params t{};
+    t.tq = tq;
+    t.k = L.k;
+    t.planes = P;
+    t.group = L.group;
+    t.groups = L.groups;
+    t.cols = L.cols;
+    t.m = m;
+    t.ks = pl.ks;
+    t.cluster = pl.cluster;
+    t.cols_per_split = pl.cps;
+    t.wpc = pl.wpc;
+    t.stage_cols = pl.stage_cols;
+    t.nstage = pl.nstage;
+    if (gemv2_smem_bytes(t, xmode) <= 227 * 1024) break;
+    if (pl.nstage > 2) {
+      --pl.nstage;
+    } else if (pl.wpc > 1) {
+      pl.wpc /= 2;
+    } else {
+      pl.ok = false;
+      return pl;
+    }
   }
+  pl.grid_x = 0;
+  for (int i = 0; i < nprob; ++i) pl.grid_x += (row_tiles[i] + pl.wpc - 1) / pl.wpc;
+  if (pl.ks > 1 && !pl.cluster) {
+    pl.ws_cnt_bytes = ((size_t)pl.grid_x * 4 + 255) / 256 * 256;
+    pl.ws_part_bytes = (size_t)pl.ks * m * row_tiles[0] * kTileRows * elem;
+  }
+  pl.ok = true;
   return pl;
 }
 
-tern_status check_common(const tern_desc* desc, const void* d_packed, int m, tern_act act, const void* d_x,
-                         const float* d_xscale, tern_out out, void* d_y, Layout* L) {
+tern_status check_one(const tern_desc* desc, const void* d_packed, tern_act act, const void* d_x,
+                      const float* d_xscale, tern_out out, void* d_y, Layout* L) {
   tern_status st = layout_of(desc, L);
   if (st != TERN_OK) return st;
-  if (m < 1) return TERN_EINVAL;
   if (!d_packed || !d_x || !d_y) return TERN_EINVAL;
-  if (act != TERN_ACT_INT8 && act != TERN_ACT_BF16) return TERN_EINVAL;
+  if (act != TERN_ACT_INT8 && act != TERN_ACT_BF16 && act != TERN_ACT_BF16_Q8) return TERN_EINVAL;
   if (out != TERN_OUT_F32 && out != TERN_OUT_BF16) return TERN_EINVAL;
   if (act == TERN_ACT_INT8 && !d_xscale) return TERN_EINVAL;
   if (!aligned16(d_packed)) return TERN_EALIGN;
@@ -81,45 +123,70 @@ tern_status check_common(const tern_desc* desc, const void* d_packed, int m, ter
   return TERN_OK;
 }
 
-tern_status run_gemv2(const tern_desc* desc, const Layout& L, const void* d_packed, int m, tern_act act,
-                      const void* d_x, const float* d_xscale, tern_out out, void* d_y, void* d_ws, size_t ws_bytes,
-                      void* stream) {
-  const int xmode = act == TERN_ACT_INT8 ? kXInt8 : kXBf16;
+// What the 2-bit kernels support for this layout and activation mode.
+tern_status supported_2bit(const Layout& L, int xmode) {
   const bool tq = L.fmt == TERN_FMT_TQ;
-  if (xmode == kXBf16 && (!tq || m != 1)) return TERN_EUNSUPPORTED;
+  if (L.fmt == TERN_FMT_BT3) return TERN_EUNSUPPORTED;
+  if (xmode == kXBf16 && !tq) return TERN_EUNSUPPORTED;
   if (tq && L.k % kColK2 != 0) return TERN_EUNSUPPORTED;
   if (!tq && (long long)L.k * 127 >= (1ll << 24)) return TERN_EUNSUPPORTED;  // exact int32 -> fp32
+  return TERN_OK;
+}
+
+void fill_common(Gemv2Params& p, const Layout& L, const Plan2& pl, int m, tern_out out) {
+  p.tq = L.fmt == TERN_FMT_TQ;
+  p.k = L.k;
+  p.planes = L.planes;
+  p.group = L.group;
+  p.groups = L.groups;
+  p.cols = L.cols;
+  p.m = m;
+  p.out_bf16 = out == TERN_OUT_BF16;
+  p.ks = pl.ks;
+  p.cluster = pl.cluster;
+  p.cols_per_split = pl.cps;
+  p.wpc = pl.wpc;
+  p.stage_cols = pl.stage_cols;
+  p.nstage = pl.nstage;
+  p.grid_x = pl.grid_x;
+}
+
+tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_packed, int m, tern_act act,
+                       const void* d_x, const float* d_xscale, tern_out out, void* d_y, void* d_ws, size_t ws_bytes,
+                       void* stream) {
+  const int xmode = xmode_of(act);
+  tern_status st = supported_2bit(L, xmode);
+  if (st != TERN_OK) return st;
+  if (xmode == kXBf16 && m != 1) return TERN_EUNSUPPORTED;
   const int sms = device_sms();
   const uint8_t* base = static_cast<const uint8_t*>(d_packed);
   const size_t in_elem = xmode == kXInt8 ? 1 : 2;
   const size_t out_elem = out == TERN_OUT_F32 ? 4 : 2;
-  for (int t0 = 0; t0 < m; t0 += kMaxGemvTokens) {
-    const int mc = std::min(kMaxGemvTokens, m - t0);
-    Plan2 pl = plan_gemv2(L, mc, xmode, sms, d_ws != nullptr);
-    if (pl.ks > 1 && ws_bytes < pl.ws_cnt_bytes + pl.ws_part_bytes) return TERN_ENOSPACE;
+  const int mt_max = gemv2_mt(xmode, m);
+  for (int t0 = 0; t0 < m; t0 += mt_max) {
+    const int mc = std::min(mt_max, m - t0);
+    const int rt = L.row_tiles;
+    const Plan2 pl = plan_gemv2(L, &rt, 1, mc, xmode, sms, d_ws != nullptr);
+    if (!pl.ok) return d_ws ? TERN_EUNSUPPORTED : TERN_ENOSPACE;
+    if (pl.ks > 1 && !pl.cluster && ws_bytes < pl.ws_cnt_bytes + pl.ws_part_bytes) return TERN_ENOSPACE;
     Gemv2Params p{};
-    p.trit = base + L.trit_offset;
-    p.scale = tq ? reinterpret_cast<const uint16_t*>(base + L.scale_offset) : nullptr;
-    p.n = L.n;
-    p.k = L.k;
-    p.planes = L.planes;
-    p.group = L.group;
-    p.groups = L.groups;
-    p.row_tiles = L.row_tiles;
-    p.cols = L.cols;
-    p.tensor_scale = desc->tensor_scale;
-    p.m = mc;
-    p.x = static_cast<const uint8_t*>(d_x) + (size_t)t0 * L.k * in_elem;
-    p.xscale = d_xscale ? d_xscale + t0 : nullptr;
-    p.y = static_cast<uint8_t*>(d_y) + (size_t)t0 * L.n * out_elem;
-    p.out_bf16 = out == TERN_OUT_BF16;
-    p.ks = pl.ks;
-    p.cols_per_split = pl.cps;
-    p.wpc = pl.wpc;
-    p.stage_cols = pl.stage_cols;
-    p.nstage = pl.nstage;
-    p.ws_cnt = pl.ks > 1 ? static_cast<unsigned*>(d_ws) : nullptr;
-    p.ws_part = pl.ks > 1 ? static_cast<uint8_t*>(d_ws) + pl.ws_cnt_bytes : nullptr;
+    fill_common(p, L, pl, mc, out);
+    p.nprob = 1;
+    Gemv2Problem& q = p.prob[0];
+    q.trit = base + L.trit_offset;
+    q.scale = p.tq ? reinterpret_cast<const uint16_t*>(base + L.scale_offset) : nullptr;
+    q.x = static_cast<const uint8_t*>(d_x) + (size_t)t0 * L.k * in_elem;
+    q.xscale = d_xscale ? d_xscale + t0 : nullptr;
+    q.y = static_cast<uint8_t*>(d_y) + (size_t)t0 * L.n * out_elem;
+    q.n = L.n;
+    q.row_tiles = L.row_tiles;
+    q.cta_begin = 0;
+    q.tensor_scale = desc->tensor_scale;
+    p.x_vec = aligned16(q.x) && L.k % 16 == 0;
+    if (pl.ks > 1 && !pl.cluster) {
+      p.ws_cnt = static_cast<unsigned*>(d_ws);
+      p.ws_part = static_cast<uint8_t*>(d_ws) + pl.ws_cnt_bytes;
+    }
     if (gemv2_smem_bytes(p, xmode) > 227 * 1024) return TERN_EUNSUPPORTED;
     const int rc = launch_gemv2(p, xmode, (desc->flags & TERN_F_PDL) != 0, stream);
     if (rc < 0) return TERN_EUNSUPPORTED;
@@ -142,10 +209,11 @@ extern "C" tern_status tern_workspace_size(const tern_desc* desc, int32_t m, siz
   const int sms = device_sms();
   size_t need = 0;
   if (L.fmt != TERN_FMT_BT3) {
-    const int mc = std::max(1, std::min<int>(m, kMaxGemvTokens));
-    for (int xmode = 0; xmode < 2; ++xmode) {
-      Plan2 pl = plan_gemv2(L, mc, xmode, sms, true);
-      need = std::max(need, pl.ws_cnt_bytes + pl.ws_part_bytes);
+    const int rt = L.row_tiles;
+    for (int xmode = 0; xmode < 3; ++xmode) {
+      const int mc = std::max(1, std::min(m, gemv2_mt(xmode, std::max(1, m))));
+      const Plan2 pl = plan_gemv2(L, &rt, 1, mc, xmode, sms, true);
+      if (pl.ok) need = std::max(need, pl.ws_cnt_bytes + pl.ws_part_bytes);
     }
   }
   *bytes = need;
@@ -162,16 +230,64 @@ extern "C" tern_status tern_gemm_batched(const tern_desc* desc, const void* d_pa
                                          const void* d_x, const float* d_xscale, tern_out out, void* d_y, void* d_ws,
                                          size_t ws_bytes, void* stream) {
   Layout L;
-  tern_status st = check_common(desc, d_packed, m, act, d_x, d_xscale, out, d_y, &L);
+  if (m < 1) return TERN_EINVAL;
+  tern_status st = check_one(desc, d_packed, act, d_x, d_xscale, out, d_y, &L);
   if (st != TERN_OK) return st;
-  if (L.fmt == TERN_FMT_BT3) return TERN_EUNSUPPORTED;
-  return run_gemv2(desc, L, d_packed, m, act, d_x, d_xscale, out, d_y, d_ws, ws_bytes, stream);
+  return run_single(desc, L, d_packed, m, act, d_x, d_xscale, out, d_y, d_ws, ws_bytes, stream);
 }
 
 extern "C" tern_status tern_gemv(const tern_desc* desc, const void* d_packed, tern_act act, const void* d_x,
                                  const float* d_xscale, tern_out out, void* d_y, void* d_ws, size_t ws_bytes,
                                  void* stream) {
   return tern_gemm_batched(desc, d_packed, 1, act, d_x, d_xscale, out, d_y, d_ws, ws_bytes, stream);
+}
+
+extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, const void* const* d_packed,
+                                         tern_act act, const void* const* d_x, const float* const* d_xscale,
+                                         tern_out out, void* const* d_y, void* stream) {
+  if (count < 1 || count > kMaxProblems || !descs || !d_packed || !d_x || !d_y) return TERN_EINVAL;
+  if (act == TERN_ACT_INT8 && !d_xscale) return TERN_EINVAL;
+  Layout L[kMaxProblems];
+  int rt[kMaxProblems];
+  for (int i = 0; i < count; ++i) {
+    tern_status st = check_one(&descs[i], d_packed[i], act, d_x[i], d_xscale ? d_xscale[i] : nullptr, out, d_y[i],
+                               &L[i]);
+    if (st != TERN_OK) return st;
+    if (L[i].fmt != L[0].fmt || L[i].k != L[0].k || L[i].planes != L[0].planes || L[i].group != L[0].group ||
+        descs[i].flags != descs[0].flags)
+      return TERN_EINVAL;
+    rt[i] = L[i].row_tiles;
+  }
+  const int xmode = xmode_of(act);
+  tern_status st = supported_2bit(L[0], xmode);
+  if (st != TERN_OK) return st;
+  const Plan2 pl = plan_gemv2(L[0], rt, count, 1, xmode, device_sms(), false);
+  if (!pl.ok) return TERN_EUNSUPPORTED;
+  Gemv2Params p{};
+  fill_common(p, L[0], pl, 1, out);
+  p.nprob = count;
+  int cta = 0;
+  bool vec = L[0].k % 16 == 0;
+  for (int i = 0; i < count; ++i) {
+    const uint8_t* base = static_cast<const uint8_t*>(d_packed[i]);
+    Gemv2Problem& q = p.prob[i];
+    q.trit = base + L[i].trit_offset;
+    q.scale = p.tq ? reinterpret_cast<const uint16_t*>(base + L[i].scale_offset) : nullptr;
+    q.x = d_x[i];
+    q.xscale = d_xscale ? d_xscale[i] : nullptr;
+    q.y = d_y[i];
+    q.n = L[i].n;
+    q.row_tiles = L[i].row_tiles;
+    q.cta_begin = cta;
+    q.tensor_scale = descs[i].tensor_scale;
+    cta += (L[i].row_tiles + pl.wpc - 1) / pl.wpc;
+    vec = vec && aligned16(q.x);
+  }
+  p.x_vec = vec;
+  if (gemv2_smem_bytes(p, xmode) > 227 * 1024) return TERN_EUNSUPPORTED;
+  const int rc = launch_gemv2(p, xmode, (descs[0].flags & TERN_F_PDL) != 0, stream);
+  if (rc < 0) return TERN_EUNSUPPORTED;
+  return rc == 0 ? TERN_OK : TERN_ECUDA;
 }
 
 extern "C" tern_status tern_device_error(void* stream) {

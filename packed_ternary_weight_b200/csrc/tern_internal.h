@@ -31,34 +31,54 @@ struct Layout {
 tern_status layout_of(const tern_desc* d, Layout* L);
 
 // ------------------------------------------------------------ kernels
-enum XMode : int { kXInt8 = 0, kXBf16 = 1 };
+// Activation modes of the 2-bit GEMV:
+//   kXInt8   int8 activations with one fp32 scale per token (exact path);
+//   kXBf16   bf16 activations (24-bit fixed-point image, fp32 group fold);
+//   kXBf16Q8 bf16 activations quantised per token inside the kernel, then the
+//            exact int8 path (same result as tern_quantize_act + kXInt8).
+enum XMode : int { kXInt8 = 0, kXBf16 = 1, kXBf16Q8 = 2 };
 
-struct Gemv2Params {
+constexpr int kMaxProblems = 32;  // independent GEMVs in one grouped launch
+constexpr int kMaxCluster = 16;   // K-splits reduced through one thread-block cluster
+
+struct Gemv2Problem {
   const uint8_t* trit;      // trit stream (device)
   const uint16_t* scale;    // TQ scale stream (fp16 bits) or nullptr
-  int n, k, planes, group, groups, row_tiles, cols;
+  const void* x;            // activations [m][k]
+  const float* xscale;      // kXInt8: [m]
+  void* y;                  // [m][n] float or bf16
+  int n, row_tiles;
+  int cta_begin;            // first blockIdx.x of this problem
   float tensor_scale;       // BitNet
+};
+
+struct Gemv2Params {
+  Gemv2Problem prob[kMaxProblems];
+  int nprob;
+  int grid_x;               // sum over problems of ceil(row_tiles / wpc)
+  int tq;                   // fp16 group scales (TQ) rather than one per-tensor scale
+  int k, planes, group, groups, cols;   // shared by all problems
   int m;                    // tokens
-  const void* x;            // int8 [m][k] or bf16 [m][k]
-  const float* xscale;      // int8 path: [m]
-  void* y;                  // float [m][n] or bf16 [m][n]
   int out_bf16;
   int ks;                   // K splits (grid.y)
+  int cluster;              // 1: splits reduce through a (1, ks, 1) cluster; 0: through ws
   int cols_per_split;       // multiple of the group's column count
   int wpc;                  // warps (row tiles) per CTA
   int stage_cols;           // columns per pipeline stage
   int nstage;               // stages per warp ring
-  void* ws_part;            // split partials [ks][m][row_tiles*32] (int32 / int64 / float)
-  unsigned* ws_cnt;         // per-CTA-row arrival counters [grid.x]
+  int x_vec;                // activations may be read with 16-byte loads
+  void* ws_part;            // global fallback: partials [ks][m][row_tiles*32]
+  unsigned* ws_cnt;         // global fallback: arrival counters [grid.x]
 };
 
 // Launchers return cudaError_t values as int (0 = success).
-int launch_gemv2(const Gemv2Params& p, int xmode, bool pdl, void* stream);
+int launch_gemv2(const Gemv2Params& p, int xmode, bool pdl, void* stream);  // -1: no kernel
 int launch_quantize(const uint16_t* x, int m, int k, int8_t* xq, float* xs, void* stream);
 
 int read_clear_dev_error_gemv2(void* stream, unsigned* out);
 
 // Shared-memory bytes a 2-bit GEMV CTA needs for these parameters.
 size_t gemv2_smem_bytes(const Gemv2Params& p, int xmode);
+int gemv2_mt(int xmode, int m);   // tokens per pass of the kernel instantiated for m
 
 }  // namespace tern

@@ -15,7 +15,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtern.so
 
 OK, EINVAL, EFORMAT, EALIGN, ENOSPACE, EUNSUPPORTED, ECUDA, ETIMEOUT = range(8)
 FMT = {"bitnet": 1, "tq": 2, "bt3": 3}
-ACT_INT8, ACT_BF16 = 1, 2
+ACT_INT8, ACT_BF16, ACT_BF16_Q8 = 1, 2, 3
 OUT_F32, OUT_BF16 = 1, 2
 F_PDL = 1
 
@@ -53,8 +53,10 @@ lib.tern_gemm_batched.argtypes = [ctypes.POINTER(Desc), _vp, ctypes.c_int32, cty
                                   _vp, _vp, _sz, _vp]
 lib.tern_device_error.argtypes = [_vp]
 lib.tern_gemv_noalloc.argtypes = [ctypes.POINTER(Desc), _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp, _vp]
+lib.tern_gemv_grouped.argtypes = [ctypes.c_int32, ctypes.POINTER(Desc), ctypes.POINTER(_vp), ctypes.c_int,
+                                  ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.c_int, ctypes.POINTER(_vp), _vp]
 for _f in (lib.tern_packed_size, lib.tern_pack, lib.tern_workspace_size, lib.tern_quantize_act, lib.tern_gemv,
-           lib.tern_gemm_batched, lib.tern_device_error, lib.tern_gemv_noalloc):
+           lib.tern_gemm_batched, lib.tern_device_error, lib.tern_gemv_noalloc, lib.tern_gemv_grouped):
     _f.restype = ctypes.c_int
 
 
@@ -141,6 +143,28 @@ def gemv(desc: Desc, packed, act: int, x, xscale, out: int, y, ws=None, stream=N
     ws_bytes = 0 if ws is None else ws.numel() * ws.element_size()
     _check(lib.tern_gemv(ctypes.byref(desc), _ptr(packed), act, _ptr(x), _ptr(xscale), out, _ptr(y), _ptr(ws),
                          ws_bytes, _stream(stream)), "tern_gemv")
+
+
+class Grouped:
+    """Marshalled arguments of tern_gemv_grouped, built once and launched many times."""
+
+    def __init__(self, descs, packed, act: int, xs, xscales, out: int, ys):
+        n = len(descs)
+        self.count = n
+        self.act, self.out = act, out
+        self.descs = (Desc * n)(*descs)
+        self.packed = (_vp * n)(*[p.data_ptr() for p in packed])
+        self.xs = (_vp * n)(*[x.data_ptr() for x in xs])
+        self.xscales = None if xscales is None else (_vp * n)(*[s.data_ptr() for s in xscales])
+        self.ys = (_vp * n)(*[y.data_ptr() for y in ys])
+
+    def launch(self, stream=None):
+        _check(lib.tern_gemv_grouped(self.count, self.descs, self.packed, self.act, self.xs, self.xscales, self.out,
+                                     self.ys, _stream(stream)), "tern_gemv_grouped")
+
+
+def gemv_grouped(descs, packed, act: int, xs, xscales, out: int, ys, stream=None):
+    Grouped(descs, packed, act, xs, xscales, out, ys).launch(stream)
 
 
 def gemv_noalloc(desc: Desc, packed, act: int, x, xscale, out: int, y, stream=None):

@@ -214,3 +214,98 @@ def test_tq_bf16_wide_dynamic_range(tern):
     y32 = run_bf16(tern, lay, x, tern.OUT_F32)
     yref = oracle.gemv_bf16(oracle.dequantize("tq", lay.trits, 256, scales=lay.scales), x)[0]
     check_bf16(y32[0], yref)
+
+
+# ----------------------------------------- in-kernel per-token quantisation
+def q8_check(tern, layer, m):
+    x = synth.draw_x_bf16(layer.seed, m, layer.k)
+    d, buf = tern.pack_layer(layer)
+    pk = dev(buf)
+    y = torch.empty((m, layer.n), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(16, tern.workspace_size(d, m)), dtype=torch.uint8, device="cuda")
+    tern.gemm_batched(d, pk, m, tern.ACT_BF16_Q8, x_dev(x), None, tern.OUT_F32, y, ws)
+    torch.cuda.synchronize()
+    assert tern.device_error() == tern.OK
+    q_ref, s_ref = oracle.quantize_act(x)
+    if layer.fmt == "bitnet":
+        y_ref = oracle.gemv_bitnet_int8(layer.trits, q_ref, s_ref, layer.tensor_scale)
+    else:
+        y_ref = oracle.gemv_tq_int8(layer.trits, layer.scales, layer.group, q_ref, s_ref)
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), y_ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("shape", synth.BITNET_2B_SHAPES, ids=[s[0] for s in synth.BITNET_2B_SHAPES])
+def test_bitnet_fused_quant_bit_exact(tern, shape):
+    name, n, k = shape
+    q8_check(tern, synth.bitnet_layer(n, k, 2000 + n + k), 1)
+
+
+@pytest.mark.parametrize("m", [1, 3, 4, 6])
+def test_fused_quant_batched_bit_exact(tern, m):
+    q8_check(tern, synth.bitnet_layer(300, 1000, seed=m), m)
+    q8_check(tern, synth.tq_layer(200, 1024, 2, 32, seed=m), m)
+
+
+def test_single_gemv_fused_quant(tern):
+    q8_check(tern, synth.single_gemv_layer(), 1)
+
+
+# ------------------------------------------------------------ grouped launch
+def test_grouped_qkv_matches_single(tern):
+    descs, packs, xs, ys, refs = [], [], [], [], []
+    for i, (name, n, k) in enumerate(synth.BITNET_2B_SHAPES[:3]):
+        lay = synth.bitnet_layer(n, k, 3000 + i)
+        d, buf = tern.pack_layer(lay)
+        x = synth.draw_x_bf16(lay.seed, 1, k)
+        q_ref, s_ref = oracle.quantize_act(x)
+        refs.append(oracle.gemv_bitnet_int8(lay.trits, q_ref, s_ref, lay.tensor_scale)[0])
+        descs.append(d)
+        packs.append(dev(buf))
+        xs.append(x_dev(x))
+        ys.append(torch.empty(n, dtype=torch.float32, device="cuda"))
+    tern.gemv_grouped(descs, packs, tern.ACT_BF16_Q8, xs, None, tern.OUT_F32, ys)
+    torch.cuda.synchronize()
+    for y, r in zip(ys, refs):
+        assert np.array_equal(y.cpu().numpy().view(np.uint32), r.view(np.uint32))
+
+
+def test_grouped_int8_and_bf16(tern):
+    lays = [synth.tq_layer(n, 1024, 3, 256, seed=60 + n) for n in (96, 300, 33)]
+    descs, packs, xs, xqs, sxs, ys, ys2 = [], [], [], [], [], [], []
+    for lay in lays:
+        d, buf = tern.pack_layer(lay)
+        descs.append(d)
+        packs.append(dev(buf))
+        x = synth.draw_x_bf16(lay.seed, 1, lay.k)
+        xs.append(x_dev(x))
+        xq = torch.empty((1, lay.k), dtype=torch.int8, device="cuda")
+        sx = torch.empty((1,), dtype=torch.float32, device="cuda")
+        tern.quantize_act(xs[-1].view(1, -1), xq, sx)
+        xqs.append(xq)
+        sxs.append(sx)
+        ys.append(torch.empty(lay.n, dtype=torch.float32, device="cuda"))
+        ys2.append(torch.empty(lay.n, dtype=torch.float32, device="cuda"))
+    tern.gemv_grouped(descs, packs, tern.ACT_INT8, xqs, sxs, tern.OUT_F32, ys)
+    tern.gemv_grouped(descs, packs, tern.ACT_BF16, xs, None, tern.OUT_F32, ys2)
+    torch.cuda.synchronize()
+    for lay, y, y2, x, in zip(lays, ys, ys2, xs):
+        xb = x.cpu().numpy().view(np.uint16)[None]
+        q_ref, s_ref = oracle.quantize_act(xb)
+        r = oracle.gemv_tq_int8(lay.trits, lay.scales, 256, q_ref, s_ref)[0]
+        assert np.array_equal(y.cpu().numpy().view(np.uint32), r.view(np.uint32))
+        yref = oracle.gemv_bf16(oracle.dequantize("tq", lay.trits, 256, scales=lay.scales), xb)[0]
+        check_bf16(y2.cpu().numpy(), yref)
+
+
+# ------------------------------------------- very long K: workspace reduction
+def test_long_k_workspace_path(tern):
+    lay = synth.tq_layer(64, 1 << 21, 1, 256, seed=8)
+    d = tern.desc_of(lay)
+    assert tern.workspace_size(d, 1) > 0
+    tq_int8_check(tern, lay, 1, rows=np.arange(0, 64, 7))
+    with pytest.raises(tern.TernError) as ei:       # no workspace -> refused
+        y = torch.empty(64, dtype=torch.float32, device="cuda")
+        xq = torch.zeros(lay.k, dtype=torch.int8, device="cuda")
+        sx = torch.ones(1, dtype=torch.float32, device="cuda")
+        tern.gemv(d, dev(tern.pack_layer(lay)[1]), tern.ACT_INT8, xq, sx, tern.OUT_F32, y, None)
+    assert ei.value.code == tern.ENOSPACE

@@ -27,48 +27,47 @@ def tern():
     return t
 
 
-def _int8_case(tern, n, k, seed):
-    lay = synth.bitnet_layer(n, k, seed=seed)
+def _run_both(tern, lay, act, x, xq=None, sx=None):
+    """tern_gemv with a caller workspace, then tern_gemv_noalloc twice; returns the three outputs."""
     d, buf = tern.pack_layer(lay)
+    need = tern.workspace_size(d, 1)
+    assert 0 < need <= (1 << 20)                           # this layer uses the scratch
     pk = torch.from_numpy(buf).cuda()
-    x = torch.from_numpy(synth.draw_x_bf16(seed, 1, k).view(np.int16)).cuda()
-    xq = torch.empty((1, k), dtype=torch.int8, device="cuda")
-    sx = torch.empty((1,), dtype=torch.float32, device="cuda")
-    tern.quantize_act(x, xq, sx)
-    return d, pk, xq, sx
+    xin = xq if act == tern.ACT_INT8 else x
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    y_ref = torch.empty(lay.n, dtype=torch.float32, device="cuda")
+    tern.gemv(d, pk, act, xin, sx, tern.OUT_F32, y_ref, ws)
+    outs = []
+    for _ in range(2):
+        y = torch.full((lay.n,), float("nan"), dtype=torch.float32, device="cuda")
+        tern.gemv_noalloc(d, pk, act, xin, sx, tern.OUT_F32, y)
+        torch.cuda.synchronize()
+        outs.append(y)
+    assert tern.device_error() == tern.OK
+    return y_ref, outs
 
 
 def test_noalloc_matches_gemv_int8_two_calls(tern):
-    d, pk, xq, sx = _int8_case(tern, 2560, 2560, 1003)      # splits K: uses the scratch
-    assert tern.workspace_size(d, 1) > 0
-    ws = torch.zeros(tern.workspace_size(d, 1), dtype=torch.uint8, device="cuda")
-    y_ref = torch.empty(2560, dtype=torch.float32, device="cuda")
-    tern.gemv(d, pk, tern.ACT_INT8, xq, sx, tern.OUT_F32, y_ref, ws)
-    for _ in range(2):
-        y = torch.full((2560,), float("nan"), dtype=torch.float32, device="cuda")
-        tern.gemv_noalloc(d, pk, tern.ACT_INT8, xq, sx, tern.OUT_F32, y)
-        torch.cuda.synchronize()
+    # a very long K splits beyond one thread-block cluster and needs the scratch
+    lay = synth.tq_layer(64, 1 << 21, 1, 256, seed=5)
+    x = torch.from_numpy(synth.draw_x_bf16(5, 1, lay.k).view(np.int16)).cuda()
+    xq = torch.empty((1, lay.k), dtype=torch.int8, device="cuda")
+    sx = torch.empty((1,), dtype=torch.float32, device="cuda")
+    tern.quantize_act(x, xq, sx)
+    y_ref, outs = _run_both(tern, lay, tern.ACT_INT8, x, xq, sx)
+    for y in outs:
         assert torch.equal(y.view(torch.int32), y_ref.view(torch.int32))
-    assert tern.device_error() == tern.OK
 
 
 def test_noalloc_matches_gemv_bf16_two_calls(tern):
-    lay = synth.tq_layer(4096, 4096, 3, 256, seed=200)
-    d, buf = tern.pack_layer(lay)
-    pk = torch.from_numpy(buf).cuda()
-    x = torch.from_numpy(synth.draw_x_bf16(200, 1, 4096).view(np.int16)).cuda()
-    ws = torch.zeros(max(16, tern.workspace_size(d, 1)), dtype=torch.uint8, device="cuda")
-    y_ref = torch.empty(4096, dtype=torch.float32, device="cuda")
-    tern.gemv(d, pk, tern.ACT_BF16, x, None, tern.OUT_F32, y_ref, ws)
+    lay = synth.tq_layer(64, 1 << 20, 1, 256, seed=6)
+    x = torch.from_numpy(synth.draw_x_bf16(6, 1, lay.k).view(np.int16)).cuda()
+    y_ref, outs = _run_both(tern, lay, tern.ACT_BF16, x)
     ref = y_ref.double()
     floor = 1e-2 * ref.pow(2).mean().sqrt()
-    for _ in range(2):
-        y = torch.full((4096,), float("nan"), dtype=torch.float32, device="cuda")
-        tern.gemv_noalloc(d, pk, tern.ACT_BF16, x, None, tern.OUT_F32, y)
-        torch.cuda.synchronize()
+    for y in outs:
         err = ((y.double() - ref).abs() / torch.maximum(ref.abs(), floor)).max().item()
         assert err <= 1e-3
-    assert tern.device_error() == tern.OK
 
 
 def test_noalloc_rejects_layer_beyond_scratch(tern):
