@@ -49,6 +49,9 @@ def parse():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--layers", type=int, default=synth.BITNET_2B_LAYERS)
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--profile", default=None,
+                    help="run only one case eagerly for a profiler: step | <shape>_indep | <shape>_chain")
+    ap.add_argument("--reps", type=int, default=3)
     return ap.parse_args()
 
 
@@ -161,6 +164,20 @@ def run_ours(args, rank, world):
     # as one launch of 30 independent GEMVs
     chain = {nm: [grouped([L]) for L in layers if L["name"] == nm] for nm, _, _ in synth.BITNET_2B_SHAPES}
     indep = {nm: grouped([L for L in layers if L["name"] == nm]) for nm, _, _ in synth.BITNET_2B_SHAPES}
+
+    if args.profile:
+        cases = {"step": step}
+        for nm, _, _ in synth.BITNET_2B_SHAPES:
+            short = nm.split("_")[0]
+            cases[f"{short}_indep"] = indep[nm].launch
+            cases[f"{short}_chain"] = (lambda gs=chain[nm]: [g.launch(stream) for g in gs])
+        fn = cases[args.profile]
+        with torch.cuda.stream(stream):
+            for _ in range(args.reps):
+                fn() if not args.profile.endswith("_indep") else fn(stream)
+            torch.cuda.synchronize()
+        assert tern.device_error(stream) == tern.OK
+        return None
 
     def capture(fn):
         g = torch.cuda.CUDAGraph()

@@ -195,6 +195,20 @@ tern_status tern_gemv_noalloc(const tern_desc* desc, const void* d_packed, tern_
                               const float* d_xscale, tern_out out, void* d_y, void* stream);
 
 /*
+ * Read-ceiling measurement: stream `bytes` of d_src once, folding them into a
+ * checksum, with one of the access shapes the GEMV kernels can use (the pages
+ * have no counterpart; the bandwidth it reaches is the roofline the GEMV
+ * kernels are reported against).
+ *   mode 0: 16-byte loads per thread, `depth` (1, 2, 4 or 8) in flight;
+ *   mode 1: bulk async copies of `chunk` bytes into a per-warp ring of `depth`
+ *           shared-memory stages; mode 2: one such ring per CTA.
+ *   ctas_per_sm x SM-count CTAs of 32*warps threads; d_sink: one unsigned
+ *   (left unchanged unless a checksum hits a fixed value). d_src 16-byte aligned.
+ */
+tern_status tern_stream_read(const void* d_src, size_t bytes, int32_t mode, int32_t chunk, int32_t depth,
+                             int32_t ctas_per_sm, int32_t warps, unsigned* d_sink, void* stream);
+
+/*
  * Read and clear the device error word (synchronises `stream`).
  * Returns TERN_OK if no kernel reported a failure, TERN_ETIMEOUT if a bounded
  * wait expired, TERN_ECUDA if the read failed.

@@ -41,7 +41,8 @@ struct Plan2 {
 //    one split fit in shared memory;
 //  * up to 16 splits reduce through a thread-block cluster; beyond that (huge
 //    K only) a single problem reduces through the caller's workspace;
-//  * each warp streams its range in stages of about 8 KB, up to 4 in flight.
+//  * each warp streams its range in stages of about 4 KB, up to 3 in flight
+//    (small stages keep enough warps resident to hide the latency).
 Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xmode, int sms, bool ws_ok) {
   Plan2 pl{};
   const bool tq = L.fmt == TERN_FMT_TQ;
@@ -52,7 +53,7 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
   int rt_total = 0;
   for (int i = 0; i < nprob; ++i) rt_total += row_tiles[i];
   pl.wpc = 4;
-  const int sc_target = std::max(gc, (8192 / (P * kPlaneColBytes)) / gc * gc);
+  const int sc_target = std::max(gc, (4096 / (P * kPlaneColBytes)) / gc * gc);
   const int ks_par = std::min(units, std::max(1, (4 * sms + rt_total - 1) / rt_total));
   const int bpk = xmode == kXInt8 ? mt : xmode == kXBf16Q8 ? 3 * mt : 3;  // staged bytes per k
   int ks_x = 1;
@@ -73,7 +74,7 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
   pl.ks = (L.cols + pl.cps - 1) / pl.cps;
   if (pl.ks == 1) pl.cluster = 0;
   pl.stage_cols = std::min(sc_target, pl.cps);
-  pl.nstage = std::min(4, (pl.cps + pl.stage_cols - 1) / pl.stage_cols);
+  pl.nstage = std::min(3, (pl.cps + pl.stage_cols - 1) / pl.stage_cols);
   // fit shared memory: fewer stages in flight, then fewer warps per CTA
   for (;;) {
     Gemv2Params t{};
@@ -293,5 +294,14 @@ extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, 
 extern "C" tern_status tern_device_error(void* stream) {
   unsigned v = 0;
   if (read_clear_dev_error_gemv2(stream, &v) != 0) return TERN_ECUDA;
+  if (read_clear_dev_error_stream(stream, &v) != 0) return TERN_ECUDA;
   return v ? TERN_ETIMEOUT : TERN_OK;
+}
+
+extern "C" tern_status tern_stream_read(const void* d_src, size_t bytes, int32_t mode, int32_t chunk, int32_t depth,
+                                        int32_t ctas_per_sm, int32_t warps, unsigned* d_sink, void* stream) {
+  if (!d_src || !d_sink) return TERN_EINVAL;
+  const int rc = launch_stream_read(d_src, bytes, mode, chunk, depth, ctas_per_sm, warps, d_sink, stream);
+  if (rc < 0) return TERN_EINVAL;
+  return rc == 0 ? TERN_OK : TERN_ECUDA;
 }

@@ -48,6 +48,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "tern_ptx.cuh"
 
 namespace tern {
@@ -65,6 +67,14 @@ struct SmemPlan {
 };
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+template <int I>
+__device__ __forceinline__ uint32_t u4_get(const uint4& v) {
+  if constexpr (I == 0) return v.x;
+  if constexpr (I == 1) return v.y;
+  if constexpr (I == 2) return v.z;
+  return v.w;
+}
 
 __host__ __device__ inline int red_elem(int xmode, bool tq) { return (xmode != kXBf16 && tq) ? 8 : 4; }
 
@@ -104,30 +114,40 @@ __host__ __device__ inline SmemPlan smem_plan(const Gemv2Params& p, int xmode, i
 }
 
 // ------------------------------------------------------------ activations
-// Per-(token, group) sums of the staged int8 activations.
-template <int MT>
-__device__ void int8_group_sums(const SmemPlan& sp, uint8_t* smem, int kr, int gsz) {
-  const int8_t* xs = reinterpret_cast<const int8_t*>(smem + sp.xa);
-  int* gs = reinterpret_cast<int*>(smem + sp.gsum);
-  const int gr = (kr + gsz - 1) / gsz;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  for (int t = warp; t < MT * gr; t += nw) {
-    const int mm = t / gr, g = t - mm * gr;
-    const int* w = reinterpret_cast<const int*>(xs + mm * kr + g * gsz);  // gsz, kr multiples of 16
-    int s = 0;
-    for (int i = lane; i < min(gsz, kr - g * gsz) / 4; i += 32) s = __dp4a(w[i], 0x01010101, s);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) gs[mm * gr + g] = s;
-  }
+// Sum of the 16 signed bytes of v.
+__device__ __forceinline__ int sum16_s8(uint4 v) {
+  int s = __dp4a((int)v.x, 0x01010101, 0);
+  s = __dp4a((int)v.y, 0x01010101, s);
+  s = __dp4a((int)v.z, 0x01010101, s);
+  return __dp4a((int)v.w, 0x01010101, s);
 }
+
+// Adds chunk sums to the per-(token, group) sums in shared memory with one
+// atomic per change of group (a thread's chunks of one BitNet token all fall
+// in the same group).
+struct GroupSumAcc {
+  int* gs;
+  int key = -1, val = 0;
+  __device__ void add(int k, int v) {
+    if (k != key) {
+      if (key >= 0) atomicAdd(&gs[key], val);
+      key = k;
+      val = 0;
+    }
+    val += v;
+  }
+  __device__ void flush() {
+    if (key >= 0) atomicAdd(&gs[key], val);
+  }
+};
 
 template <int MT>
 __device__ void stage_x_int8(const Gemv2Params& p, const Gemv2Problem& pr, const SmemPlan& sp, uint8_t* smem, int k0,
-                             int kr) {
+                             int kr, int gsz) {
   int8_t* xs = reinterpret_cast<int8_t*>(smem + sp.xa);
   const int8_t* x = static_cast<const int8_t*>(pr.x);
-  const int m = p.m, K = p.k, nch = kr / 16;
+  const int m = p.m, K = p.k, nch = kr / 16, gr = (kr + gsz - 1) / gsz;
+  GroupSumAcc acc{reinterpret_cast<int*>(smem + sp.gsum)};
   for (int i = threadIdx.x; i < MT * nch; i += blockDim.x) {
     const int t = i / nch, c = i - t * nch, k = k0 + 16 * c;
     uint4 v = make_uint4(0, 0, 0, 0);
@@ -144,7 +164,9 @@ __device__ void stage_x_int8(const Gemv2Params& p, const Gemv2Problem& pr, const
       }
     }
     *reinterpret_cast<uint4*>(xs + t * kr + 16 * c) = v;
+    acc.add(t * gr + (16 * c) / gsz, sum16_s8(v));
   }
+  acc.flush();
 }
 
 __device__ __forceinline__ float bf16_abs_max8(uint4 v) {
@@ -162,7 +184,7 @@ __device__ __forceinline__ float bf16_abs_max8(uint4 v) {
 // the token maxima of all K-splits are exchanged through the cluster.
 template <int MT>
 __device__ void stage_x_q8(const Gemv2Params& p, const Gemv2Problem& pr, const SmemPlan& sp, uint8_t* smem, int k0,
-                           int kr, bool clus, int split) {
+                           int kr, int gsz, bool clus, int split) {
   uint16_t* raw = reinterpret_cast<uint16_t*>(smem + sp.xraw);
   int8_t* xs = reinterpret_cast<int8_t*>(smem + sp.xa);
   unsigned* tmax = reinterpret_cast<unsigned*>(smem + sp.misc);     // [MT], zeroed in the prologue
@@ -170,6 +192,9 @@ __device__ void stage_x_q8(const Gemv2Params& p, const Gemv2Problem& pr, const S
   float* amx = reinterpret_cast<float*>(smem + sp.amx);             // [ks][MT]
   const uint16_t* x = static_cast<const uint16_t*>(pr.x);
   const int m = p.m, K = p.k, nch = kr / 8;
+  float lmax[MT];
+#pragma unroll
+  for (int t = 0; t < MT; ++t) lmax[t] = 0.f;
   for (int i = threadIdx.x; i < MT * nch; i += blockDim.x) {
     const int t = i / nch, c = i - t * nch, k = k0 + 8 * c;
     uint4 v = make_uint4(0, 0, 0, 0);
@@ -186,8 +211,17 @@ __device__ void stage_x_q8(const Gemv2Params& p, const Gemv2Problem& pr, const S
       }
     }
     *reinterpret_cast<uint4*>(raw + t * kr + 8 * c) = v;
-    const float mx = bf16_abs_max8(v);
-    if (mx > 0.f) atomicMax(&tmax[t], __float_as_uint(mx));
+    const float mx8 = bf16_abs_max8(v);
+#pragma unroll
+    for (int u = 0; u < MT; ++u)
+      if (t == u) lmax[u] = fmaxf(lmax[u], mx8);
+  }
+#pragma unroll
+  for (int t = 0; t < MT; ++t) {
+    float mx = lmax[t];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0 && mx > 0.f) atomicMax(&tmax[t], __float_as_uint(mx));
   }
   __syncthreads();
   if (clus) {
@@ -209,24 +243,30 @@ __device__ void stage_x_q8(const Gemv2Params& p, const Gemv2Problem& pr, const S
     inv[t] = a > 0.f ? __fdiv_rn(127.0f, a) : 0.f;
     if (threadIdx.x == 0) sxs[t] = a > 0.f ? __fdiv_rn(a, 127.0f) : 0.f;
   }
-  const int n4 = kr / 4;
-  for (int i = threadIdx.x; i < MT * n4; i += blockDim.x) {
-    const int t = i / n4, c = i - t * n4;
+  const int n16 = kr / 16, gr = (kr + gsz - 1) / gsz;
+  GroupSumAcc acc{reinterpret_cast<int*>(smem + sp.gsum)};
+  for (int i = threadIdx.x; i < MT * n16; i += blockDim.x) {
+    const int t = i / n16, c = i - t * n16;
     float it = inv[0];
 #pragma unroll
     for (int u = 1; u < MT; ++u)
       if (t == u) it = inv[u];
-    const uint2 v = *reinterpret_cast<const uint2*>(raw + t * kr + 4 * c);
-    const uint32_t h[4] = {v.x & 0xFFFFu, v.x >> 16, v.y & 0xFFFFu, v.y >> 16};
-    uint32_t packed = 0;
+    const uint4 v0 = *reinterpret_cast<const uint4*>(raw + t * kr + 16 * c);
+    const uint4 v1 = *reinterpret_cast<const uint4*>(raw + t * kr + 16 * c + 8);
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint32_t packed[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      int q = __float2int_rn(__fmul_rn(__uint_as_float(h[j] << 16), it));
+    for (int j = 0; j < 16; ++j) {
+      const uint32_t h = (j & 1) ? (w[j >> 1] >> 16) : (w[j >> 1] & 0xFFFFu);
+      int q = __float2int_rn(__fmul_rn(__uint_as_float(h << 16), it));
       q = max(-127, min(127, q));
-      packed |= ((uint32_t)q & 0xFFu) << (8 * j);
+      packed[j >> 2] |= ((uint32_t)q & 0xFFu) << (8 * (j & 3));
     }
-    *reinterpret_cast<uint32_t*>(xs + t * kr + 4 * c) = packed;
+    const uint4 pv = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    *reinterpret_cast<uint4*>(xs + t * kr + 16 * c) = pv;
+    acc.add(t * gr + (16 * c) / gsz, sum16_s8(pv));
   }
+  acc.flush();
 }
 
 __device__ void stage_x_bf16(const Gemv2Params& p, const Gemv2Problem& pr, const SmemPlan& sp, uint8_t* smem, int k0,
@@ -292,35 +332,63 @@ __global__ void __launch_bounds__(256) gemv2_kernel(const __grid_constant__ Gemv
   constexpr bool kIntX = XM != kXBf16;
   const SmemPlan sp = smem_plan(p, XM, MT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int pi = 0;
-  while (pi + 1 < p.nprob && (int)blockIdx.x >= p.prob[pi + 1].cta_begin) ++pi;
-  const Gemv2Problem& pr = p.prob[pi];
-  const int T = ((int)blockIdx.x - pr.cta_begin) * p.wpc + warp;
-  const bool active = T < pr.row_tiles;
   const int split = blockIdx.y;
   const bool clus = p.cluster && p.ks > 1;
   const int c0 = split * p.cols_per_split;
   const int c1 = min(p.cols, c0 + p.cols_per_split);
   const int ncols = c1 - c0;
   const int sc = p.stage_cols, nst = p.nstage;
-  const int nstages = (ncols + sc - 1) / sc;
+  const int spt = (ncols + sc - 1) / sc;  // stages per row tile
+  const int m = p.m;
+  const int k0 = c0 * kColK2, kr = ncols * kColK2;
+  const int gr = kTQ ? kr / p.group : 1;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sp.bars) + warp * nst;
   uint8_t* ring = smem + sp.ring + (size_t)warp * nst * sp.stage_bytes;
 
+  // Row groups (wpc consecutive row tiles of one problem) handled by this CTA:
+  // one, or, in a persistent launch (no K split), a contiguous range of them,
+  // so that each warp's weight stream runs on across tile boundaries and the
+  // activations are staged once per problem.
+  int gbeg = blockIdx.x, gend = blockIdx.x + 1;
+  if (p.persistent) {
+    gbeg = (int)((long long)p.groups_total * blockIdx.x / gridDim.x);
+    gend = (int)((long long)p.groups_total * (blockIdx.x + 1) / gridDim.x);
+  }
+  auto prob_of = [&](int gi) {
+    int q = 0;
+    while (q + 1 < p.nprob && gi >= p.prob[q + 1].cta_begin) ++q;
+    return q;
+  };
+  auto tile_of = [&](int gi, int q) { return (gi - p.prob[q].cta_begin) * p.wpc + warp; };
+
   // ---- prologue (independent of the preceding kernel): barriers, first weight stages
   if (clus) cluster_arrive_relaxed();  // DSMEM is used only after every CTA of the cluster runs
-  if (active && lane == 0) {
+  if (lane == 0) {
     for (int s = 0; s < nst; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
   }
-  if (XM == kXBf16Q8 && threadIdx.x < MT) reinterpret_cast<unsigned*>(smem + sp.misc)[threadIdx.x] = 0u;
   __syncwarp();
   const uint64_t pol = policy_evict_first();
-  auto issue = [&](int i) {
-    const int slot = i % nst;
-    const int cs = c0 + i * sc, ce = min(c1, cs + sc);
+  // issue cursor of this warp (used by lane 0): next (row group, stage) to
+  // request, with the problem of that row group tracked incrementally
+  int ig = gbeg, iq = prob_of(gbeg), is_ = 0, nissued = 0, islot = 0;
+  auto cursor_skip_inactive = [&]() {
+    while (ig < gend) {
+      while (iq + 1 < p.nprob && ig >= p.prob[iq + 1].cta_begin) ++iq;
+      if (tile_of(ig, iq) < p.prob[iq].row_tiles) break;
+      ++ig;
+    }
+  };
+  cursor_skip_inactive();
+  auto issue_next = [&]() {
+    if (ig >= gend) return;
+    const Gemv2Problem& pq = p.prob[iq];
+    const int T = tile_of(ig, iq);
+    const int slot = islot;
+    islot = islot + 1 == nst ? 0 : islot + 1;
+    const int cs = c0 + is_ * sc, ce = min(c1, cs + sc);
     const uint32_t tb = (uint32_t)(ce - cs) * P * kPlaneColBytes;
-    const uint8_t* src = pr.trit + ((size_t)T * p.cols + cs) * P * kPlaneColBytes;
+    const uint8_t* src = pq.trit + ((size_t)T * p.cols + cs) * P * kPlaneColBytes;
     uint8_t* dst = ring + (size_t)slot * sp.stage_bytes;
     uint32_t sb = 0;
     int ga = 0;
@@ -333,117 +401,162 @@ __global__ void __launch_bounds__(256) gemv2_kernel(const __grid_constant__ Gemv
     bulk_g2s(dst, src, tb, &bars[slot], pol);
     if (kTQ)
       bulk_g2s(dst + (size_t)sc * P * kPlaneColBytes,
-               reinterpret_cast<const uint8_t*>(pr.scale) + ((size_t)T * p.groups + ga) * P * 64, sb, &bars[slot],
+               reinterpret_cast<const uint8_t*>(pq.scale) + ((size_t)T * p.groups + ga) * P * 64, sb, &bars[slot],
                pol);
+    ++nissued;
+    if (++is_ == spt) {
+      is_ = 0;
+      ++ig;
+      cursor_skip_inactive();
+    }
   };
-  if (active && lane == 0)
-    for (int i = 0; i < min(nst, nstages); ++i) issue(i);
+  if (lane == 0)
+    for (int i = 0; i < nst; ++i) issue_next();
   pdl_launch_dependents();
 
-  // ---- wait for the producer of x, then stage x for this K-split
+  // ---- wait for the producer of x
   pdl_wait();
   if (clus) cluster_wait_acquire();
-  __syncthreads();
-  const int k0 = c0 * kColK2, kr = ncols * kColK2;
-  if (XM == kXInt8) {
-    stage_x_int8<MT>(p, pr, sp, smem, k0, kr);
-    __syncthreads();
-    int8_group_sums<MT>(sp, smem, kr, kTQ ? p.group : kr);
-  } else if (XM == kXBf16Q8) {
-    stage_x_q8<MT>(p, pr, sp, smem, k0, kr, clus, split);
-    __syncthreads();
-    int8_group_sums<MT>(sp, smem, kr, kTQ ? p.group : kr);
-  } else {
-    stage_x_bf16(p, pr, sp, smem, k0, kr);
-  }
-  __syncthreads();
 
-  const int8_t* xs = reinterpret_cast<const int8_t*>(smem + sp.xa);
-  const uint8_t* xmid = smem + sp.xb;
-  const uint8_t* xl = smem + sp.xc;
   const int* gsum = reinterpret_cast<const int*>(smem + sp.gsum);
   const long long* gsum64 = reinterpret_cast<const long long*>(smem + sp.gsum);
   const float* gmul = reinterpret_cast<const float*>(smem + sp.gmult);
-  const int gr = kTQ ? kr / p.group : 1;
-  const int m = p.m;
+  const float* sxs = reinterpret_cast<const float*>(smem + sp.misc) + MT;
 
-  // accumulators: a = fields 0,1 (weight 1), b = fields 2,3 (weight 16)
-  int a[P][MT], b[P][MT];     // int8 x   (or high bytes for bf16)
-  unsigned ma[P], mb[P];      // bf16 middle bytes
-  unsigned la[P], lb[P];      // bf16 low bytes
-  long long acc64[MT];        // TQ int8
-  float yacc = 0.f;           // bf16
+  // Accumulators. After the digit transform a word holds 16 digits F = 1 - t,
+  // four 2-bit fields per byte; field f of every byte lines up with the four
+  // activations x[4f .. 4f+3]. With one token each field is masked in place
+  // (value 4^f * F) and keeps its own accumulator, combined exactly at the end
+  // (acc_f is a multiple of 4^f); with several tokens, fields 1 and 3 are
+  // shifted down first and two accumulators (weights 1 and 16) are kept.
+  constexpr int NF = MT == 1 ? 4 : 2;
+  int acc[P][MT][NF];          // int8 x, or the high bytes of the bf16 image
+  unsigned accm[P][NF];        // bf16 image: middle bytes
+  unsigned accl[P][NF];        // bf16 image: low bytes
+  long long acc64[MT];         // TQ int8: exact sum in units of 2^-24
+  float yacc;                  // bf16
+  auto reset = [&]() {
 #pragma unroll
-  for (int q = 0; q < P; ++q) {
+    for (int q = 0; q < P; ++q)
 #pragma unroll
-    for (int t = 0; t < MT; ++t) a[q][t] = b[q][t] = 0;
-    la[q] = lb[q] = ma[q] = mb[q] = 0;
-  }
+      for (int f = 0; f < NF; ++f) {
 #pragma unroll
-  for (int t = 0; t < MT; ++t) acc64[t] = 0;
-
-  int ifail = -1;
-  if (active) {
-    for (int i = 0; i < nstages; ++i) {
-      const int slot = i % nst;
-      // warp-uniform outcome, so that no lane is left behind at __syncwarp
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[slot], (uint32_t)(i / nst) & 1u))) {
-        ifail = i;
-        break;
+        for (int t = 0; t < MT; ++t) acc[q][t][f] = 0;
+        accm[q][f] = accl[q][f] = 0;
       }
-      const uint8_t* st = ring + (size_t)slot * sp.stage_bytes;
-      const uint16_t* sst = reinterpret_cast<const uint16_t*>(st + (size_t)sc * P * kPlaneColBytes);
-      const int cs = c0 + i * sc;
-      const int ncs = min(sc, c1 - cs);
-      const int ga_stage = kTQ ? cs * kColK2 / p.group : 0;
-      for (int cc = 0; cc < ncs; ++cc) {
-        const int kx = (cs + cc - c0) * kColK2;
-        uint4 wv[P];
 #pragma unroll
-        for (int q = 0; q < P; ++q)
-          wv[q] = *reinterpret_cast<const uint4*>(st + ((size_t)cc * P + q) * kPlaneColBytes + lane * 16);
+    for (int t = 0; t < MT; ++t) acc64[t] = 0;
+    yacc = 0.f;
+  };
+  // sum F*x over the chains
+  auto fold_int = [&](const int* c) -> int {
+    if (NF == 4) return c[0] + (c[1] >> 2) + (c[2] >> 4) + (c[3] >> 6);
+    return c[0] + (c[NF - 1] >> 4);
+  };
+  auto fold_u = [&](const unsigned* c) -> int {
+    if (NF == 4) return (int)(c[0] + (c[1] >> 2) + (c[2] >> 4) + (c[3] >> 6));
+    return (int)(c[0] + (c[NF - 1] >> 4));
+  };
+  // one 16-k word of plane q against the int8 activations of token t
+  auto word_int = [&](int q, int t, uint32_t F, int4 xv) {
+    if (NF == 4) {
+      acc[q][t][0] = dp4a_ss((int)(F & 0x03030303u), xv.x, acc[q][t][0]);
+      acc[q][t][1] = dp4a_ss((int)(F & 0x0C0C0C0Cu), xv.y, acc[q][t][1]);
+      acc[q][t][2] = dp4a_ss((int)(F & 0x30303030u), xv.z, acc[q][t][2]);
+      acc[q][t][NF - 1] = dp4a_us(F & 0xC0C0C0C0u, xv.w, acc[q][t][NF - 1]);
+    } else {
+      const uint32_t F2 = F >> 2;
+      acc[q][t][0] = dp4a_ss((int)(F & kM03), xv.x, acc[q][t][0]);
+      acc[q][t][0] = dp4a_ss((int)(F2 & kM03), xv.y, acc[q][t][0]);
+      acc[q][t][NF - 1] = dp4a_ss((int)(F & kM30), xv.z, acc[q][t][NF - 1]);
+      acc[q][t][NF - 1] = dp4a_ss((int)(F2 & kM30), xv.w, acc[q][t][NF - 1]);
+    }
+  };
+  // one word of plane q against the three bytes of the bf16 image (one token)
+  auto word_bf = [&](int q, uint32_t F, int4 hv, uint4 mv, uint4 lv) {
+    const uint32_t d0 = F & 0x03030303u, d1 = F & 0x0C0C0C0Cu, d2 = F & 0x30303030u, d3 = F & 0xC0C0C0C0u;
+    acc[q][0][0] = dp4a_ss((int)d0, hv.x, acc[q][0][0]);
+    acc[q][0][1] = dp4a_ss((int)d1, hv.y, acc[q][0][1]);
+    acc[q][0][2] = dp4a_ss((int)d2, hv.z, acc[q][0][2]);
+    acc[q][0][NF - 1] = dp4a_us(d3, hv.w, acc[q][0][NF - 1]);
+    accm[q][0] = dp4a_uu(d0, mv.x, accm[q][0]);
+    accm[q][1] = dp4a_uu(d1, mv.y, accm[q][1]);
+    accm[q][2] = dp4a_uu(d2, mv.z, accm[q][2]);
+    accm[q][NF - 1] = dp4a_uu(d3, mv.w, accm[q][NF - 1]);
+    accl[q][0] = dp4a_uu(d0, lv.x, accl[q][0]);
+    accl[q][1] = dp4a_uu(d1, lv.y, accl[q][1]);
+    accl[q][2] = dp4a_uu(d2, lv.z, accl[q][2]);
+    accl[q][NF - 1] = dp4a_uu(d3, lv.w, accl[q][NF - 1]);
+  };
+
+  int cur_prob = -1, nconsumed = 0, ifail = -1, pi = prob_of(gbeg);
+  int cslot = 0;
+  uint32_t cphase = 0;
+  const uint32_t x32 = smem_u32(smem + sp.xa), xm32 = smem_u32(smem + sp.xb), xl32 = smem_u32(smem + sp.xc);
+  const uint32_t ring32 = smem_u32(ring) + lane * 16;
+  for (int gi = gbeg; gi < gend; ++gi) {
+    while (pi + 1 < p.nprob && gi >= p.prob[pi + 1].cta_begin) ++pi;
+    const Gemv2Problem& pr = p.prob[pi];
+    if (pi != cur_prob) {
+      // ---- stage x of this problem for this K-split (once per problem)
+      __syncthreads();
+      if (kIntX)
+        for (int i = threadIdx.x; i < MT * gr; i += blockDim.x) reinterpret_cast<int*>(smem + sp.gsum)[i] = 0;
+      if (XM == kXBf16Q8 && threadIdx.x < MT) reinterpret_cast<unsigned*>(smem + sp.misc)[threadIdx.x] = 0u;
+      __syncthreads();
+      if (XM == kXInt8)
+        stage_x_int8<MT>(p, pr, sp, smem, k0, kr, kTQ ? p.group : kr);
+      else if (XM == kXBf16Q8)
+        stage_x_q8<MT>(p, pr, sp, smem, k0, kr, kTQ ? p.group : kr, clus, split);
+      else
+        stage_x_bf16(p, pr, sp, smem, k0, kr);
+      __syncthreads();
+      cur_prob = pi;
+    }
+    const int T = tile_of(gi, pi);
+    const bool active = T < pr.row_tiles;
+    reset();
+    if (active && ifail < 0) {
+      for (int s = 0; s < spt; ++s, ++nconsumed) {
+        const int slot = cslot;
+        const uint32_t phase = cphase;
+        if (++cslot == nst) {
+          cslot = 0;
+          cphase ^= 1u;
+        }
+        // warp-uniform outcome, so that no lane is left behind at __syncwarp
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[slot], phase))) {
+          ifail = nconsumed;
+          break;
+        }
+        const uint8_t* st = ring + (size_t)slot * sp.stage_bytes;
+        const uint32_t st32 = ring32 + (uint32_t)slot * sp.stage_bytes;
+        const uint16_t* sst = reinterpret_cast<const uint16_t*>(st + (size_t)sc * P * kPlaneColBytes);
+        const int cs = c0 + s * sc;
+        const int ncs = min(sc, c1 - cs);
+        const int ga_stage = kTQ ? cs * kColK2 / p.group : 0;
+        // one 16-k word (index WI of the column) of every plane
+        auto word_step = [&](auto wi_c, const uint4* wv, int cc, int kx) {
+          constexpr int wi = decltype(wi_c)::value;
+          const uint32_t xo = (uint32_t)kx;
+          uint32_t F[P];
 #pragma unroll
-        for (int wi = 0; wi < 4; ++wi) {
-          uint32_t F[P], F2[P];
-#pragma unroll
-          for (int q = 0; q < P; ++q) {
-            const uint32_t w = wi == 0 ? wv[q].x : wi == 1 ? wv[q].y : wi == 2 ? wv[q].z : wv[q].w;
-            F[q] = lop3_ternary_digit(w);
-            F2[q] = F[q] >> 2;
-          }
+          for (int q = 0; q < P; ++q) F[q] = lop3_ternary_digit(u4_get<wi>(wv[q]));
           if (kIntX) {
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
-              if (t < m) {
-                const int4 xv = *reinterpret_cast<const int4*>(xs + t * kr + kx + wi * 16);
+              if (MT == 1 || t < m) {
+                const int4 xv = u4_as_i4(lds128<wi * 16>(x32 + (uint32_t)(t * kr) + xo));
 #pragma unroll
-                for (int q = 0; q < P; ++q) {
-                  a[q][t] = dp4a_ss((int)(F[q] & kM03), xv.x, a[q][t]);
-                  a[q][t] = dp4a_ss((int)(F2[q] & kM03), xv.y, a[q][t]);
-                  b[q][t] = dp4a_ss((int)(F[q] & kM30), xv.z, b[q][t]);
-                  b[q][t] = dp4a_ss((int)(F2[q] & kM30), xv.w, b[q][t]);
-                }
+                for (int q = 0; q < P; ++q) word_int(q, t, F[q], xv);
               }
             }
           } else {
-            const int4 hv = *reinterpret_cast<const int4*>(xs + kx + wi * 16);
-            const uint4 mv = *reinterpret_cast<const uint4*>(xmid + kx + wi * 16);
-            const uint4 lv = *reinterpret_cast<const uint4*>(xl + kx + wi * 16);
+            const int4 hv = u4_as_i4(lds128<wi * 16>(x32 + xo));
+            const uint4 mv = lds128<wi * 16>(xm32 + xo);
+            const uint4 lv = lds128<wi * 16>(xl32 + xo);
 #pragma unroll
-            for (int q = 0; q < P; ++q) {
-              a[q][0] = dp4a_ss((int)(F[q] & kM03), hv.x, a[q][0]);
-              a[q][0] = dp4a_ss((int)(F2[q] & kM03), hv.y, a[q][0]);
-              b[q][0] = dp4a_ss((int)(F[q] & kM30), hv.z, b[q][0]);
-              b[q][0] = dp4a_ss((int)(F2[q] & kM30), hv.w, b[q][0]);
-              ma[q] = dp4a_uu(F[q] & kM03, mv.x, ma[q]);
-              ma[q] = dp4a_uu(F2[q] & kM03, mv.y, ma[q]);
-              mb[q] = dp4a_uu(F[q] & kM30, mv.z, mb[q]);
-              mb[q] = dp4a_uu(F2[q] & kM30, mv.w, mb[q]);
-              la[q] = dp4a_uu(F[q] & kM03, lv.x, la[q]);
-              la[q] = dp4a_uu(F2[q] & kM03, lv.y, la[q]);
-              lb[q] = dp4a_uu(F[q] & kM30, lv.z, lb[q]);
-              lb[q] = dp4a_uu(F2[q] & kM30, lv.w, lb[q]);
-            }
+            for (int q = 0; q < P; ++q) word_bf(q, F[q], hv, mv, lv);
           }
           // ---- group fold (TQ): after the last word of each group
           if constexpr (kTQ) {
@@ -457,95 +570,155 @@ __global__ void __launch_bounds__(256) gemv2_kernel(const __grid_constant__ Gemv
                 if (kIntX) {
 #pragma unroll
                   for (int t = 0; t < MT; ++t) {
-                    if (t < m) {
-                      const int S = gsum[t * gr + gl] - (a[q][t] + (b[q][t] >> 4));
+                    if (MT == 1 || t < m) {
+                      const int S = gsum[t * gr + gl] - fold_int(acc[q][t]);
                       acc64[t] += fold_fp16_exact(h, S);
                     }
-                    a[q][t] = b[q][t] = 0;
+#pragma unroll
+                    for (int f = 0; f < NF; ++f) acc[q][t][f] = 0;
                   }
                 } else {
-                  const int H = a[q][0] + (b[q][0] >> 4);
-                  const int Mi = (int)(ma[q] + (mb[q] >> 4));
-                  const int L = (int)(la[q] + (lb[q] >> 4));
+                  const int H = fold_int(acc[q][0]);
+                  const int Mi = fold_u(accm[q]);
+                  const int L = fold_u(accl[q]);
                   const long long S = gsum64[gl] - ((long long)H * 65536 + (long long)Mi * 256 + L);
                   yacc = fmaf(__half2float(__ushort_as_half(h)) * gmul[gl], __ll2float_rn(S), yacc);
-                  a[q][0] = b[q][0] = 0;
-                  la[q] = lb[q] = ma[q] = mb[q] = 0;
+#pragma unroll
+                  for (int f = 0; f < NF; ++f) acc[q][0][f] = accm[q][f] = accl[q][f] = 0;
                 }
               }
             }
           }
+        };
+        for (int cc = 0; cc < ncs; ++cc) {
+          const int kx = (cs + cc - c0) * kColK2;
+          uint4 wv[P];
+          const uint32_t wc = st32 + (uint32_t)(cc * P * kPlaneColBytes);
+          wv[0] = lds128<0>(wc);
+          if constexpr (P > 1) wv[1] = lds128<kPlaneColBytes>(wc);
+          if constexpr (P > 2) wv[2] = lds128<2 * kPlaneColBytes>(wc);
+          if constexpr (P > 3) wv[3] = lds128<3 * kPlaneColBytes>(wc);
+          word_step(std::integral_constant<int, 0>{}, wv, cc, kx);
+          word_step(std::integral_constant<int, 1>{}, wv, cc, kx);
+          word_step(std::integral_constant<int, 2>{}, wv, cc, kx);
+          word_step(std::integral_constant<int, 3>{}, wv, cc, kx);
+        }
+        // release the slot: reads of this stage are complete before the refill
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) issue_next();
+      }
+    }
+
+    // ---- epilogue of this row tile: per-lane results (int32 BitNet / int64 TQ-int8 / fp32 bf16)
+    const int npad = pr.row_tiles * kTileRows;
+    const int row = T * kTileRows + lane;
+    int accb[MT];
+    if (!kTQ) {
+#pragma unroll
+      for (int t = 0; t < MT; ++t) accb[t] = (MT == 1 || t < m) ? gsum[t] - fold_int(acc[0][t]) : 0;
+    }
+    auto write_out = [&](int t, float v) {
+      if (p.out_bf16)
+        reinterpret_cast<__nv_bfloat16*>(pr.y)[(size_t)t * pr.n + row] = __float2bfloat16_rn(v);
+      else
+        reinterpret_cast<float*>(pr.y)[(size_t)t * pr.n + row] = v;
+    };
+    auto finish = [&](int t, long long v64, int v32, float vf) {
+      if (row >= pr.n) return;
+      const float sx = XM == kXBf16Q8 ? sxs[t] : (XM == kXInt8 ? pr.xscale[t] : 0.f);
+      if (XM == kXBf16) {
+        write_out(t, vf);
+      } else if (kTQ) {
+        const float sv = __fmul_rn(__ll2float_rn(v64), 0x1p-24f);
+        write_out(t, __fmul_rn(sv, sx));
+      } else {
+        write_out(t, __fmul_rn(__fmul_rn(__int2float_rn(v32), pr.tensor_scale), sx));
+      }
+    };
+
+    if (p.ks == 1) {
+      if (active) {
+#pragma unroll
+        for (int t = 0; t < MT; ++t)
+          if (t < m) finish(t, acc64[t], kTQ ? 0 : accb[t], yacc);
+      }
+      continue;
+    }
+
+    // ---- K is split (one row group per CTA): combine the splits' partial sums
+    if (active && ifail >= 0) {
+      // a wait expired: give the copies still in flight a bounded chance to land
+      for (int j = ifail; j < min(nissued, ifail + nst); ++j)
+        mbar_wait_bounded(&bars[j % nst], (uint32_t)(j / nst) & 1u);  // error path only
+    }
+    if (clus) {
+      // the splits of this row group form the cluster: reduce in CTA rank 0
+      const int rows_cta = p.wpc * kTileRows;
+      const int esz = red_elem(XM, kTQ);
+      if (active) {
+#pragma unroll
+        for (int t = 0; t < MT; ++t) {
+          if (t >= m) continue;
+          const size_t idx = ((size_t)split * MT + t) * rows_cta + warp * kTileRows + lane;
+          const uint32_t dst = map_cluster_rank(smem_u32(smem + sp.red + idx * esz), 0);
+          if (XM == kXBf16)
+            st_cluster_u32(dst, __float_as_uint(yacc));
+          else if (kTQ)
+            st_cluster_u64(dst, (unsigned long long)acc64[t]);
+          else
+            st_cluster_u32(dst, (uint32_t)accb[t]);
         }
       }
-      // release the slot: reads of this stage are complete before the refill
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0 && i + nst < nstages) issue(i + nst);
-    }
-  }
-  if (active && ifail >= 0) {
-    // a wait expired: give the copies still in flight a bounded chance to land
-    for (int j = ifail; j < min(nstages, ifail + nst); ++j) mbar_wait_bounded(&bars[j % nst], (uint32_t)(j / nst) & 1u);
-  }
-
-  // ---- epilogue: per-lane row results (int32 BitNet / int64 TQ-int8 / fp32 bf16)
-  const int npad = pr.row_tiles * kTileRows;
-  const int row = T * kTileRows + lane;
-  int accb[MT];
-  if (!kTQ) {
+      cluster_sync();
+      if (split == 0 && active) {
 #pragma unroll
-    for (int t = 0; t < MT; ++t) accb[t] = (t < m) ? gsum[t] - (a[0][t] + (b[0][t] >> 4)) : 0;
-  }
-  const float* sxs = reinterpret_cast<const float*>(smem + sp.misc) + MT;
-
-  auto write_out = [&](int t, float v) {
-    if (p.out_bf16)
-      reinterpret_cast<__nv_bfloat16*>(pr.y)[(size_t)t * pr.n + row] = __float2bfloat16_rn(v);
-    else
-      reinterpret_cast<float*>(pr.y)[(size_t)t * pr.n + row] = v;
-  };
-  auto finish = [&](int t, long long v64, int v32, float vf) {
-    if (row >= pr.n) return;
-    const float sx = XM == kXBf16Q8 ? sxs[t] : (XM == kXInt8 ? pr.xscale[t] : 0.f);
-    if (XM == kXBf16) {
-      write_out(t, vf);
-    } else if (kTQ) {
-      const float s = __fmul_rn(__ll2float_rn(v64), 0x1p-24f);
-      write_out(t, __fmul_rn(s, sx));
-    } else {
-      write_out(t, __fmul_rn(__fmul_rn(__int2float_rn(v32), pr.tensor_scale), sx));
+        for (int t = 0; t < MT; ++t) {
+          if (t >= m) continue;
+          long long s64 = 0;
+          int s32 = 0;
+          float sf = 0.f;
+          for (int s = 0; s < p.ks; ++s) {
+            const size_t idx = ((size_t)s * MT + t) * rows_cta + warp * kTileRows + lane;
+            if (XM == kXBf16)
+              sf += reinterpret_cast<const float*>(smem + sp.red)[idx];
+            else if (kTQ)
+              s64 += reinterpret_cast<const long long*>(smem + sp.red)[idx];
+            else
+              s32 += reinterpret_cast<const int*>(smem + sp.red)[idx];
+          }
+          finish(t, s64, s32, sf);
+        }
+      }
+      return;
     }
-  };
 
-  if (p.ks == 1) {
-    if (active) {
-#pragma unroll
-      for (int t = 0; t < MT; ++t)
-        if (t < m) finish(t, acc64[t], kTQ ? 0 : accb[t], yacc);
-    }
-    return;
-  }
-
-  if (clus) {
-    // ---- K-splits of this row group form the cluster: reduce in CTA rank 0
-    const int rows_cta = p.wpc * kTileRows;
-    const int esz = red_elem(XM, kTQ);
-    if (active) {
+    // more splits than a cluster holds: partials through the global workspace,
+    // reduced by the last CTA of this row group to arrive
+    if (active && row < npad) {
 #pragma unroll
       for (int t = 0; t < MT; ++t) {
         if (t >= m) continue;
-        const size_t idx = ((size_t)split * MT + t) * rows_cta + warp * kTileRows + lane;
-        const uint32_t dst = map_cluster_rank(smem_u32(smem + sp.red + idx * esz), 0);
+        const size_t idx = ((size_t)split * m + t) * npad + row;
         if (XM == kXBf16)
-          st_cluster_u32(dst, __float_as_uint(yacc));
+          reinterpret_cast<float*>(p.ws_part)[idx] = yacc;
         else if (kTQ)
-          st_cluster_u64(dst, (unsigned long long)acc64[t]);
+          reinterpret_cast<long long*>(p.ws_part)[idx] = acc64[t];
         else
-          st_cluster_u32(dst, (uint32_t)accb[t]);
+          reinterpret_cast<int*>(p.ws_part)[idx] = accb[t];
       }
     }
-    cluster_sync();
-    if (split == 0 && active) {
+    __threadfence();
+    __syncthreads();
+    int* flag = reinterpret_cast<int*>(smem + sp.misc) + 2 * MT;
+    if (threadIdx.x == 0) {
+      const unsigned prev = atomicAdd(&p.ws_cnt[blockIdx.x], 1u);
+      *flag = (prev == (unsigned)(p.ks - 1));
+    }
+    __syncthreads();
+    if (!*flag) return;
+    __threadfence();
+    if (active) {
 #pragma unroll
       for (int t = 0; t < MT; ++t) {
         if (t >= m) continue;
@@ -553,65 +726,24 @@ __global__ void __launch_bounds__(256) gemv2_kernel(const __grid_constant__ Gemv
         int s32 = 0;
         float sf = 0.f;
         for (int s = 0; s < p.ks; ++s) {
-          const size_t idx = ((size_t)s * MT + t) * rows_cta + warp * kTileRows + lane;
+          const size_t idx = ((size_t)s * m + t) * npad + row;
           if (XM == kXBf16)
-            sf += reinterpret_cast<const float*>(smem + sp.red)[idx];
+            sf += __ldcg(reinterpret_cast<const float*>(p.ws_part) + idx);
           else if (kTQ)
-            s64 += reinterpret_cast<const long long*>(smem + sp.red)[idx];
+            s64 += __ldcg(reinterpret_cast<const long long*>(p.ws_part) + idx);
           else
-            s32 += reinterpret_cast<const int*>(smem + sp.red)[idx];
+            s32 += __ldcg(reinterpret_cast<const int*>(p.ws_part) + idx);
         }
         finish(t, s64, s32, sf);
       }
     }
+    if (threadIdx.x == 0) p.ws_cnt[blockIdx.x] = 0u;  // leave the counters at zero
     return;
   }
-
-  // ---- more splits than a cluster holds: partials through the global workspace,
-  // reduced by the last CTA of this row group to arrive
-  if (active && row < npad) {
-#pragma unroll
-    for (int t = 0; t < MT; ++t) {
-      if (t >= m) continue;
-      const size_t idx = ((size_t)split * m + t) * npad + row;
-      if (XM == kXBf16)
-        reinterpret_cast<float*>(p.ws_part)[idx] = yacc;
-      else if (kTQ)
-        reinterpret_cast<long long*>(p.ws_part)[idx] = acc64[t];
-      else
-        reinterpret_cast<int*>(p.ws_part)[idx] = accb[t];
-    }
+  if (ifail >= 0) {
+    // a wait expired: give the copies still in flight a bounded chance to land
+    for (int j = ifail; j < min(nissued, ifail + nst); ++j) mbar_wait_bounded(&bars[j % nst], (uint32_t)(j / nst) & 1u);
   }
-  __threadfence();
-  __syncthreads();
-  int* flag = reinterpret_cast<int*>(smem + sp.misc) + 2 * MT;
-  if (threadIdx.x == 0) {
-    const unsigned prev = atomicAdd(&p.ws_cnt[blockIdx.x], 1u);
-    *flag = (prev == (unsigned)(p.ks - 1));
-  }
-  __syncthreads();
-  if (!*flag) return;
-  __threadfence();
-  if (active) {
-#pragma unroll
-    for (int t = 0; t < MT; ++t) {
-      if (t >= m) continue;
-      long long s64 = 0;
-      int s32 = 0;
-      float sf = 0.f;
-      for (int s = 0; s < p.ks; ++s) {
-        const size_t idx = ((size_t)s * m + t) * npad + row;
-        if (XM == kXBf16)
-          sf += __ldcg(reinterpret_cast<const float*>(p.ws_part) + idx);
-        else if (kTQ)
-          s64 += __ldcg(reinterpret_cast<const long long*>(p.ws_part) + idx);
-        else
-          s32 += __ldcg(reinterpret_cast<const int*>(p.ws_part) + idx);
-      }
-      finish(t, s64, s32, sf);
-    }
-  }
-  if (threadIdx.x == 0) p.ws_cnt[blockIdx.x] = 0u;  // leave the counters at zero
 }
 
 // ------------------------------------------------------------------ launch
@@ -634,8 +766,25 @@ static int launch_one(const Gemv2Params& p, bool pdl, void* stream) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return (int)e;
   }
+  // without a K split, run at most as many CTAs as fit at once; each then
+  // walks a contiguous range of row groups
+  Gemv2Params q = p;
+  q.groups_total = p.grid_x;
+  q.persistent = 0;
+  int gx = p.grid_x;
+  if (p.ks == 1) {
+    int dev = 0, sms = 0, occ = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * p.wpc, sp.total);
+    if (e != cudaSuccess) return (int)e;
+    if (occ > 0 && gx > sms * occ) {
+      gx = sms * occ;
+      q.persistent = 1;
+    }
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.grid_x, p.ks, 1);
+  cfg.gridDim = dim3(gx, p.ks, 1);
   cfg.blockDim = dim3(32 * p.wpc, 1, 1);
   cfg.dynamicSmemBytes = sp.total;
   cfg.stream = static_cast<cudaStream_t>(stream);
@@ -655,50 +804,57 @@ static int launch_one(const Gemv2Params& p, bool pdl, void* stream) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  e = cudaLaunchKernelEx(&cfg, kern, p);
+  e = cudaLaunchKernelEx(&cfg, kern, q);
   return (int)e;
 }
 
 // Instantiated combinations; anything else reports "unsupported" (-1).
+// Planes x group: TQ with 1-4 planes at g = 256 and the fine-group variants
+// of the workloads (2 planes at g = 32, 3 planes at g = 64); BitNet one plane.
+#define TERN_TQ_CASES(XM, MT)                                                    \
+  switch (p.planes * 100 + wg) {                                                \
+    case 116: return launch_one<XM, 1, 16, MT>(p, pdl, stream);                 \
+    case 216: return launch_one<XM, 2, 16, MT>(p, pdl, stream);                 \
+    case 316: return launch_one<XM, 3, 16, MT>(p, pdl, stream);                 \
+    case 416: return launch_one<XM, 4, 16, MT>(p, pdl, stream);                 \
+    case 202: return launch_one<XM, 2, 2, MT>(p, pdl, stream);                  \
+    case 304: return launch_one<XM, 3, 4, MT>(p, pdl, stream);                  \
+    default: return -1;                                                         \
+  }
+
 int launch_gemv2(const Gemv2Params& p, int xmode, bool pdl, void* stream) {
   const bool tq = p.tq != 0;
   const int wg = tq ? p.group / 16 : 0;
   const int mt = gemv2_mt(xmode, p.m);
-  if (xmode == kXInt8) {
-    if (!tq && p.planes == 1) {
+  if (!tq) {
+    if (p.planes != 1) return -1;
+    if (xmode == kXInt8) {
       if (mt == 1) return launch_one<kXInt8, 1, 0, 1>(p, pdl, stream);
       if (mt == 4) return launch_one<kXInt8, 1, 0, 4>(p, pdl, stream);
       return launch_one<kXInt8, 1, 0, 16>(p, pdl, stream);
     }
-    if (tq && p.planes == 2 && wg == 2) {
-      if (mt == 1) return launch_one<kXInt8, 2, 2, 1>(p, pdl, stream);
-      if (mt == 4) return launch_one<kXInt8, 2, 2, 4>(p, pdl, stream);
-      return launch_one<kXInt8, 2, 2, 16>(p, pdl, stream);
-    }
-    if (tq && p.planes == 3 && wg == 16 && mt == 1) return launch_one<kXInt8, 3, 16, 1>(p, pdl, stream);
-    return -1;
-  }
-  if (xmode == kXBf16Q8) {
-    if (!tq && p.planes == 1) {
+    if (xmode == kXBf16Q8) {
       if (mt == 1) return launch_one<kXBf16Q8, 1, 0, 1>(p, pdl, stream);
       return launch_one<kXBf16Q8, 1, 0, 4>(p, pdl, stream);
     }
-    if (tq && p.planes == 2 && wg == 2) {
-      if (mt == 1) return launch_one<kXBf16Q8, 2, 2, 1>(p, pdl, stream);
-      return launch_one<kXBf16Q8, 2, 2, 4>(p, pdl, stream);
+    return -1;
+  }
+  if (xmode == kXInt8) {
+    if (mt == 1) TERN_TQ_CASES(kXInt8, 1)
+    if (p.planes == 2 && wg == 2) {
+      if (mt == 4) return launch_one<kXInt8, 2, 2, 4>(p, pdl, stream);
+      return launch_one<kXInt8, 2, 2, 16>(p, pdl, stream);
     }
     return -1;
   }
-  if (!tq || p.m != 1) return -1;
-  switch (p.planes * 100 + wg) {
-    case 116: return launch_one<kXBf16, 1, 16, 1>(p, pdl, stream);
-    case 216: return launch_one<kXBf16, 2, 16, 1>(p, pdl, stream);
-    case 316: return launch_one<kXBf16, 3, 16, 1>(p, pdl, stream);
-    case 416: return launch_one<kXBf16, 4, 16, 1>(p, pdl, stream);
-    case 202: return launch_one<kXBf16, 2, 2, 1>(p, pdl, stream);
-    case 304: return launch_one<kXBf16, 3, 4, 1>(p, pdl, stream);
-    default: return -1;
+  if (xmode == kXBf16Q8) {
+    if (mt == 1) TERN_TQ_CASES(kXBf16Q8, 1)
+    if (p.planes == 2 && wg == 2) return launch_one<kXBf16Q8, 2, 2, 4>(p, pdl, stream);
+    return -1;
   }
+  if (p.m != 1) return -1;
+  TERN_TQ_CASES(kXBf16, 1)
 }
+#undef TERN_TQ_CASES
 
 }  // namespace tern

@@ -55,7 +55,9 @@ struct Gemv2Problem {
 struct Gemv2Params {
   Gemv2Problem prob[kMaxProblems];
   int nprob;
-  int grid_x;               // sum over problems of ceil(row_tiles / wpc)
+  int grid_x;               // sum over problems of ceil(row_tiles / wpc): the row groups
+  int groups_total;         // set at launch: row groups in all problems
+  int persistent;           // set at launch: CTAs walk ranges of row groups (no K split)
   int tq;                   // fp16 group scales (TQ) rather than one per-tensor scale
   int k, planes, group, groups, cols;   // shared by all problems
   int m;                    // tokens
@@ -76,6 +78,9 @@ int launch_gemv2(const Gemv2Params& p, int xmode, bool pdl, void* stream);  // -
 int launch_quantize(const uint16_t* x, int m, int k, int8_t* xq, float* xs, void* stream);
 
 int read_clear_dev_error_gemv2(void* stream, unsigned* out);
+int read_clear_dev_error_stream(void* stream, unsigned* out);
+int launch_stream_read(const void* src, size_t bytes, int mode, int chunk, int depth, int ctas_per_sm, int warps,
+                       unsigned* sink, void* stream);
 
 // Shared-memory bytes a 2-bit GEMV CTA needs for these parameters.
 size_t gemv2_smem_bytes(const Gemv2Params& p, int xmode);

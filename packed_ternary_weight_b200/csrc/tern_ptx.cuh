@@ -67,14 +67,17 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
       : "memory");
 }
 
+// One potentially blocking test of the phase: the thread may be suspended
+// for up to about 0.5 ms waiting for the phase to complete (so a waiting warp
+// does not spin on the issue slots).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(500000u)
       : "memory");
   return ok != 0;
 }
@@ -92,10 +95,13 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
+  // back off between tests so that waiting warps leave the issue slots to the
+  // warps that have data; check the time limit only now and then
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 0;; ++it) {
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(it < 4 ? 32u : 128u);
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 63u && global_timer_ns() - t0 > kWaitLimitNs) {
+    if ((it & 63u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
       atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
       return false;
     }
@@ -139,9 +145,26 @@ __device__ __forceinline__ void st_cluster_u64(uint32_t addr, unsigned long long
   asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
 }
 
+// 16-byte shared-memory loads from a 32-bit shared address plus an immediate offset.
+template <int OFF>
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4+%5];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr), "n"(OFF));
+  return v;
+}
+__device__ __forceinline__ int4 u4_as_i4(uint4 v) { return make_int4((int)v.x, (int)v.y, (int)v.z, (int)v.w); }
+
 // Four-way byte dot products with 32-bit accumulation.
 __device__ __forceinline__ int dp4a_ss(int a, int b, int c) { return __dp4a(a, b, c); }
 __device__ __forceinline__ unsigned dp4a_uu(unsigned a, unsigned b, unsigned c) { return __dp4a(a, b, c); }
+// unsigned bytes of a times signed bytes of b
+__device__ __forceinline__ int dp4a_us(uint32_t a, int b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
 
 __device__ __forceinline__ uint32_t lop3_ternary_digit(uint32_t w) {
   // Per 2-bit field with code c (00 -> 0, 01 -> +1, 10 -> -1) produce the

@@ -53,10 +53,13 @@ lib.tern_gemm_batched.argtypes = [ctypes.POINTER(Desc), _vp, ctypes.c_int32, cty
                                   _vp, _vp, _sz, _vp]
 lib.tern_device_error.argtypes = [_vp]
 lib.tern_gemv_noalloc.argtypes = [ctypes.POINTER(Desc), _vp, ctypes.c_int, _vp, _vp, ctypes.c_int, _vp, _vp]
+lib.tern_stream_read.argtypes = [_vp, _sz, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                 ctypes.c_int32, _vp, _vp]
 lib.tern_gemv_grouped.argtypes = [ctypes.c_int32, ctypes.POINTER(Desc), ctypes.POINTER(_vp), ctypes.c_int,
                                   ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.c_int, ctypes.POINTER(_vp), _vp]
 for _f in (lib.tern_packed_size, lib.tern_pack, lib.tern_workspace_size, lib.tern_quantize_act, lib.tern_gemv,
-           lib.tern_gemm_batched, lib.tern_device_error, lib.tern_gemv_noalloc, lib.tern_gemv_grouped):
+           lib.tern_gemm_batched, lib.tern_device_error, lib.tern_gemv_noalloc, lib.tern_gemv_grouped,
+           lib.tern_stream_read):
     _f.restype = ctypes.c_int
 
 
@@ -171,6 +174,12 @@ def gemv_noalloc(desc: Desc, packed, act: int, x, xscale, out: int, y, stream=No
     """tern_gemv with the library's fixed device scratch instead of a caller workspace."""
     _check(lib.tern_gemv_noalloc(ctypes.byref(desc), _ptr(packed), act, _ptr(x), _ptr(xscale), out, _ptr(y),
                                  _stream(stream)), "tern_gemv_noalloc")
+
+
+def stream_read(src, mode: int, chunk: int, depth: int, ctas_per_sm: int, warps: int, sink, stream=None):
+    """Read-ceiling kernel: stream all of `src` once with the given access shape."""
+    _check(lib.tern_stream_read(_ptr(src), src.numel() * src.element_size(), mode, chunk, depth, ctas_per_sm, warps,
+                                _ptr(sink), _stream(stream)), "tern_stream_read")
 
 
 def device_error(stream=None) -> int:
