@@ -35,7 +35,7 @@ struct Plan2 {
 };
 
 // Launch plan of the 2-bit GEMV for problems that share K and format.
-//  * K is split into `ks` ranges of whole scale groups so that about four
+//  * K is split into `ks` ranges of whole scale groups so that about twelve
 //    warps per SM have work (small layers are latency-bound; splitting K
 //    spreads their bytes over all SMs), and so that the staged activations of
 //    one split fit in shared memory;
@@ -54,7 +54,7 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
   for (int i = 0; i < nprob; ++i) rt_total += row_tiles[i];
   pl.wpc = 4;
   const int sc_target = std::max(gc, (4096 / (P * kPlaneColBytes)) / gc * gc);
-  const int ks_par = std::min(units, std::max(1, (4 * sms + rt_total - 1) / rt_total));
+  const int ks_par = std::min(units, std::max(1, (12 * sms + rt_total - 1) / rt_total));
   const int bpk = xmode == kXInt8 ? mt : xmode == kXBf16Q8 ? 3 * mt : 3;  // staged bytes per k
   int ks_x = 1;
   while (ks_x < units && (size_t)((units + ks_x - 1) / ks_x) * gc * kColK2 * bpk > 96 * 1024) ++ks_x;
