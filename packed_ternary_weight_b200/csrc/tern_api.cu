@@ -46,27 +46,34 @@ struct Plan2 {
 Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xmode, int sms, bool ws_ok) {
   Plan2 pl{};
   const bool tq = L.fmt == TERN_FMT_TQ;
+  const bool bt3 = L.fmt == TERN_FMT_BT3;
   const int gc = (tq && L.group >= 64) ? L.group / 64 : 1;  // columns per group
   const int units = (L.cols + gc - 1) / gc;
   const int P = L.planes;
+  const int colk = bt3 ? kColK3 : kColK2;                      // k per column
+  const int colb = bt3 ? kBt3ColBytes : P * kPlaneColBytes;   // bytes per column of a row tile
   const int mt = gemv2_mt(xmode, m);
   int rt_total = 0;
   for (int i = 0; i < nprob; ++i) rt_total += row_tiles[i];
   pl.wpc = 4;
-  const int sc_target = std::max(gc, (4096 / (P * kPlaneColBytes)) / gc * gc);
+  const int sc_target = std::max(gc, (4096 / colb) / gc * gc);
   const int ks_par = std::min(units, std::max(1, (12 * sms + rt_total - 1) / rt_total));
   const int bpk = xmode == kXInt8 ? mt : xmode == kXBf16Q8 ? 3 * mt : 3;  // staged bytes per k
   int ks_x = 1;
-  while (ks_x < units && (size_t)((units + ks_x - 1) / ks_x) * gc * kColK2 * bpk > 96 * 1024) ++ks_x;
+  while (ks_x < units && (size_t)((units + ks_x - 1) / ks_x) * gc * colk * bpk > 96 * 1024) ++ks_x;
   int ks = std::max(ks_par, ks_x);
   const size_t elem = (xmode != kXBf16 && tq) ? 8 : 4;
+  if (bt3 && ks_x > kMaxCluster) {
+    pl.ok = false;
+    return pl;
+  }
   if (ks > kMaxCluster && ks_x <= kMaxCluster) ks = kMaxCluster;
   pl.cluster = 0;
   if (ks > 1 && ks <= kMaxCluster) {
     while ((size_t)ks * mt * pl.wpc * 32 * elem > 32 * 1024 && pl.wpc > 1) pl.wpc /= 2;
     if ((size_t)ks * mt * pl.wpc * 32 * elem <= 32 * 1024) pl.cluster = 1;
   }
-  if (ks > 1 && !pl.cluster && (!ws_ok || nprob != 1 || xmode == kXBf16Q8)) {
+  if (ks > 1 && !pl.cluster && (!ws_ok || nprob != 1 || xmode == kXBf16Q8 || bt3)) {
     pl.ok = false;
     return pl;
   }
@@ -91,7 +98,7 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
     t.wpc = pl.wpc;
     t.stage_cols = pl.stage_cols;
     t.nstage = pl.nstage;
-    if (gemv2_smem_bytes(t, xmode) <= 227 * 1024) break;
+    if ((bt3 ? gemv3_smem_bytes(t) : gemv2_smem_bytes(t, xmode)) <= 227 * 1024) break;
     if (pl.nstage > 2) {
       --pl.nstage;
     } else if (pl.wpc > 1) {
@@ -124,10 +131,10 @@ tern_status check_one(const tern_desc* desc, const void* d_packed, tern_act act,
   return TERN_OK;
 }
 
-// What the 2-bit kernels support for this layout and activation mode.
+// What the kernels support for this layout and activation mode.
 tern_status supported_2bit(const Layout& L, int xmode) {
   const bool tq = L.fmt == TERN_FMT_TQ;
-  if (L.fmt == TERN_FMT_BT3) return TERN_EUNSUPPORTED;
+  if (L.fmt == TERN_FMT_BT3) return xmode == kXBf16 ? TERN_OK : TERN_EUNSUPPORTED;
   if (xmode == kXBf16 && !tq) return TERN_EUNSUPPORTED;
   if (tq && L.k % kColK2 != 0) return TERN_EUNSUPPORTED;
   if (!tq && (long long)L.k * 127 >= (1ll << 24)) return TERN_EUNSUPPORTED;  // exact int32 -> fp32
@@ -188,8 +195,8 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
       p.ws_cnt = static_cast<unsigned*>(d_ws);
       p.ws_part = static_cast<uint8_t*>(d_ws) + pl.ws_cnt_bytes;
     }
-    if (gemv2_smem_bytes(p, xmode) > 227 * 1024) return TERN_EUNSUPPORTED;
-    const int rc = launch_gemv2(p, xmode, (desc->flags & TERN_F_PDL) != 0, stream);
+    const bool pdl = (desc->flags & TERN_F_PDL) != 0;
+    const int rc = L.fmt == TERN_FMT_BT3 ? launch_gemv3(p, pdl, stream) : launch_gemv2(p, xmode, pdl, stream);
     if (rc < 0) return TERN_EUNSUPPORTED;
     if (rc != 0) return TERN_ECUDA;
   }
@@ -285,8 +292,8 @@ extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, 
     vec = vec && aligned16(q.x);
   }
   p.x_vec = vec;
-  if (gemv2_smem_bytes(p, xmode) > 227 * 1024) return TERN_EUNSUPPORTED;
-  const int rc = launch_gemv2(p, xmode, (descs[0].flags & TERN_F_PDL) != 0, stream);
+  const bool pdl = (descs[0].flags & TERN_F_PDL) != 0;
+  const int rc = L[0].fmt == TERN_FMT_BT3 ? launch_gemv3(p, pdl, stream) : launch_gemv2(p, xmode, pdl, stream);
   if (rc < 0) return TERN_EUNSUPPORTED;
   return rc == 0 ? TERN_OK : TERN_ECUDA;
 }
@@ -295,6 +302,7 @@ extern "C" tern_status tern_device_error(void* stream) {
   unsigned v = 0;
   if (read_clear_dev_error_gemv2(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_stream(stream, &v) != 0) return TERN_ECUDA;
+  if (read_clear_dev_error_gemv3(stream, &v) != 0) return TERN_ECUDA;
   return v ? TERN_ETIMEOUT : TERN_OK;
 }
 

@@ -50,6 +50,7 @@
 
 #include <type_traits>
 
+#include "tern_gemv_common.cuh"
 #include "tern_ptx.cuh"
 
 namespace tern {
@@ -66,15 +67,8 @@ struct SmemPlan {
   int stage_bytes;
 };
 
-__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
-
-template <int I>
-__device__ __forceinline__ uint32_t u4_get(const uint4& v) {
-  if constexpr (I == 0) return v.x;
-  if constexpr (I == 1) return v.y;
-  if constexpr (I == 2) return v.z;
-  return v.w;
-}
+using gemv_common::align_up;
+using gemv_common::u4_get;
 
 __host__ __device__ inline int red_elem(int xmode, bool tq) { return (xmode != kXBf16 && tq) ? 8 : 4; }
 
@@ -271,45 +265,9 @@ __device__ void stage_x_q8(const Gemv2Params& p, const Gemv2Problem& pr, const S
 
 __device__ void stage_x_bf16(const Gemv2Params& p, const Gemv2Problem& pr, const SmemPlan& sp, uint8_t* smem, int k0,
                              int kr) {
-  int8_t* xh = reinterpret_cast<int8_t*>(smem + sp.xa);
-  uint8_t* xm = smem + sp.xb;
-  uint8_t* xl = smem + sp.xc;
-  long long* gs = reinterpret_cast<long long*>(smem + sp.gsum);
-  float* gm = reinterpret_cast<float*>(smem + sp.gmult);
-  const uint16_t* x = static_cast<const uint16_t*>(pr.x);
-  const int g = p.group, gr = kr / g;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  for (int grp = warp; grp < gr; grp += nw) {
-    const int kb = grp * g;
-    float amax = 0.f;
-    for (int kk = kb + lane; kk < kb + g; kk += 32) {
-      const int k = k0 + kk;
-      const float v = k < p.k ? __uint_as_float((uint32_t)x[k] << 16) : 0.f;
-      amax = fmaxf(amax, fabsf(v));
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const int e = amax > 0.f ? ilogbf(amax) : 0;
-    // multiply by 2^(22-e) in at most two exact power-of-two steps
-    const int sh = 22 - e;
-    const float up1 = ldexpf(1.0f, sh > 100 ? 100 : sh), up2 = ldexpf(1.0f, sh > 100 ? sh - 100 : 0);
-    long long s = 0;
-    for (int kk = kb + lane; kk < kb + g; kk += 32) {
-      const int k = k0 + kk;
-      const float v = k < p.k ? __uint_as_float((uint32_t)x[k] << 16) : 0.f;
-      const int q = __float2int_rn(__fmul_rn(__fmul_rn(v, up1), up2));  // |q| < 2^23
-      s += q;
-      xh[kk] = (int8_t)(q >> 16);
-      xm[kk] = (uint8_t)((q >> 8) & 0xFF);
-      xl[kk] = (uint8_t)(q & 0xFF);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    if (lane == 0) {
-      gs[grp] = s;
-      gm[grp] = amax > 0.f ? ldexpf(1.0f, e - 22) : 0.f;
-    }
-  }
+  gemv_common::stage_x_bf16_image(static_cast<const uint16_t*>(pr.x), p.k, p.group, k0, kr,
+                                  reinterpret_cast<int8_t*>(smem + sp.xa), smem + sp.xb, smem + sp.xc,
+                                  reinterpret_cast<long long*>(smem + sp.gsum), reinterpret_cast<float*>(smem + sp.gmult));
 }
 
 // Exact fold of an fp16 scale times an integer group sum into a count of 2^-24.

@@ -1,0 +1,361 @@
+// Decode GEMV over balanced ternary of depth 3 (Entrit Llama-3.1-8B-trit-uniform-d3
+// card, "Quantization details": 27 levels per weight, group 16, 27-entry
+// log-spaced scale codebook; weight = cb[idx] * (9 t2 + 3 t1 + t0)), bf16
+// activations.
+//
+// Layout of one 80-k column of a 32-row tile (the packer's): three digit
+// planes of 16 bytes per row, byte i holding the digits u = t + 1 of
+// k = 80c + 16j + i as its base-3 digit j (j = 0..4), then three bytes per row
+// holding the base-3 digits of the five groups' codebook indices. Digit j of
+// the 16 bytes of a row is exactly group 5c + j.
+//
+// Work split, weight stream, K-splits and persistence follow the 2-bit kernel:
+// one warp per 32-row tile and K-split, per-warp rings of shared-memory stages
+// filled by 1-D bulk async copies on mbarriers, splits reduced in a
+// thread-block cluster, persistent CTAs when K is not split.
+//
+// Decode (per lane = one row, per 4 bytes of a plane): the bytes are spread
+// into two 16-bit lanes each and their five digits extracted with the exact
+// reciprocal floor(v / 3) = (171 v) >> 9 (v <= 242), both lanes at once.
+// U = u0 + 3 u1 + 9 u2 = level + 13 in 0..26 is formed in byte lanes and
+// dotted with the 24-bit fixed-point image of the activations (same as the
+// 2-bit bf16 path) with byte dot-products, so the group sum is
+// sum U q - 13 sum q, exact in integers; each group is then scaled once,
+// cb[idx] * 2^(E-22), and accumulated in fp32.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <type_traits>
+
+#include "tern_gemv_common.cuh"
+#include "tern_ptx.cuh"
+
+namespace tern {
+
+int read_clear_dev_error_gemv3(void* stream, unsigned* out) { return read_clear_dev_error_tu(stream, out); }
+
+namespace {
+
+using gemv_common::align_up;
+
+struct Smem3 {
+  size_t bars, ring, xa, xb, xc, gsum, gmult, cb, red, total;
+  int stage_bytes;
+};
+
+__host__ __device__ inline Smem3 smem3_plan(const Gemv2Params& p) {
+  Smem3 s{};
+  const int kr = p.cols_per_split * kColK3;
+  const int gr = kr / 16;
+  s.stage_bytes = (int)align_up((size_t)p.stage_cols * kBt3ColBytes, 128);
+  size_t off = 0;
+  s.bars = off;
+  off = align_up(off + (size_t)p.wpc * p.nstage * 8, 128);
+  s.ring = off;
+  off += (size_t)p.wpc * p.nstage * s.stage_bytes;
+  s.xa = off;
+  off = align_up(off + (size_t)kr, 128);
+  s.xb = off;
+  off = align_up(off + (size_t)kr, 128);
+  s.xc = off;
+  off = align_up(off + (size_t)kr, 128);
+  s.gsum = off;
+  off = align_up(off + (size_t)gr * 8, 16);
+  s.gmult = off;
+  off = align_up(off + (size_t)gr * 4, 16);
+  s.cb = off;
+  off = align_up(off + 27 * 4, 16);
+  s.red = off;
+  off = align_up(off + ((p.cluster && p.ks > 1) ? (size_t)p.ks * p.wpc * 32 * 4 : 0), 16);
+  s.total = off;
+  return s;
+}
+
+// Five base-3 digits of the two values (each <= 242) held in the 16-bit lanes of v.
+__device__ __forceinline__ void digits5(uint32_t v, uint32_t (&d)[5]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t q = ((v * 171u) >> 9) & 0x007F007Fu;  // floor(v / 3) in both lanes
+    d[j] = v - 3u * q;
+    v = q;
+  }
+  d[4] = v;
+}
+
+__device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv2Params p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const Smem3 sp = smem3_plan(p);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.y;
+  const bool clus = p.cluster && p.ks > 1;
+  const int c0 = split * p.cols_per_split;
+  const int c1 = min(p.cols, c0 + p.cols_per_split);
+  const int ncols = c1 - c0;
+  const int sc = p.stage_cols, nst = p.nstage;
+  const int spt = (ncols + sc - 1) / sc;
+  const int k0 = c0 * kColK3, kr = ncols * kColK3;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sp.bars) + warp * nst;
+  uint8_t* ring = smem + sp.ring + (size_t)warp * nst * sp.stage_bytes;
+
+  int gbeg = blockIdx.x, gend = blockIdx.x + 1;
+  if (p.persistent) {
+    gbeg = (int)((long long)p.groups_total * blockIdx.x / gridDim.x);
+    gend = (int)((long long)p.groups_total * (blockIdx.x + 1) / gridDim.x);
+  }
+  auto prob_of = [&](int gi) {
+    int q = 0;
+    while (q + 1 < p.nprob && gi >= p.prob[q + 1].cta_begin) ++q;
+    return q;
+  };
+  auto tile_of = [&](int gi, int q) { return (gi - p.prob[q].cta_begin) * p.wpc + warp; };
+
+  // ---- prologue: barriers, first weight stages
+  if (clus) cluster_arrive_relaxed();
+  if (lane == 0) {
+    for (int s = 0; s < nst; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const uint64_t pol = policy_evict_first();
+  int ig = gbeg, iq = prob_of(gbeg), is_ = 0, nissued = 0, islot = 0;
+  auto cursor_skip_inactive = [&]() {
+    while (ig < gend) {
+      while (iq + 1 < p.nprob && ig >= p.prob[iq + 1].cta_begin) ++iq;
+      if (tile_of(ig, iq) < p.prob[iq].row_tiles) break;
+      ++ig;
+    }
+  };
+  cursor_skip_inactive();
+  auto issue_next = [&]() {
+    if (ig >= gend) return;
+    const Gemv2Problem& pq = p.prob[iq];
+    const int T = tile_of(ig, iq);
+    const int slot = islot;
+    islot = islot + 1 == nst ? 0 : islot + 1;
+    const int cs = c0 + is_ * sc, ce = min(c1, cs + sc);
+    const uint32_t tb = (uint32_t)(ce - cs) * kBt3ColBytes;
+    mbar_arrive_expect_tx(&bars[slot], tb);
+    bulk_g2s(ring + (size_t)slot * sp.stage_bytes, pq.trit + ((size_t)T * p.cols + cs) * kBt3ColBytes, tb,
+             &bars[slot], pol);
+    ++nissued;
+    if (++is_ == spt) {
+      is_ = 0;
+      ++ig;
+      cursor_skip_inactive();
+    }
+  };
+  if (lane == 0)
+    for (int i = 0; i < nst; ++i) issue_next();
+  pdl_launch_dependents();
+  pdl_wait();
+  if (clus) cluster_wait_acquire();
+
+  const long long* gsum = reinterpret_cast<const long long*>(smem + sp.gsum);
+  const float* gmul = reinterpret_cast<const float*>(smem + sp.gmult);
+  const uint32_t x32 = smem_u32(smem + sp.xa), xm32 = smem_u32(smem + sp.xb), xl32 = smem_u32(smem + sp.xc);
+  const uint32_t cb32 = smem_u32(smem + sp.cb);
+  const uint32_t ring32 = smem_u32(ring);
+
+  int cur_prob = -1, nconsumed = 0, ifail = -1, pi = prob_of(gbeg);
+  int cslot = 0;
+  uint32_t cphase = 0;
+  float yacc = 0.f;
+  for (int gi = gbeg; gi < gend; ++gi) {
+    while (pi + 1 < p.nprob && gi >= p.prob[pi + 1].cta_begin) ++pi;
+    const Gemv2Problem& pr = p.prob[pi];
+    if (pi != cur_prob) {
+      __syncthreads();
+      // codebook from the packed header (trit stream starts 256 bytes after the
+      // header; the codebook sits at header byte 128)
+      if (threadIdx.x < 27)
+        reinterpret_cast<float*>(smem + sp.cb)[threadIdx.x] =
+            reinterpret_cast<const float*>(pr.trit - kHeaderBytes + kCodebookOffset)[threadIdx.x];
+      gemv_common::stage_x_bf16_image(static_cast<const uint16_t*>(pr.x), p.k, 16, k0, kr,
+                                      reinterpret_cast<int8_t*>(smem + sp.xa), smem + sp.xb, smem + sp.xc,
+                                      reinterpret_cast<long long*>(smem + sp.gsum),
+                                      reinterpret_cast<float*>(smem + sp.gmult));
+      __syncthreads();
+      cur_prob = pi;
+    }
+    const int T = tile_of(gi, pi);
+    const bool active = T < pr.row_tiles;
+    yacc = 0.f;
+    if (active && ifail < 0) {
+      for (int s = 0; s < spt; ++s, ++nconsumed) {
+        const int slot = cslot;
+        const uint32_t phase = cphase;
+        if (++cslot == nst) {
+          cslot = 0;
+          cphase ^= 1u;
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&bars[slot], phase))) {
+          ifail = nconsumed;
+          break;
+        }
+        const uint32_t st32 = ring32 + (uint32_t)slot * sp.stage_bytes;
+        const int cs = c0 + s * sc;
+        const int ncs = min(sc, c1 - cs);
+        for (int cc = 0; cc < ncs; ++cc) {
+          const uint32_t col = st32 + (uint32_t)(cc * kBt3ColBytes);
+          const uint32_t kx = (uint32_t)((cs + cc - c0) * kColK3);
+          // scale indices of the column's five groups (three bytes of base-3 digits)
+          uint32_t ia[5], ib[5];
+          digits5(lds_u8(col + 3 * kPlaneColBytes + lane) | (lds_u8(col + 3 * kPlaneColBytes + 32 + lane) << 16), ia);
+          digits5(lds_u8(col + 3 * kPlaneColBytes + 64 + lane), ib);
+          // U = u0 + 3 u1 + 9 u2 in byte lanes, for the 4 words x 5 digit positions
+          uint32_t U[4][5];
+          const uint4 b0 = lds128<0>(col + lane * 16);
+          const uint4 b1 = lds128<kPlaneColBytes>(col + lane * 16);
+          const uint4 b2 = lds128<2 * kPlaneColBytes>(col + lane * 16);
+          auto word_u = [&](auto wi_c, uint32_t w0, uint32_t w1, uint32_t w2) {
+            constexpr int w = decltype(wi_c)::value;
+            uint32_t l0[5], h0[5], l1[5], h1[5], l2[5], h2[5];
+            digits5(w0 & 0x00FF00FFu, l0);
+            digits5((w0 >> 8) & 0x00FF00FFu, h0);
+            digits5(w1 & 0x00FF00FFu, l1);
+            digits5((w1 >> 8) & 0x00FF00FFu, h1);
+            digits5(w2 & 0x00FF00FFu, l2);
+            digits5((w2 >> 8) & 0x00FF00FFu, h2);
+#pragma unroll
+            for (int j = 0; j < 5; ++j) {
+              const uint32_t ul = l0[j] + 3u * l1[j] + 9u * l2[j];  // bytes 0, 2 in 16-bit lanes
+              const uint32_t uh = h0[j] + 3u * h1[j] + 9u * h2[j];  // bytes 1, 3
+              U[w][j] = ul | (uh << 8);
+            }
+          };
+          word_u(std::integral_constant<int, 0>{}, b0.x, b1.x, b2.x);
+          word_u(std::integral_constant<int, 1>{}, b0.y, b1.y, b2.y);
+          word_u(std::integral_constant<int, 2>{}, b0.z, b1.z, b2.z);
+          word_u(std::integral_constant<int, 3>{}, b0.w, b1.w, b2.w);
+#pragma unroll
+          for (int j = 0; j < 5; ++j) {
+            const uint32_t xo = kx + 16u * j;
+            const uint4 hv = lds128<0>(x32 + xo), mv = lds128<0>(xm32 + xo), lv = lds128<0>(xl32 + xo);
+            int H = 0;
+            unsigned M = 0, L = 0;
+            H = dp4a_us(U[0][j], (int)hv.x, H);
+            H = dp4a_us(U[1][j], (int)hv.y, H);
+            H = dp4a_us(U[2][j], (int)hv.z, H);
+            H = dp4a_us(U[3][j], (int)hv.w, H);
+            M = dp4a_uu(U[0][j], mv.x, M);
+            M = dp4a_uu(U[1][j], mv.y, M);
+            M = dp4a_uu(U[2][j], mv.z, M);
+            M = dp4a_uu(U[3][j], mv.w, M);
+            L = dp4a_uu(U[0][j], lv.x, L);
+            L = dp4a_uu(U[1][j], lv.y, L);
+            L = dp4a_uu(U[2][j], lv.z, L);
+            L = dp4a_uu(U[3][j], lv.w, L);
+            const int g = (int)(kx >> 4) + j;  // group within the split
+            const long long S = ((long long)H * 65536 + (long long)M * 256 + L) - 13ll * gsum[g];
+            const uint32_t idx = (ia[j] & 0xFFFFu) + 3u * (ia[j] >> 16) + 9u * ib[j];
+            yacc = fmaf(lds_f32(cb32 + 4u * idx) * gmul[g], __ll2float_rn(S), yacc);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) issue_next();
+      }
+    }
+
+    const int row = T * kTileRows + lane;
+    auto write_out = [&](float v) {
+      if (row >= pr.n) return;
+      if (p.out_bf16)
+        reinterpret_cast<__nv_bfloat16*>(pr.y)[row] = __float2bfloat16_rn(v);
+      else
+        reinterpret_cast<float*>(pr.y)[row] = v;
+    };
+    if (p.ks == 1) {
+      if (active) write_out(yacc);
+      continue;
+    }
+    if (active && ifail >= 0) {
+      for (int j = ifail; j < min(nissued, ifail + nst); ++j)
+        mbar_wait_bounded(&bars[j % nst], (uint32_t)(j / nst) & 1u);  // error path only
+    }
+    // K is split: the splits of this row group form the cluster; reduce in rank 0
+    const int rows_cta = p.wpc * kTileRows;
+    if (active) {
+      const size_t idx = (size_t)split * rows_cta + warp * kTileRows + lane;
+      st_cluster_u32(map_cluster_rank(smem_u32(smem + sp.red + idx * 4), 0), __float_as_uint(yacc));
+    }
+    cluster_sync();
+    if (split == 0 && active) {
+      float sf = 0.f;
+      for (int s = 0; s < p.ks; ++s)
+        sf += reinterpret_cast<const float*>(smem + sp.red)[(size_t)s * rows_cta + warp * kTileRows + lane];
+      write_out(sf);
+    }
+    return;
+  }
+  if (ifail >= 0) {
+    for (int j = ifail; j < min(nissued, ifail + nst); ++j) mbar_wait_bounded(&bars[j % nst], (uint32_t)(j / nst) & 1u);
+  }
+}
+
+size_t gemv3_smem_bytes(const Gemv2Params& p) { return smem3_plan(p).total; }
+
+int launch_gemv3(const Gemv2Params& p, bool pdl, void* stream) {
+  if (p.m != 1 || (p.ks > 1 && !p.cluster)) return -1;
+  const Smem3 sp = smem3_plan(p);
+  cudaError_t e = cudaFuncSetAttribute(gemv3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
+  if (e != cudaSuccess) return (int)e;
+  const bool clus = p.cluster && p.ks > 1;
+  if (clus && p.ks > 8) {
+    e = cudaFuncSetAttribute(gemv3_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return (int)e;
+  }
+  Gemv2Params q = p;
+  q.groups_total = p.grid_x;
+  q.persistent = 0;
+  int gx = p.grid_x;
+  if (p.ks == 1) {
+    int dev = 0, sms = 0, occ = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv3_kernel, 32 * p.wpc, sp.total);
+    if (e != cudaSuccess) return (int)e;
+    if (occ > 0 && gx > sms * occ) {
+      gx = sms * occ;
+      q.persistent = 1;
+    }
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(gx, p.ks, 1);
+  cfg.blockDim = dim3(32 * p.wpc, 1, 1);
+  cfg.dynamicSmemBytes = sp.total;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (clus) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = p.ks;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return (int)cudaLaunchKernelEx(&cfg, gemv3_kernel, q);
+}
+
+}  // namespace tern

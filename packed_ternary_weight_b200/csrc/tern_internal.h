@@ -79,6 +79,9 @@ int launch_quantize(const uint16_t* x, int m, int k, int8_t* xq, float* xs, void
 
 int read_clear_dev_error_gemv2(void* stream, unsigned* out);
 int read_clear_dev_error_stream(void* stream, unsigned* out);
+int read_clear_dev_error_gemv3(void* stream, unsigned* out);
+int launch_gemv3(const Gemv2Params& p, bool pdl, void* stream);  // balanced ternary d = 3, bf16 x, m = 1
+size_t gemv3_smem_bytes(const Gemv2Params& p);
 int launch_stream_read(const void* src, size_t bytes, int mode, int chunk, int depth, int ctas_per_sm, int warps,
                        unsigned* sink, void* stream);
 

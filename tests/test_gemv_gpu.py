@@ -309,3 +309,55 @@ def test_long_k_workspace_path(tern):
         sx = torch.ones(1, dtype=torch.float32, device="cuda")
         tern.gemv(d, dev(tern.pack_layer(lay)[1]), tern.ACT_INT8, xq, sx, tern.OUT_F32, y, None)
     assert ei.value.code == tern.ENOSPACE
+
+
+# ------------------------------------------------- balanced ternary d = 3
+def bt3_check(tern, layer, rows=None, use_ws=True):
+    x = synth.draw_x_bf16(layer.seed, 1, layer.k)
+    y32 = run_bf16(tern, layer, x, tern.OUT_F32, use_ws)
+    y16 = run_bf16(tern, layer, x, tern.OUT_BF16, use_ws)
+    r = slice(None) if rows is None else rows
+    w = oracle.dequantize("bt3", layer.trits[:, r], 16, idx=layer.idx[r], codebook=layer.codebook)
+    yref = oracle.gemv_bf16(w, x)[0]
+    check_bf16(y32[0, r], yref)
+    assert np.array_equal(y16.view(np.uint16), synth.f32_to_bf16_bits(y32))
+
+
+@pytest.mark.parametrize("shape", synth.LLAMA_8B_SHAPES, ids=[s[0] for s in synth.LLAMA_8B_SHAPES])
+def test_bt3_llama_shapes(tern, shape):
+    name, n, k = shape
+    lay = synth.bt3_layer(n, k, seed=300 + [s[0] for s in synth.LLAMA_8B_SHAPES].index(name))
+    rows = np.sort(np.random.default_rng(2).choice(n, min(n, 384), replace=False))
+    bt3_check(tern, lay, rows=rows)
+
+
+@pytest.mark.parametrize("n,k", [(1, 16), (45, 96), (32, 160), (70, 4096), (300, 1040)])
+def test_bt3_ragged(tern, n, k):
+    lay = synth.bt3_layer(n, k, seed=n * 3 + k)
+    bt3_check(tern, lay)
+    bt3_check(tern, lay, use_ws=False)
+
+
+def test_bt3_codebook_extremes(tern):
+    lay = synth.bt3_layer(64, 320, seed=77)
+    lay.idx[:32] = 0
+    lay.idx[32:] = 26
+    bt3_check(tern, lay)
+
+
+def test_bt3_grouped(tern):
+    lays = [synth.bt3_layer(n, 1024, seed=90 + n) for n in (64, 200, 33)]
+    descs, packs, xs, ys, xbits = [], [], [], [], []
+    for lay in lays:
+        d, buf = tern.pack_layer(lay)
+        descs.append(d)
+        packs.append(dev(buf))
+        xb = synth.draw_x_bf16(lay.seed, 1, lay.k)
+        xbits.append(xb)
+        xs.append(x_dev(xb))
+        ys.append(torch.empty(lay.n, dtype=torch.float32, device="cuda"))
+    tern.gemv_grouped(descs, packs, tern.ACT_BF16, xs, None, tern.OUT_F32, ys)
+    torch.cuda.synchronize()
+    for lay, y, xb in zip(lays, ys, xbits):
+        w = oracle.dequantize("bt3", lay.trits, 16, idx=lay.idx, codebook=lay.codebook)
+        check_bf16(y.cpu().numpy(), oracle.gemv_bf16(w, xb)[0])
