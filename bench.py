@@ -51,10 +51,15 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--layers", type=int, default=synth.BITNET_2B_LAYERS)
+    ap.add_argument("--config", default="bitnet2b", choices=("bitnet2b", "single", "tq3p", "bt3", "tq2p"),
+                    help="bitnet2b: the headline layer set; single: one 512x1024 GEMV; tq3p / bt3: "
+                         "Llama-3.1-8B shapes; tq2p: the batched sweep (per-shape tables only)")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--profile", default=None,
                     help="run only one case eagerly for a profiler: step | <shape>_indep | <shape>_chain")
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--ceiling", action="store_true",
+                    help="measure the read ceiling (tern_stream_read) for a few access shapes and exit")
     return ap.parse_args()
 
 
@@ -246,7 +251,7 @@ def run_ours(args, rank, world):
             g_step.replay()
         torch.cuda.synchronize()
     clocks = ClockSampler(dev.index, not args.no_clocks and rank == 0)
-    t_end = time.time() + 1.0       # soak so the clock samples see this load
+    t_end = time.time() + (1.0 if not args.no_clocks else 0.0)   # soak so the clock samples see this load
     with torch.cuda.stream(stream):
         while time.time() < t_end:
             for _ in range(20):
@@ -344,6 +349,133 @@ def run_ours(args, rank, world):
     if rank == 0 and world == 1:
         out["cpu_baseline"] = cpu_baseline(budget_s=12.0)
     return out
+
+
+def run_config(args):
+    """Per-shape tables for the other workloads (one JSON line, rank 0, one GPU).
+
+    Each shape's packed layer is replicated on the device until the pool holds
+    at least 512 MB (4x L2), so every launch streams from HBM; "independent" is
+    one grouped launch over all copies, "chain" launches the copies one after
+    another with programmatic dependent launch.
+    """
+    import torch
+
+    from packed_ternary_weight_b200 import tern
+
+    torch.cuda.set_device(0)
+    stream = torch.cuda.Stream()
+    if args.config == "single":
+        layers = [synth.single_gemv_layer()]
+        act = tern.ACT_BF16_Q8
+    elif args.config == "tq3p":
+        layers = list(synth.tq3p_llama_layers())
+        act = tern.ACT_BF16
+    elif args.config == "bt3":
+        layers = list(synth.bt3_llama_layers())
+        act = tern.ACT_BF16
+    else:
+        layers = list(synth.tq2p_prefill_layers())
+        act = tern.ACT_INT8
+    peak, _ = measured_peaks()
+    rows = []
+    reps = max(3, min(args.steps, 50))
+    for lay in layers:
+        d, buf = tern.pack_layer(lay, flags=tern.F_PDL)
+        wbytes = len(buf) - 256
+        copies = max(2, min(256, -(-512_000_000 // wbytes)))
+        pk = torch.from_numpy(buf).cuda()
+        packs = [pk] + [pk.clone() for _ in range(copies - 1)]
+        del lay.trits
+        tokens = synth.PREFILL_TOKENS if args.config == "tq2p" else (1,)
+        for m in tokens:
+            if m >= 16:
+                continue                      # prefill sizes: tensor-core path, reported separately
+            x = synth.draw_x_bf16(lay.seed, m, lay.k)
+            xd = torch.from_numpy(x.view(np.int16)).cuda()
+            ys = [torch.empty((m, lay.n), dtype=torch.float32, device="cuda") for _ in range(copies)]
+            xq = torch.empty((m, lay.k), dtype=torch.int8, device="cuda")
+            sx = torch.empty((m,), dtype=torch.float32, device="cuda")
+            tern.quantize_act(xd, xq, sx, stream)
+            ws = torch.zeros(max(16, tern.workspace_size(d, m)), dtype=torch.uint8, device="cuda")
+            xin = xq if act == tern.ACT_INT8 else xd
+            sin = sx if act == tern.ACT_INT8 else None
+            algo = wbytes + m * lay.k * (1 if act == tern.ACT_INT8 else 2) + 4 * m * lay.n
+
+            def chain():
+                for pkc, y in zip(packs, ys):
+                    tern.gemm_batched(d, pkc, m, act, xin, sin, tern.OUT_F32, y, ws, stream)
+
+            indep = None
+            if m == 1:   # grouped launches of up to 32 independent GEMVs
+                indep = [tern.Grouped([d] * len(packs[i:i + 32]), packs[i:i + 32], act,
+                                      [xin.view(-1)] * len(packs[i:i + 32]),
+                                      None if sin is None else [sin] * len(packs[i:i + 32]), tern.OUT_F32,
+                                      [y.view(-1) for y in ys[i:i + 32]]) for i in range(0, copies, 32)]
+
+            def timed(fn):
+                with torch.cuda.stream(stream):
+                    fn()
+                    torch.cuda.synchronize()
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g, stream=stream):
+                        fn()
+                    for _ in range(2):
+                        g.replay()
+                    torch.cuda.synchronize()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    for _ in range(reps):
+                        g.replay()
+                    e1.record(stream)
+                    torch.cuda.synchronize()
+                return e0.elapsed_time(e1) / reps
+
+            ms_c = timed(chain)
+            row = dict(shape=f"{lay.name} {lay.n}x{lay.k}", m=m, bytes_per_gemv=algo, copies=copies,
+                       chain_us_per_gemv=round(ms_c * 1e3 / copies, 3),
+                       chain_gbs=round(algo * copies / (ms_c * 1e-3) / 1e9, 1))
+            if indep is not None:
+                ms_i = timed(lambda: [g.launch(stream) for g in indep])
+                row["independent_gbs"] = round(algo * copies / (ms_i * 1e-3) / 1e9, 1)
+                row["independent_frac"] = round(row["independent_gbs"] / peak, 4)
+            rows.append(row)
+        del packs
+        torch.cuda.empty_cache()
+    assert tern.device_error(stream) == tern.OK
+    return {"metric": METRIC, "config": {"workload": args.config}, "unit": "GB/s", "peak": peak, "per_shape": rows}
+
+
+def run_ceiling(args):
+    """Read-ceiling sweep: stream a 2 GiB buffer once per launch with several access shapes."""
+    import torch
+
+    from packed_ternary_weight_b200 import tern
+
+    torch.cuda.set_device(0)
+    buf = torch.empty(2 << 30, dtype=torch.uint8, device="cuda")
+    buf.random_(0, 255)
+    sink = torch.zeros(1, dtype=torch.int32, device="cuda")
+    shapes = [(0, 16, d, cps, w) for w, cps in ((8, 4), (16, 4)) for d in (1, 4, 8)]
+    shapes += [(1, c, d, cps, w) for c in (2048, 4096, 8192) for d in (2, 3, 4) for w, cps in ((4, 2), (4, 1), (8, 1))
+               if w * d * c * cps <= 220 * 1024]
+    shapes += [(2, c, d, cps, w) for c in (8192, 16384, 32768) for d in (2, 4) for w, cps in ((4, 1), (4, 2), (8, 2))
+               if d * c * cps <= 220 * 1024]
+    rows = []
+    for mode, chunk, depth, cps, warps in shapes:
+        tern.stream_read(buf, mode, chunk, depth, cps, warps, sink)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(5):
+            tern.stream_read(buf, mode, chunk, depth, cps, warps, sink)
+        e1.record()
+        torch.cuda.synchronize()
+        gbs = buf.numel() / (e0.elapsed_time(e1) / 5 * 1e-3) / 1e9
+        rows.append(dict(mode=mode, chunk=chunk, depth=depth, ctas_per_sm=cps, warps=warps, gbs=round(gbs, 1)))
+    assert tern.device_error() == tern.OK
+    return {"metric": "read ceiling", "unit": "GB/s", "bytes": buf.numel(), "rows": rows,
+            "best": max(r["gbs"] for r in rows)}
 
 
 def committed_traffic(algo_bytes_per_launch):
@@ -450,7 +582,12 @@ def main():
 
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    out = run_reference(args, rank, world) if args.impl == "reference" else run_ours(args, rank, world)
+    if args.impl == "ours" and args.ceiling:
+        out = run_ceiling(args) if rank == 0 else None
+    elif args.impl == "ours" and args.config != "bitnet2b":
+        out = run_config(args) if rank == 0 else None
+    else:
+        out = run_reference(args, rank, world) if args.impl == "reference" else run_ours(args, rank, world)
     if rank == 0 and out is not None:
         print(json.dumps(out))
     if world > 1 and args.impl == "ours":
