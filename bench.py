@@ -329,7 +329,7 @@ def run_ours(args, rank, world):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
                      "traffic": committed_traffic(step_bytes / len(step_launches)),
-                     "kernel": "gemv2_kernel<bf16->int8 in-kernel, 1 plane, per-tensor scale, M=1>",
+                     "kernel": "gemv2w_kernel<bf16->int8 in-kernel, 1 plane, per-tensor scale> (one CTA per SM)",
                      "peak_kind": peak_kind,
                      "achieved_basis": "algorithmic bytes of the step's GEMV launches (weights, bf16 activations, "
                                        "fp32 outputs) / their duration; every launch of the step is this kernel"},

@@ -118,6 +118,59 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
   return pl;
 }
 
+// Plan of the single-token kernel with one CTA per SM (gemv2w): equal tile
+// ranges per CTA, about 6 KB stages, as many warps and stages in flight as
+// shared memory allows next to the resident activation images. Applies when
+// the launch has at least four tiles per SM (smaller launches are spread
+// over the SMs by K splits in the row-group kernel).
+bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, int sms, Gemv2wParams& p) {
+  if (L.fmt == TERN_FMT_BT3) return false;
+  int begin[kMaxProblems + 1];
+  begin[0] = 0;
+  for (int i = 0; i < nprob; ++i) begin[i + 1] = begin[i] + row_tiles[i];
+  const int T = begin[nprob];
+  if (T < 4 * sms) return false;
+  // the kernel's index arithmetic is 32-bit: tiles x CTAs and a CTA's
+  // columns x warps stay below 2^31
+  if ((long long)T * sms >= (1ll << 31) || ((long long)T / sms + 1) * L.cols * 16 >= (1ll << 31)) return false;
+  const bool tq = L.fmt == TERN_FMT_TQ;
+  p.tq = tq;
+  p.k = L.k;
+  p.planes = L.planes;
+  p.group = L.group;
+  p.groups = L.groups;
+  p.cols = L.cols;
+  p.gcols = (tq && L.group >= 64) ? L.group / 64 : 1;
+  p.nprob = nprob;
+  p.tiles_total = T;
+  p.grid = std::min(sms, T);
+  for (int i = 0; i <= nprob; ++i) p.tile_begin[i] = begin[i];
+  auto prob_of = [&](int t) {
+    int q = 0;
+    while (q + 1 < nprob && t >= begin[q + 1]) ++q;
+    return q;
+  };
+  int xs = 1;
+  for (int c = 0; c < p.grid; ++c) {
+    const int t0 = (int)((long long)T * c / p.grid), t1 = (int)((long long)T * (c + 1) / p.grid);
+    xs = std::max(xs, prob_of(t1 - 1) - prob_of(t0) + 1);
+  }
+  p.xslots = xs;
+  const int colb = L.planes * kPlaneColBytes;
+  p.stage_cols = std::max(p.gcols, (6144 / colb) / p.gcols * p.gcols);
+  // (warps, stages): sixteen warps with two 6 KB stages each measured best on
+  // the BitNet-2B layer set; fewer when the activation images need the room
+  static const int kShapes[][2] = {{16, 2}, {12, 2}, {8, 3}, {8, 2}, {4, 3}, {4, 2}};
+  for (const auto& sh : kShapes) {
+    p.nw = sh[0];
+    p.nstage = sh[1];
+    // the kernel adds its shared copy of the problem table
+    if (gemv2w_smem_bytes(p, xmode) + sizeof(Gemv2wProblem) * kMaxProblems + 4 * (kMaxProblems + 1) <= 227 * 1024)
+      return true;
+  }
+  return false;
+}
+
 tern_status check_one(const tern_desc* desc, const void* d_packed, tern_act act, const void* d_x,
                       const float* d_xscale, tern_out out, void* d_y, Layout* L) {
   tern_status st = layout_of(desc, L);
@@ -168,6 +221,27 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
   if (xmode == kXBf16 && m != 1) return TERN_EUNSUPPORTED;
   const int sms = device_sms();
   const uint8_t* base = static_cast<const uint8_t*>(d_packed);
+  const bool pdl = (desc->flags & TERN_F_PDL) != 0;
+  if (m == 1) {
+    Gemv2wParams w{};
+    const int rt = L.row_tiles;
+    if (plan_gemv2w(L, &rt, 1, xmode, sms, w)) {
+      w.out_bf16 = out == TERN_OUT_BF16;
+      Gemv2wProblem& q = w.prob[0];
+      q.trit = base + L.trit_offset;
+      q.scale = w.tq ? reinterpret_cast<const uint16_t*>(base + L.scale_offset) : nullptr;
+      q.x = d_x;
+      q.xscale = d_xscale;
+      q.y = d_y;
+      q.n = L.n;
+      q.row_tiles = L.row_tiles;
+      q.tensor_scale = desc->tensor_scale;
+      w.x_vec = aligned16(d_x) && L.k % 16 == 0;
+      const int rc = launch_gemv2w(w, xmode, pdl, stream);
+      if (rc < 0) return TERN_EUNSUPPORTED;
+      return rc == 0 ? TERN_OK : TERN_ECUDA;
+    }
+  }
   const size_t in_elem = xmode == kXInt8 ? 1 : 2;
   const size_t out_elem = out == TERN_OUT_F32 ? 4 : 2;
   const int mt_max = gemv2_mt(xmode, m);
@@ -195,7 +269,6 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
       p.ws_cnt = static_cast<unsigned*>(d_ws);
       p.ws_part = static_cast<uint8_t*>(d_ws) + pl.ws_cnt_bytes;
     }
-    const bool pdl = (desc->flags & TERN_F_PDL) != 0;
     const int rc = L.fmt == TERN_FMT_BT3 ? launch_gemv3(p, pdl, stream) : launch_gemv2(p, xmode, pdl, stream);
     if (rc < 0) return TERN_EUNSUPPORTED;
     if (rc != 0) return TERN_ECUDA;
@@ -269,7 +342,33 @@ extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, 
   const int xmode = xmode_of(act);
   tern_status st = supported_2bit(L[0], xmode);
   if (st != TERN_OK) return st;
-  const Plan2 pl = plan_gemv2(L[0], rt, count, 1, xmode, device_sms(), false);
+  const int sms = device_sms();
+  const bool pdl = (descs[0].flags & TERN_F_PDL) != 0;
+  {
+    Gemv2wParams w{};
+    if (plan_gemv2w(L[0], rt, count, xmode, sms, w)) {
+      w.out_bf16 = out == TERN_OUT_BF16;
+      bool vec = L[0].k % 16 == 0;
+      for (int i = 0; i < count; ++i) {
+        const uint8_t* base = static_cast<const uint8_t*>(d_packed[i]);
+        Gemv2wProblem& q = w.prob[i];
+        q.trit = base + L[i].trit_offset;
+        q.scale = w.tq ? reinterpret_cast<const uint16_t*>(base + L[i].scale_offset) : nullptr;
+        q.x = d_x[i];
+        q.xscale = d_xscale ? d_xscale[i] : nullptr;
+        q.y = d_y[i];
+        q.n = L[i].n;
+        q.row_tiles = L[i].row_tiles;
+        q.tensor_scale = descs[i].tensor_scale;
+        vec = vec && aligned16(q.x);
+      }
+      w.x_vec = vec;
+      const int rc = launch_gemv2w(w, xmode, pdl, stream);
+      if (rc < 0) return TERN_EUNSUPPORTED;
+      return rc == 0 ? TERN_OK : TERN_ECUDA;
+    }
+  }
+  const Plan2 pl = plan_gemv2(L[0], rt, count, 1, xmode, sms, false);
   if (!pl.ok) return TERN_EUNSUPPORTED;
   Gemv2Params p{};
   fill_common(p, L[0], pl, 1, out);
@@ -292,7 +391,6 @@ extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, 
     vec = vec && aligned16(q.x);
   }
   p.x_vec = vec;
-  const bool pdl = (descs[0].flags & TERN_F_PDL) != 0;
   const int rc = L[0].fmt == TERN_FMT_BT3 ? launch_gemv3(p, pdl, stream) : launch_gemv2(p, xmode, pdl, stream);
   if (rc < 0) return TERN_EUNSUPPORTED;
   return rc == 0 ? TERN_OK : TERN_ECUDA;
@@ -301,6 +399,7 @@ extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, 
 extern "C" tern_status tern_device_error(void* stream) {
   unsigned v = 0;
   if (read_clear_dev_error_gemv2(stream, &v) != 0) return TERN_ECUDA;
+  if (read_clear_dev_error_gemv2w(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_stream(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_gemv3(stream, &v) != 0) return TERN_ECUDA;
   return v ? TERN_ETIMEOUT : TERN_OK;

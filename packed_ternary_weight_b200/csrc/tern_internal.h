@@ -73,8 +73,43 @@ struct Gemv2Params {
   unsigned* ws_cnt;         // global fallback: arrival counters [grid.x]
 };
 
+// Single-token 2-bit GEMV with one CTA per SM ("whole-K" kernel, gemv2w):
+// the row tiles of all problems are split into equal contiguous ranges, one
+// per CTA, and each CTA's columns (tiles x columns) into equal contiguous
+// ranges, one per warp; tiles that two or more warps share are combined in
+// shared memory in warp order.
+struct Gemv2wProblem {
+  const uint8_t* trit;
+  const uint16_t* scale;
+  const void* x;            // [k]
+  const float* xscale;      // kXInt8: [1]
+  void* y;                  // [n]
+  int n, row_tiles;
+  float tensor_scale;
+};
+
+// Scalars first and the tiles' problem boundaries as one compact array, so
+// that a CTA's start-up reads touch few lines of the parameter buffer (every
+// SM misses on the same lines at once).
+struct Gemv2wParams {
+  int nprob, tiles_total;
+  int grid;                 // CTAs (at most one per SM)
+  int tq, k, planes, group, groups, cols;
+  int gcols;                // columns per granule of the warp ranges (a whole scale group)
+  int out_bf16;
+  int nw;                   // warps per CTA
+  int stage_cols, nstage;   // per-warp ring: columns per stage, stages
+  int xslots;               // activation images resident per CTA
+  int x_vec;                // activations may be read with 16-byte loads
+  int tile_begin[kMaxProblems + 1];  // first tile of each problem; [nprob] = tiles_total
+  Gemv2wProblem prob[kMaxProblems];
+};
+
 // Launchers return cudaError_t values as int (0 = success).
 int launch_gemv2(const Gemv2Params& p, int xmode, bool pdl, void* stream);  // -1: no kernel
+int launch_gemv2w(const Gemv2wParams& p, int xmode, bool pdl, void* stream);  // -1: no kernel
+size_t gemv2w_smem_bytes(const Gemv2wParams& p, int xmode);
+int read_clear_dev_error_gemv2w(void* stream, unsigned* out);
 int launch_quantize(const uint16_t* x, int m, int k, int8_t* xq, float* xs, void* stream);
 
 int read_clear_dev_error_gemv2(void* stream, unsigned* out);
