@@ -7,10 +7,12 @@ benchmark's CPU baseline can start from the same bytes the GPU reads.
 
 Format (all little-endian):
 
-* 256-byte header: u32 magic 0x4E524554, u32 version 1, u32 fmt (1 BitNet,
+* 256-byte header: u32 magic 0x4E524554, u32 version 2, u32 fmt (1 BitNet,
   2 TQ, 3 balanced ternary d=3), u32 N, u32 K, u32 planes, u32 group,
   f32 tensor scale, u32 row tiles ceil(N/32), u32 columns, u64 trit offset,
-  u64 trit bytes, u64 scale offset, u64 scale bytes; the 27 fp32 codebook
+  u64 trit bytes, u64 scale offset, u64 scale bytes; at byte 72 u32 "scale
+  digits": TQ, the number of base-128 digits of the largest |s| / 2^-24 over
+  all scales (at least 1); BitNet 1; balanced ternary 0. The 27 fp32 codebook
   entries at byte 128 (balanced ternary only). Everything else is zero.
 * 2-bit planes (BitNet, TQ): a chunk is 16 bytes holding 64 consecutive k of
   one row of one plane, as four u32 words; word w holds k = 64c + 16w + j for
@@ -48,12 +50,13 @@ def parse_header(buf: np.ndarray) -> dict:
     (tscale,) = struct.unpack_from("<f", b, 28)
     row_tiles, cols = struct.unpack_from("<2I", b, 32)
     toff, tbytes, soff, sbytes = struct.unpack_from("<4Q", b, 40)
+    (digits,) = struct.unpack_from("<I", b, 72)
     cb = np.frombuffer(b, dtype="<f4", count=27, offset=128).copy()
-    if magic != MAGIC or version != 1:
+    if magic != MAGIC or version != 2:
         raise ValueError("not a packed ternary buffer")
     return dict(fmt=FMT_NAMES[fmt], n=n, k=k, planes=planes, group=group, tensor_scale=tscale,
                 row_tiles=row_tiles, cols=cols, trit_offset=toff, trit_bytes=tbytes,
-                scale_offset=soff, scale_bytes=sbytes, codebook=cb)
+                scale_offset=soff, scale_bytes=sbytes, scale_digits=digits, codebook=cb)
 
 
 def _decode_2bit(code: np.ndarray) -> np.ndarray:

@@ -171,6 +171,76 @@ bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, in
   return false;
 }
 
+// Plan of the tensor-core batched GEMM (m >= 16 int8 tokens, 2-bit formats)
+// for one launch of up to kTcMaxTokens tokens. The digit count D of the scales
+// is read by the kernel from the packed header, so the token passes and the
+// activation slot are sized here for every D the kernel may meet.
+// Workspace: arrival counters [tiles][4] | int64 partial sums [256][n_pad]
+// (both zero on entry and left zero; sized and placed for the largest launch,
+// so that calls with any token count can share one workspace) | activations
+// in MMA order | (bf16 input) int8 activations and their scales.
+struct PlanTc {
+  GemmTcParams p;
+  int kchunks;
+  size_t cnt_off, part_off, xp_off, xq_off, sx_off, total;
+  bool ok;
+};
+
+PlanTc plan_tc(const Layout& L, int mb, int xmode, int sms) {
+  PlanTc t{};
+  const bool tq = L.fmt == TERN_FMT_TQ;
+  if (L.fmt == TERN_FMT_BT3 || (xmode != kXInt8 && xmode != kXBf16Q8) || mb < 1 || mb > kTcMaxTokens) return t;
+  // every digit accumulator stays below 2^31: planes * 127 * 127 * K
+  if ((long long)L.planes * 127 * 127 * L.k >= (1ll << 31)) return t;
+  GemmTcParams& p = t.p;
+  p.tq = tq;
+  p.n = L.n;
+  p.k = L.k;
+  p.planes = L.planes;
+  p.group = tq ? L.group : 0;
+  p.cols = L.cols;
+  p.row_tiles = L.row_tiles;
+  p.tiles = (L.row_tiles + 3) / 4;
+  p.n_pad = p.tiles * kTcRows;
+  p.m = mb;
+  p.m16 = (mb + 15) & ~15;
+  int mp = 0, xcap = 0, pcap = 0;
+  for (int d = 1; d <= (tq ? kTcMaxDigits : 1); ++d) {
+    int ps, tp;
+    tc_passes(d, p.m16, &ps, &tp);
+    mp = std::max(mp, ps * tp);
+    xcap = std::max(xcap, tp);
+    pcap = std::max(pcap, ps);
+  }
+  p.mp = mp;
+  p.xcap = xcap;
+  p.passes_cap = pcap;
+  p.grid = (int)std::min<long long>(sms, (long long)p.tiles * p.cols);
+  t.kchunks = L.cols * 4;
+  size_t off = 0;
+  auto take = [&off](size_t bytes) {
+    const size_t o = off;
+    off = (off + bytes + 255) / 256 * 256;
+    return o;
+  };
+  int pmax = 0, tdummy = 0;
+  tc_passes(kTcMaxDigits, kTcMaxTokens, &pmax, &tdummy);
+  t.cnt_off = take((size_t)p.tiles * pmax * 4);
+  t.part_off = take((size_t)kTcMaxTokens * p.n_pad * 8);
+  t.xp_off = take((size_t)t.kchunks * mp * 16);
+  if (xmode == kXBf16Q8) {
+    t.xq_off = take((size_t)mb * L.k);
+    t.sx_off = take((size_t)mb * 4);
+  }
+  t.total = off;
+  // three stages; as many A slots (8 KB each) as shared memory allows, up to 24
+  p.nstage = 3;
+  p.nslot = 24;
+  while (p.nslot >= 4 && gemm_tc_smem_bytes(p) > 227 * 1024) --p.nslot;
+  t.ok = p.nslot >= 4;
+  return t;
+}
+
 tern_status check_one(const tern_desc* desc, const void* d_packed, tern_act act, const void* d_x,
                       const float* d_xscale, tern_out out, void* d_y, Layout* L) {
   tern_status st = layout_of(desc, L);
@@ -222,6 +292,48 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
   const int sms = device_sms();
   const uint8_t* base = static_cast<const uint8_t*>(d_packed);
   const bool pdl = (desc->flags & TERN_F_PDL) != 0;
+  if (m >= 16) {
+    const int mb = std::min(m, kTcMaxTokens);
+    const PlanTc tp = plan_tc(L, mb, xmode, sms);
+    if (tp.ok) {
+      if (!d_ws || ws_bytes < tp.total) return TERN_ENOSPACE;
+      if ((reinterpret_cast<uintptr_t>(d_ws) & 255u) != 0) return TERN_EALIGN;
+      uint8_t* ws = static_cast<uint8_t*>(d_ws);
+      const size_t in_elem = xmode == kXInt8 ? 1 : 2;
+      const size_t out_elem = out == TERN_OUT_F32 ? 4 : 2;
+      for (int t0 = 0; t0 < m; t0 += kTcMaxTokens) {
+        const int mc = std::min(kTcMaxTokens, m - t0);
+        PlanTc pc = plan_tc(L, mc, xmode, sms);
+        if (!pc.ok) return TERN_EUNSUPPORTED;
+        GemmTcParams& p = pc.p;
+        const uint8_t* xin = static_cast<const uint8_t*>(d_x) + (size_t)t0 * L.k * in_elem;
+        const int8_t* xq = reinterpret_cast<const int8_t*>(xin);
+        const float* sx = d_xscale ? d_xscale + t0 : nullptr;
+        if (xmode == kXBf16Q8) {
+          xq = reinterpret_cast<const int8_t*>(ws + pc.xq_off);
+          sx = reinterpret_cast<const float*>(ws + pc.sx_off);
+          if (launch_quantize(reinterpret_cast<const uint16_t*>(xin), mc, L.k, const_cast<int8_t*>(xq),
+                              const_cast<float*>(sx), stream) != 0)
+            return TERN_ECUDA;
+        }
+        if (launch_tc_prep_x(xq, mc, L.k, pc.kchunks, p.mp, ws + pc.xp_off, stream) != 0) return TERN_ECUDA;
+        p.trit = base + L.trit_offset;
+        p.scale = p.tq ? reinterpret_cast<const uint16_t*>(base + L.scale_offset) : nullptr;
+        p.header = base;
+        p.xp = ws + pc.xp_off;
+        p.xscale = sx;
+        p.y = static_cast<uint8_t*>(d_y) + (size_t)t0 * L.n * out_elem;
+        p.part = reinterpret_cast<unsigned long long*>(ws + pc.part_off);
+        p.cnt = reinterpret_cast<unsigned*>(ws + pc.cnt_off);
+        p.out_bf16 = out == TERN_OUT_BF16;
+        p.tensor_scale = desc->tensor_scale;
+        const int rc = launch_gemm_tc(p, stream);
+        if (rc < 0) return TERN_EUNSUPPORTED;
+        if (rc != 0) return TERN_ECUDA;
+      }
+      return TERN_OK;
+    }
+  }
   if (m == 1) {
     Gemv2wParams w{};
     const int rt = L.row_tiles;
@@ -289,6 +401,12 @@ extern "C" tern_status tern_workspace_size(const tern_desc* desc, int32_t m, siz
   if (m < 0) return TERN_EINVAL;
   const int sms = device_sms();
   size_t need = 0;
+  if (m >= 16) {
+    for (int xmode = 0; xmode < 3; ++xmode) {
+      const PlanTc tp = plan_tc(L, std::min<int>(m, kTcMaxTokens), xmode, sms);
+      if (tp.ok) need = std::max(need, tp.total);
+    }
+  }
   if (L.fmt != TERN_FMT_BT3) {
     const int rt = L.row_tiles;
     for (int xmode = 0; xmode < 3; ++xmode) {
@@ -402,7 +520,9 @@ extern "C" tern_status tern_device_error(void* stream) {
   if (read_clear_dev_error_gemv2w(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_stream(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_gemv3(stream, &v) != 0) return TERN_ECUDA;
-  return v ? TERN_ETIMEOUT : TERN_OK;
+  if (read_clear_dev_error_gemm_tc(stream, &v) != 0) return TERN_ECUDA;
+  if (v & TERN_DEVERR_TIMEOUT) return TERN_ETIMEOUT;
+  return v ? TERN_EFORMAT : TERN_OK;
 }
 
 extern "C" tern_status tern_stream_read(const void* d_src, size_t bytes, int32_t mode, int32_t chunk, int32_t depth,

@@ -1,0 +1,499 @@
+// Batched (prefill) packed ternary GEMM on the 5th-generation tensor cores:
+// Y[m][n] = sum_p sum_groups s[p][n][grp] * sum_{k in grp} t[p][n][k] * xq[m][k]
+// for m >= 16 int8 tokens, bit-identical to the exact integer rule of the
+// int8 path (every fp16 scale is an integer multiple of 2^-24, so the sum is an
+// exact integer count of 2^-24, rounded once to fp32, then times the token's
+// activation scale). Formats: sasori-style additive TQ{K}P planes with fp16
+// group scales (sasori README, "How it works", "K and g"), and the BitNet
+// b1.58 single plane with one per-tensor scale (QORA-LLM-2B, "Ternary GEMV").
+//
+// Group scales without per-group promotion. An int8 MMA of K = 32 produces
+// one integer per row and token; applying a different fp16 scale to every 32
+// columns would cost several CUDA-core instructions per accumulator element
+// and K step. Instead the scale goes into the A operand: u = |s| / 2^-24 is an
+// integer below 2^40, written in D base-128 digits u_d (D from the packed
+// header: the largest scale's digit count). For digit d the A tile holds
+// sign(s) * t * u_d, which fits int8 because t is -1, 0 or +1 and u_d <= 127;
+// one tensor-memory int32 accumulator per digit then sums every group and
+// plane of the K range, and the exact result is sum_d 128^d * acc_d, formed in
+// int64 once per output. (|acc_d| <= P * 127 * 127 * K stays below 2^31 for
+// the shapes the host admits.) The tensor cores do D times the algorithmic
+// MACs; the CUDA cores only decode.
+//
+// Decode. A 2-bit code selects one of three bytes {0, a, -a} of a per-digit
+// lookup word by byte permutation (PRMT), four weights per instruction. The
+// selector nibbles come from masking the packed word, which yields the 16
+// weights of a word in the order 0,8,1,9,...,7,15; the activations are staged
+// in the same order (tc_prep_x), so every dot product sees matching pairs.
+//
+// Pipeline (one CTA per SM, persistent). Work = (128-row tile, token pass) x
+// 64-k columns; CTA c takes the contiguous range [W c / G, W (c+1) / G).
+//   warp 0     bulk async copies of each column's packed trits, scales and
+//              activations into a ring of stages (mbarrier transaction counts);
+//   warp 1     allocates tensor memory; one thread issues tcgen05.mma and
+//              commits completion to mbarriers;
+//   warps 2-9  decode A tiles (plane x digit x column) into a ring of shared
+//              slots, then drain the accumulators: a tile whose whole K range
+//              lies in this CTA is written directly; a tile cut between CTAs is
+//              summed exactly in an int64 workspace with atomic adds and
+//              finished by the last CTA to arrive (integer sums, so the order
+//              does not matter).
+// Every wait is bounded (about 1 s); on expiry the device error word records a
+// timeout and the CTA runs to completion without waiting further.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "tern_tc.cuh"
+
+namespace tern {
+
+int read_clear_dev_error_gemm_tc(void* stream, unsigned* out) { return read_clear_dev_error_tu(stream, out); }
+
+namespace {
+
+constexpr int kDecWarps = 8;
+constexpr int kThreads = 32 * (2 + kDecWarps);
+constexpr int kChunkStride = kTcRows * kChunkBytes;  // 2048: one 16-k chunk of a 128-row A tile
+constexpr int kSlotBytes = 4 * kChunkStride;         // one A tile: 128 rows x 64 k
+constexpr int kTmemCols = 512;
+
+__host__ __device__ inline uint32_t up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
+
+struct TcSmem {
+  uint32_t bars, misc, stages, slots, total;
+  uint32_t raw_bytes, sc_bytes, x_bytes, stage_bytes;
+};
+
+// Shared memory: mbarriers | misc words | stages [nstage] (raw trits of four
+// row tiles, their scales, activations) | A slots [nslot].
+__host__ __device__ inline TcSmem tc_smem(const GemmTcParams& p) {
+  TcSmem s{};
+  const int ngc = p.tq ? (p.group >= 64 ? 1 : 64 / p.group) : 0;
+  s.raw_bytes = 4u * kPlaneColBytes * p.planes;
+  s.sc_bytes = up(4u * ngc * p.planes * 64u, 128);
+  s.x_bytes = up(64u * p.xcap, 128);
+  s.stage_bytes = s.raw_bytes + s.sc_bytes + s.x_bytes;
+  const uint32_t nbar = 2u * p.nstage + 2u * p.nslot + 3u;
+  s.bars = 0;
+  s.misc = up(nbar * 8u, 16);
+  s.stages = up(s.misc + 64u, 1024);
+  s.slots = up(s.stages + (uint32_t)p.nstage * s.stage_bytes, 1024);
+  s.total = s.slots + (uint32_t)p.nslot * kSlotBytes;
+  return s;
+}
+
+// misc words
+constexpr int kMiscTmem = 0, kMiscAbort = 1, kMiscLast = 2;
+
+// Bounded wait that gives up at once when another thread of the CTA has
+// already given up (misc[kMiscAbort]), so that a failure costs about one
+// time limit, not one per wait.
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* misc) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (misc[kMiscAbort]) return false;
+    __nanosleep(it < 8 ? 20u : 100u);
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
+      misc[kMiscAbort] = 1u;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Bulk copy without a cache-policy hint (a tile's weights are read again by
+// its next token pass, so they should stay in L2).
+__device__ __forceinline__ void bulk_g2s_plain(uint32_t dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst_smem),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void named_sync_decoders() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kDecWarps) : "memory"); }
+
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+
+// Per-digit lookup words of one fp16 scale: byte 1 = sign(s) * u_d (code 01,
+// t = +1), byte 2 = its negation (code 10, t = -1), bytes 0 and 3 zero.
+__device__ __forceinline__ void scale_luts(uint32_t h, int D, uint32_t (&lut)[kTcMaxDigits]) {
+  const uint32_t ex = (h >> 10) & 31u, man = h & 1023u;
+  const uint64_t u = ex ? (uint64_t)(1024u | man) << (ex - 1u) : (uint64_t)man;
+  const bool neg = (h & 0x8000u) != 0;
+#pragma unroll
+  for (int d = 0; d < kTcMaxDigits; ++d) {
+    const int ud = (int)((u >> (7 * d)) & 127u);
+    const int a = neg ? -ud : ud;
+    lut[d] = d < D ? (((uint32_t)a & 0xFFu) << 8) | (((uint32_t)(-a) & 0xFFu) << 16) : 0u;
+  }
+}
+
+// One packed word (16 weights, 2-bit codes) -> 16 int8 A bytes in the order
+// 0,8,1,9,2,10,3,11,4,12,5,13,6,14,7,15 (selector nibble i of the masked word
+// is the code of weight 0,8,1,9,... for the low half, 4,12,5,13,... for the high).
+__device__ __forceinline__ void decode_word(uint32_t w, uint32_t lut, uint32_t a) {
+  const uint32_t lo = w & 0x33333333u, hi = (w >> 2) & 0x33333333u;
+  sts128(a, __byte_perm(lut, 0u, lo), __byte_perm(lut, 0u, lo >> 16), __byte_perm(lut, 0u, hi),
+         __byte_perm(lut, 0u, hi >> 16));
+}
+
+__device__ __forceinline__ void store_y(const GemmTcParams& p, int t, int n, long long acc) {
+  const float sx = __ldg(p.xscale + t);
+  float v;
+  if (p.tq) {
+    v = __fmul_rn(__fmul_rn(__ll2float_rn(acc), 0x1p-24f), sx);
+  } else {
+    v = __fmul_rn(__fmul_rn(__int2float_rn((int)acc), p.tensor_scale), sx);
+  }
+  const size_t o = (size_t)t * p.n + n;
+  if (p.out_bf16) {
+    static_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(v);
+  } else {
+    static_cast<float*>(p.y)[o] = v;
+  }
+}
+
+template <int P>
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmTcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const TcSmem L = tc_smem(p);
+  const int NS = p.nstage, NA = p.nslot;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* full = bars;
+  uint64_t* sfree = bars + NS;
+  uint64_t* afull = bars + 2 * NS;
+  uint64_t* afree = afull + NA;
+  uint64_t* accfull = afree + NA;
+  uint64_t* accfree = accfull + 1;
+  uint64_t* fin = accfree + 1;
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L.misc);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  int D = 1;
+  if (p.tq) D = (int)__ldg(reinterpret_cast<const unsigned*>(p.header + kDigitsOffset));
+  bool bad = D < 1 || D > kTcMaxDigits;
+  int passes = 1, tpass = 16;
+  tc_passes(bad ? 1 : D, p.m16, &passes, &tpass);
+  bad = bad || tpass > p.xcap || passes > p.passes_cap;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&sfree[i], 1);
+    }
+    for (int j = 0; j < NA; ++j) {
+      mbar_init(&afull[j], kDecWarps);
+      mbar_init(&afree[j], 1);
+    }
+    mbar_init(accfull, 1);
+    mbar_init(accfree, kDecWarps);
+    mbar_init(fin, 1);
+    misc[kMiscAbort] = 0u;
+    misc[kMiscLast] = 0u;
+    if (bad && blockIdx.x == 0) atomicOr(&g_dev_error, TERN_DEVERR_FORMAT);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(smem_u32((const void*)&misc[kMiscTmem]), kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = misc[kMiscTmem];
+
+  const int cols = p.cols;
+  const long long W = (long long)p.tiles * passes * cols;
+  const int G = p.grid;
+  long long q0 = W * blockIdx.x / G, q1 = W * (blockIdx.x + 1) / G;
+  if (bad) q1 = q0;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      const int ngc = p.tq ? (p.group >= 64 ? 1 : 64 / p.group) : 0;
+      const int groups = p.tq ? p.k / p.group : 0;
+      long long i = 0;
+      for (long long q = q0; q < q1; ++q, ++i) {
+        const int s = (int)(i % NS);
+        if (i >= NS && !tc_wait(&sfree[s], (uint32_t)((i / NS) - 1) & 1u, misc)) break;
+        if (misc[kMiscAbort]) break;
+        const int unit = (int)(q / cols), col = (int)(q % cols);
+        const int tile = unit / passes, pass = unit % passes;
+        const int nrt = min(4, p.row_tiles - 4 * tile);
+        const uint32_t scb = (uint32_t)ngc * P * 64u;
+        const uint32_t bytes = (uint32_t)nrt * (P * kPlaneColBytes + scb) + 4u * tpass * 16u;
+        const uint32_t st = smem_u32(smem + L.stages + (size_t)s * L.stage_bytes);
+        mbar_arrive_expect_tx(&full[s], bytes);
+        for (int r4 = 0; r4 < nrt; ++r4) {
+          const int rt = 4 * tile + r4;
+          bulk_g2s_plain(st + r4 * P * kPlaneColBytes, p.trit + ((size_t)rt * cols + col) * P * kPlaneColBytes,
+                         P * kPlaneColBytes, &full[s]);
+          if (p.tq) {
+            const int g0 = (col * kColK2) / p.group;
+            bulk_g2s_plain(st + L.raw_bytes + r4 * scb, p.scale + ((size_t)rt * groups + g0) * P * kTileRows, scb,
+                           &full[s]);
+          }
+        }
+        const int t0 = pass * tpass;
+        for (int w = 0; w < 4; ++w)
+          bulk_g2s_plain(st + L.raw_bytes + L.sc_bytes + w * tpass * 16,
+                         p.xp + (((size_t)col * 4 + w) * p.mp + t0) * 16, tpass * 16u, &full[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t idesc = tc::idesc_i8_s32(tpass);
+      const uint32_t slots = smem_u32(smem + L.slots);
+      long long i = 0, sc = 0;
+      int seg = 0;
+      for (long long q = q0; q < q1; ++q, ++i) {
+        if (misc[kMiscAbort]) break;
+        const int col = (int)(q % cols);
+        const bool first = q == q0 || col == 0;
+        const bool last = q == q1 - 1 || col == cols - 1;
+        const int s = (int)(i % NS);
+        if (first && seg > 0) {
+          tc_wait(accfree, (uint32_t)(seg - 1) & 1u, misc);
+          tc::fence_after_sync();
+        }
+        tc_wait(&full[s], (uint32_t)(i / NS) & 1u, misc);
+        const uint32_t xs = smem_u32(smem + L.stages + (size_t)s * L.stage_bytes + L.raw_bytes + L.sc_bytes);
+#pragma unroll
+        for (int pl = 0; pl < P; ++pl) {
+          for (int d = 0; d < D; ++d, ++sc) {
+            const int j = (int)(sc % NA);
+            tc_wait(&afull[j], (uint32_t)(sc / NA) & 1u, misc);
+            tc::fence_after_sync();
+            const uint32_t a0 = slots + (uint32_t)j * kSlotBytes;
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const uint64_t ad = tc::smem_desc(a0 + kk * 2 * kChunkStride, kChunkStride, 128);
+              const uint64_t bd = tc::smem_desc(xs + kk * 2 * tpass * 16, tpass * 16, 128);
+              tc::mma_i8(tmem + (uint32_t)(d * tpass), ad, bd, idesc, (first && pl == 0 && kk == 0) ? 0u : 1u);
+            }
+            tc::commit(&afree[j]);
+          }
+        }
+        tc::commit(&sfree[s]);
+        if (last) {
+          tc::commit(accfull);
+          ++seg;
+        }
+      }
+      // every MMA issued has completed before tensor memory is released
+      tc::commit(fin);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(fin, 0u)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
+          break;
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ decoders + epilogue
+    const int ew = warp - 2, q4 = warp & 3, h = ew >> 2;
+    const int r = 32 * q4 + lane;  // row of the 128-row tile = tensor-memory lane
+    const int ngc = p.tq ? (p.group >= 64 ? 1 : 64 / p.group) : 0;
+    const int gla = p.group >= 64 ? 0 : (32 * h) / max(p.group, 1);
+    const int glb = p.group >= 64 ? 0 : (32 * h + 16) / max(p.group, 1);
+    const uint32_t slots = smem_u32(smem + L.slots) + (uint32_t)r * kChunkBytes + (uint32_t)(2 * h) * kChunkStride;
+    const uint32_t taddr = tmem + ((uint32_t)(32 * q4) << 16);
+    long long i = 0, sc = 0;
+    int seg = 0;
+    for (long long q = q0; q < q1; ++q, ++i) {
+      const int unit = (int)(q / cols), col = (int)(q % cols);
+      const bool last = q == q1 - 1 || col == cols - 1;
+      const int s = (int)(i % NS);
+      tc_wait(&full[s], (uint32_t)(i / NS) & 1u, misc);
+      const uint32_t st = smem_u32(smem + L.stages + (size_t)s * L.stage_bytes);
+      const uint32_t raw = st + (uint32_t)(q4 * P * kPlaneColBytes + lane * kChunkBytes + 8 * h);
+      const uint32_t scs = st + L.raw_bytes + (uint32_t)(q4 * ngc * P * 64 + lane * 2);
+#pragma unroll
+      for (int pl = 0; pl < P; ++pl) {
+        const uint2 wv = lds64(raw + pl * kPlaneColBytes);
+        uint32_t la[kTcMaxDigits], lb[kTcMaxDigits];
+        if (p.tq) {
+          const uint32_t ha = lds16(scs + (uint32_t)((gla * P + pl) * 64));
+          scale_luts(ha, D, la);
+          if (glb != gla) {
+            scale_luts(lds16(scs + (uint32_t)((glb * P + pl) * 64)), D, lb);
+          } else {
+#pragma unroll
+            for (int d = 0; d < kTcMaxDigits; ++d) lb[d] = la[d];
+          }
+        } else {
+#pragma unroll
+          for (int d = 0; d < kTcMaxDigits; ++d) la[d] = lb[d] = d == 0 ? 0x00FF0100u : 0u;
+        }
+#pragma unroll
+        for (int d = 0; d < kTcMaxDigits; ++d) {
+          if (d < D) {
+            const int j = (int)(sc % NA);
+            if (sc >= NA) tc_wait(&afree[j], (uint32_t)((sc / NA) - 1) & 1u, misc);
+            const uint32_t a = slots + (uint32_t)j * kSlotBytes;
+            decode_word(wv.x, la[d], a);
+            decode_word(wv.y, lb[d], a + kChunkStride);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&afull[j]);
+            ++sc;
+          }
+        }
+      }
+      if (!last) continue;
+      // ------------------------------------------------ segment epilogue
+      const int tile = unit / passes, pass = unit % passes;
+      // the tile's whole K range lies in this CTA's range
+      const bool owned = col == cols - 1 && q0 <= (long long)unit * cols;
+      tc_wait(accfull, (uint32_t)seg & 1u, misc);
+      tc::fence_after_sync();
+      const int n = tile * kTcRows + r;
+      const int tokh = tpass >> 1, tb = h * tokh, t0 = pass * tpass;
+      for (int c8 = 0; c8 < tokh; c8 += 8) {
+        long long acc[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) acc[jj] = 0;
+#pragma unroll
+        for (int d = 0; d < kTcMaxDigits; ++d) {
+          if (d < D) {
+            uint32_t v[8];
+            tc::ld_x8_sync(taddr + (uint32_t)(d * tpass + tb + c8), v);
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) acc[jj] += (long long)(int)v[jj] << (7 * d);
+          }
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int t = t0 + tb + c8 + jj;
+          if (t < p.m && n < p.n) {
+            if (owned) {
+              store_y(p, t, n, acc[jj]);
+            } else {
+              atomicAdd(p.part + (size_t)t * p.n_pad + n, (unsigned long long)acc[jj]);
+            }
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(accfree);
+      ++seg;
+      if (!owned) {
+        // the last CTA of this tile to arrive converts the exact sums
+        __threadfence();
+        named_sync_decoders();
+        if (ew == 0 && lane == 0) {
+          const long long qa = (long long)unit * cols, qb = qa + cols - 1;
+          const long long ca = ((qa + 1) * G - 1) / W, cb = ((qb + 1) * G - 1) / W;
+          const unsigned old = atomicAdd(p.cnt + unit, 1u);
+          misc[kMiscLast] = (old + 1u == (unsigned)(cb - ca + 1)) ? 1u : 0u;
+        }
+        named_sync_decoders();
+        if (misc[kMiscLast]) {
+          __threadfence();
+          for (int tt = tb; tt < tb + tokh; ++tt) {
+            const int t = t0 + tt;
+            if (t < p.m && n < p.n) {
+              const unsigned long long v = atomicExch(p.part + (size_t)t * p.n_pad + n, 0ull);
+              store_y(p, t, n, (long long)v);
+            }
+          }
+          if (ew == 0 && lane == 0) atomicExch(p.cnt + unit, 0u);
+        }
+      }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Activations in MMA order: xp[(kc * mp + t) * 16 + j] = xq[t][16 kc + perm(j)]
+// with perm = 0,8,1,9,...,7,15 (the decode order of a packed word); zero for
+// tokens t >= m and columns k >= K.
+__global__ void tc_prep_x_kernel(const int8_t* __restrict__ xq, int m, int k, int kchunks, int mp, bool vec,
+                                 uint8_t* __restrict__ xp) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)kchunks * mp) return;
+  const int t = (int)(idx % mp), kc = (int)(idx / mp);
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (t < m) {
+    const int k0 = kc * 16;
+    const int8_t* row = xq + (size_t)t * k;
+    if (vec && k0 + 16 <= k) {
+      v = *reinterpret_cast<const uint4*>(row + k0);
+    } else {
+      uint32_t wds[4] = {0u, 0u, 0u, 0u};
+      for (int j = 0; j < 16 && k0 + j < k; ++j) wds[j >> 2] |= (uint32_t)(uint8_t)row[k0 + j] << (8 * (j & 3));
+      v = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+    }
+  }
+  const uint4 o = make_uint4(__byte_perm(v.x, v.z, 0x5140), __byte_perm(v.x, v.z, 0x7362),
+                             __byte_perm(v.y, v.w, 0x5140), __byte_perm(v.y, v.w, 0x7362));
+  reinterpret_cast<uint4*>(xp)[idx] = o;
+}
+
+template <int P>
+int launch_p(const GemmTcParams& p, void* stream) {
+  const TcSmem s = tc_smem(p);
+  auto kern = gemm_tc_kernel<P>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s.total);
+  if (e != cudaSuccess) return (int)e;
+  kern<<<p.grid, kThreads, s.total, static_cast<cudaStream_t>(stream)>>>(p);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace
+
+size_t gemm_tc_smem_bytes(const GemmTcParams& p) { return tc_smem(p).total; }
+
+int launch_gemm_tc(const GemmTcParams& p, void* stream) {
+  if (tc_smem(p).total > 227u * 1024u) return -1;
+  switch (p.planes) {
+    case 1: return launch_p<1>(p, stream);
+    case 2: return launch_p<2>(p, stream);
+    case 3: return launch_p<3>(p, stream);
+    case 4: return launch_p<4>(p, stream);
+    default: return -1;
+  }
+}
+
+int launch_tc_prep_x(const int8_t* xq, int m, int k, int kchunks, int mp, uint8_t* xp, void* stream) {
+  const long long total = (long long)kchunks * mp;
+  if (total == 0) return 0;
+  const bool vec = (reinterpret_cast<uintptr_t>(xq) & 15u) == 0 && k % 16 == 0;
+  const int threads = 256;
+  const long long blocks = (total + threads - 1) / threads;
+  tc_prep_x_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(xq, m, k, kchunks, mp, vec, xp);
+  return (int)cudaGetLastError();
+}
+
+}  // namespace tern

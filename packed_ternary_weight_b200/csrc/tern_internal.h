@@ -6,14 +6,22 @@
 #include "../../include/tern.h"
 
 #define TERN_DEVERR_TIMEOUT 1u
+#define TERN_DEVERR_FORMAT 2u  /* a kernel found packed data it cannot use */
+
+#if defined(__CUDACC__)
+#define TERN_HD __host__ __device__
+#else
+#define TERN_HD
+#endif
 
 namespace tern {
 
 // ---------------------------------------------------------------- format
 constexpr uint32_t kMagic = 0x4E524554u;  // "TERN"
-constexpr uint32_t kVersion = 1;
+constexpr uint32_t kVersion = 2;
 constexpr size_t kHeaderBytes = 256;
 constexpr size_t kCodebookOffset = 128;
+constexpr size_t kDigitsOffset = 72;  // u32: 7-bit digits of the largest TQ scale in units of 2^-24
 constexpr int kTileRows = 32;       // rows per row tile (one per lane)
 constexpr int kColK2 = 64;          // k per 16-byte chunk, 2-bit planes
 constexpr int kColK3 = 80;          // k per 16-byte chunk, base-3 planes
@@ -104,6 +112,47 @@ struct Gemv2wParams {
   int tile_begin[kMaxProblems + 1];  // first tile of each problem; [nprob] = tiles_total
   Gemv2wProblem prob[kMaxProblems];
 };
+
+// Batched GEMM on the tensor cores (tcgen05 kind::i8), m >= 16 tokens. The
+// fp16 group scale s of every (plane, row, group) is an integer u = |s| / 2^-24
+// written in D base-128 digits u_d; the A operand of digit d holds
+// sign(s) * t * u_d (int8), so one int32 accumulator per digit sums over all
+// groups and planes and the exact result is sum_d 128^d * acc_d (int64).
+constexpr int kTcRows = 128;       // weight rows per MMA tile (four 32-row tiles)
+constexpr int kTcMaxDigits = 6;    // fp16 magnitudes are below 2^40 units of 2^-24
+constexpr int kTcMaxTokens = 256;  // tokens per launch (MMA N <= 256)
+
+struct GemmTcParams {
+  const uint8_t* trit;           // trit stream
+  const uint16_t* scale;         // TQ scale stream, or nullptr
+  const uint8_t* header;         // packed header (digit count at kDigitsOffset)
+  const uint8_t* xp;             // activations in MMA order [cols*4][mp][16] (workspace)
+  const float* xscale;           // [m]
+  void* y;                       // [m][n]
+  unsigned long long* part;      // [m][n_pad] int64 partial sums (zero on entry and exit)
+  unsigned* cnt;                 // [tiles][passes_cap] arrival counters (zero on entry and exit)
+  int n, k, planes, group, cols, row_tiles, tiles, n_pad;
+  int m, m16, mp, xcap, passes_cap;
+  int tq, out_bf16;
+  float tensor_scale;
+  int nstage, nslot, grid;
+};
+
+// Token passes for D digits: the D accumulators of one pass share the 512
+// tensor-memory columns. Host and device compute the same values.
+TERN_HD inline void tc_passes(int digits, int m16, int* passes, int* tpass) {
+  int tmax = (512 / digits) & ~15;
+  if (tmax > kTcMaxTokens) tmax = kTcMaxTokens;
+  const int ps = (m16 + tmax - 1) / tmax;
+  const int t = ((m16 + ps - 1) / ps + 15) & ~15;
+  *passes = ps;
+  *tpass = t;
+}
+
+int launch_gemm_tc(const GemmTcParams& p, void* stream);  // -1: no kernel for this shape
+size_t gemm_tc_smem_bytes(const GemmTcParams& p);
+int launch_tc_prep_x(const int8_t* xq, int m, int k, int kchunks, int mp, uint8_t* xp, void* stream);
+int read_clear_dev_error_gemm_tc(void* stream, unsigned* out);
 
 // Launchers return cudaError_t values as int (0 = success).
 int launch_gemv2(const Gemv2Params& p, int xmode, bool pdl, void* stream);  // -1: no kernel

@@ -1,6 +1,10 @@
 // Host-side layout computation and packer (no device work).
 //
 // Packed buffer = 256-byte header + trit stream (+ scale stream for TQ).
+// Header (version 2): magic, version, format, N, K, planes, group, tensor
+// scale, row tiles, columns, stream offsets and sizes, at byte 72 the number
+// of base-128 digits of the largest TQ scale in units of 2^-24 (1 for BitNet,
+// 0 for d = 3), and the d = 3 codebook at byte 128.
 //
 // 2-bit planes (BitNet b1.58 layout of the QORA-LLM-2B page, "Ternary GEMV";
 // sasori TQ{K}P planes): each weight is a 2-bit code 00 -> 0, 01 -> +1,
@@ -91,6 +95,8 @@ static void write_header(uint8_t* out, const Layout& L, const tern_desc* d, cons
   uint64_t q[4] = {L.trit_offset, L.trit_bytes, L.scale_offset, L.scale_bytes};
   std::memcpy(out + 40, q, 32);
   if (L.fmt == TERN_FMT_BT3) std::memcpy(out + kCodebookOffset, codebook, 27 * sizeof(float));
+  const uint32_t digits = L.fmt == TERN_FMT_BITNET ? 1u : 0u;  // TQ: set by pack_tq_scales
+  std::memcpy(out + kDigitsOffset, &digits, 4);
 }
 
 static bool fp16_finite(uint16_t h) { return ((h >> 10) & 0x1F) != 0x1F; }
@@ -142,6 +148,17 @@ static tern_status pack_tq_scales(const Layout& L, const uint16_t* s, uint8_t* o
       for (int g = 0; g < G; ++g) tot += fp16_units(s[((size_t)p * N + n) * G + g]) * 127.0 * L.group;
     if (tot >= std::ldexp(1.0, 62)) return TERN_EFORMAT;
   }
+  // Digit count of the largest |s| / 2^-24 in base 128 (at least 1): the
+  // batched tensor-core kernel splits every scale into that many 7-bit digits.
+  uint64_t umax = 0;
+  for (size_t i = 0; i < (size_t)P * N * G; ++i) {
+    const uint32_t ex = (s[i] >> 10) & 0x1F, man = s[i] & 0x3FF;
+    const uint64_t u = ex ? (uint64_t)(1024 + man) << (ex - 1) : man;
+    umax = u > umax ? u : umax;
+  }
+  uint32_t digits = 1;
+  while (digits < 6 && (umax >> (7 * digits)) != 0) ++digits;
+  std::memcpy(out + kDigitsOffset, &digits, 4);
   uint16_t* dst = reinterpret_cast<uint16_t*>(out + L.scale_offset);
   for (int T = 0; T < L.row_tiles; ++T)
     for (int g = 0; g < G; ++g)
