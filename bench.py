@@ -63,6 +63,20 @@ def parse():
     return ap.parse_args()
 
 
+def measured_bf16_tflops():
+    """Dense bf16 tensor throughput (burst) measured on this machine, else the fallback figure."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"])
+    return 1590.0
+
+
+def header_scale_digits(buf) -> int:
+    """Digit count the packer stored in the header (u32 at byte 72)."""
+    return int(np.asarray(buf[72:76]).view("<u4")[0])
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -378,6 +392,7 @@ def run_config(args):
         layers = list(synth.tq2p_prefill_layers())
         act = tern.ACT_INT8
     peak, _ = measured_peaks()
+    bf16_peak = measured_bf16_tflops()
     rows = []
     reps = max(3, min(args.steps, 50))
     for lay in layers:
@@ -389,8 +404,6 @@ def run_config(args):
         del lay.trits
         tokens = synth.PREFILL_TOKENS if args.config == "tq2p" else (1,)
         for m in tokens:
-            if m >= 16:
-                continue                      # prefill sizes: tensor-core path, reported separately
             x = synth.draw_x_bf16(lay.seed, m, lay.k)
             xd = torch.from_numpy(x.view(np.int16)).cuda()
             ys = [torch.empty((m, lay.n), dtype=torch.float32, device="cuda") for _ in range(copies)]
@@ -435,6 +448,14 @@ def run_config(args):
             row = dict(shape=f"{lay.name} {lay.n}x{lay.k}", m=m, bytes_per_gemv=algo, copies=copies,
                        chain_us_per_gemv=round(ms_c * 1e3 / copies, 3),
                        chain_gbs=round(algo * copies / (ms_c * 1e-3) / 1e9, 1))
+            if m >= 16:
+                # tensor-core path: algorithmic int8 ops 2 m N K P (both planes' MACs)
+                ops = 2.0 * m * lay.n * lay.k * lay.planes
+                tops = ops * copies / (ms_c * 1e-3) / 1e12
+                row.update(path="tcgen05 kind::i8 (activation staging + GEMM per call)",
+                           tops=round(tops, 1), int8_peak_tops=round(2 * bf16_peak, 1),
+                           tensor_frac=round(tops / (2 * bf16_peak), 4),
+                           scale_digits=int(header_scale_digits(buf)))
             if indep is not None:
                 ms_i = timed(lambda: [g.launch(stream) for g in indep])
                 row["independent_gbs"] = round(algo * copies / (ms_i * 1e-3) / 1e9, 1)

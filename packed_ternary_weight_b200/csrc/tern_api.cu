@@ -190,8 +190,10 @@ PlanTc plan_tc(const Layout& L, int mb, int xmode, int sms) {
   PlanTc t{};
   const bool tq = L.fmt == TERN_FMT_TQ;
   if (L.fmt == TERN_FMT_BT3 || (xmode != kXInt8 && xmode != kXBf16Q8) || mb < 1 || mb > kTcMaxTokens) return t;
-  // every digit accumulator stays below 2^31: planes * 127 * 127 * K
+  // every digit accumulator stays below 2^31: planes * 127 * 127 * K; the
+  // kernel's positions (128-row tiles x token passes x columns) fit in 31 bits
   if ((long long)L.planes * 127 * 127 * L.k >= (1ll << 31)) return t;
+  if ((long long)(L.row_tiles + 3) / 4 * kTcMaxDigits * L.cols >= (1ll << 31)) return t;
   GemmTcParams& p = t.p;
   p.tq = tq;
   p.n = L.n;
@@ -233,11 +235,12 @@ PlanTc plan_tc(const Layout& L, int mb, int xmode, int sms) {
     t.sx_off = take((size_t)mb * 4);
   }
   t.total = off;
-  // three stages; as many A slots (8 KB each) as shared memory allows, up to 24
-  p.nstage = 3;
-  p.nslot = 24;
-  while (p.nslot >= 4 && gemm_tc_smem_bytes(p) > 227 * 1024) --p.nslot;
-  t.ok = p.nslot >= 4;
+  // A ring of twelve 8 KB tiles (two groups at the largest digit count); as
+  // many input stages in flight as the rest of shared memory holds, up to 12
+  p.nslot = 2 * kTcMaxDigits;
+  p.nstage = 12;
+  while (p.nstage > 2 && gemm_tc_smem_bytes(p) > 227 * 1024) --p.nstage;
+  t.ok = gemm_tc_smem_bytes(p) <= 227 * 1024;
   return t;
 }
 

@@ -32,8 +32,9 @@
 //              activations into a ring of stages (mbarrier transaction counts);
 //   warp 1     allocates tensor memory; one thread issues tcgen05.mma and
 //              commits completion to mbarriers;
-//   warps 2-9  decode A tiles (plane x digit x column) into a ring of shared
-//              slots, then drain the accumulators: a tile whose whole K range
+//   warps 2-17 decode A tiles (the D digit tiles of one plane of one column
+//              form a group of the shared ring; one warp per 32 rows and
+//              16-k chunk), then drain the accumulators: a tile whose whole K range
 //              lies in this CTA is written directly; a tile cut between CTAs is
 //              summed exactly in an int64 workspace with atomic adds and
 //              finished by the last CTA to arrive (integer sums, so the order
@@ -51,7 +52,7 @@ int read_clear_dev_error_gemm_tc(void* stream, unsigned* out) { return read_clea
 
 namespace {
 
-constexpr int kDecWarps = 8;
+constexpr int kDecWarps = 16;
 constexpr int kThreads = 32 * (2 + kDecWarps);
 constexpr int kChunkStride = kTcRows * kChunkBytes;  // 2048: one 16-k chunk of a 128-row A tile
 constexpr int kSlotBytes = 4 * kChunkStride;         // one A tile: 128 rows x 64 k
@@ -85,20 +86,35 @@ __host__ __device__ inline TcSmem tc_smem(const GemmTcParams& p) {
 // misc words
 constexpr int kMiscTmem = 0, kMiscAbort = 1, kMiscLast = 2;
 
-// Bounded wait that gives up at once when another thread of the CTA has
-// already given up (misc[kMiscAbort]), so that a failure costs about one
-// time limit, not one per wait.
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait by polling (a suspended try_wait resumes too late for the
+// one-thread roles on the critical path). Gives up at once when another thread
+// of the CTA has already given up (misc[kMiscAbort]), so that a failure costs
+// about one time limit, not one per wait.
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* misc) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (misc[kMiscAbort]) return false;
-    __nanosleep(it < 8 ? 20u : 100u);
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
-      atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
-      misc[kMiscAbort] = 1u;
-      return false;
+    if (mbar_test(bar, parity)) return true;
+    if ((it & 255u) == 0u) {
+      if (misc[kMiscAbort]) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
+        misc[kMiscAbort] = 1u;
+        return false;
+      }
     }
   }
 }
@@ -118,9 +134,9 @@ __device__ __forceinline__ void bulk_g2s_plain(uint32_t dst_smem, const void* sr
 
 __device__ __forceinline__ void named_sync_decoders() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kDecWarps) : "memory"); }
 
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
 __device__ __forceinline__ uint32_t lds16(uint32_t a) {
@@ -132,29 +148,29 @@ __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint3
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
 
-// Per-digit lookup words of one fp16 scale: byte 1 = sign(s) * u_d (code 01,
-// t = +1), byte 2 = its negation (code 10, t = -1), bytes 0 and 3 zero.
-__device__ __forceinline__ void scale_luts(uint32_t h, int D, uint32_t (&lut)[kTcMaxDigits]) {
+// Per-digit lookup words of one fp16 scale h: byte 1 = sign(s) * u_d (code
+// 01, t = +1), byte 2 = its negation (code 10, t = -1), byte 0 zero (code 00);
+// byte 3 is never selected (code 11 does not occur). u_d * 0x00FF0100 puts u_d
+// in byte 1 and -u_d mod 256 in byte 2; a negative scale swaps the two bytes.
+template <int D>
+__device__ __forceinline__ void scale_luts(uint32_t h, uint32_t (&lut)[D]) {
   const uint32_t ex = (h >> 10) & 31u, man = h & 1023u;
-  const uint64_t u = ex ? (uint64_t)(1024u | man) << (ex - 1u) : (uint64_t)man;
-  const bool neg = (h & 0x8000u) != 0;
+  const uint32_t sel = (h & 0x8000u) ? 0x3120u : 0x3210u;
+  if constexpr (D <= 4) {
+    // the largest scale has at most 4 digits, so every u is below 2^28
+    const uint32_t u = ex ? (1024u | man) << (ex - 1u) : man;
 #pragma unroll
-  for (int d = 0; d < kTcMaxDigits; ++d) {
-    const int ud = (int)((u >> (7 * d)) & 127u);
-    const int a = neg ? -ud : ud;
-    lut[d] = d < D ? (((uint32_t)a & 0xFFu) << 8) | (((uint32_t)(-a) & 0xFFu) << 16) : 0u;
+    for (int d = 0; d < D; ++d) lut[d] = __byte_perm(((u >> (7 * d)) & 127u) * 0x00FF0100u, 0u, sel);
+  } else {
+    const uint64_t u = ex ? (uint64_t)(1024u | man) << (ex - 1u) : (uint64_t)man;
+#pragma unroll
+    for (int d = 0; d < D; ++d) lut[d] = __byte_perm((uint32_t)((u >> (7 * d)) & 127u) * 0x00FF0100u, 0u, sel);
   }
 }
 
-// One packed word (16 weights, 2-bit codes) -> 16 int8 A bytes in the order
-// 0,8,1,9,2,10,3,11,4,12,5,13,6,14,7,15 (selector nibble i of the masked word
-// is the code of weight 0,8,1,9,... for the low half, 4,12,5,13,... for the high).
-__device__ __forceinline__ void decode_word(uint32_t w, uint32_t lut, uint32_t a) {
-  const uint32_t lo = w & 0x33333333u, hi = (w >> 2) & 0x33333333u;
-  sts128(a, __byte_perm(lut, 0u, lo), __byte_perm(lut, 0u, lo >> 16), __byte_perm(lut, 0u, hi),
-         __byte_perm(lut, 0u, hi >> 16));
-}
-
+// y = fl32(fl32(acc * 2^-24) * s_x) for the group-scaled sum (acc counts 2^-24,
+// converted to fp32 with one rounding), y = fl32(fl32(acc * s_w) * s_x) for the
+// single plane (acc is an exact integer below 2^24).
 __device__ __forceinline__ void store_y(const GemmTcParams& p, int t, int n, long long acc) {
   const float sx = __ldg(p.xscale + t);
   float v;
@@ -171,92 +187,80 @@ __device__ __forceinline__ void store_y(const GemmTcParams& p, int t, int n, lon
   }
 }
 
-template <int P>
-__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmTcParams p) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const TcSmem L = tc_smem(p);
-  const int NS = p.nstage, NA = p.nslot;
+__device__ __forceinline__ long long to_ll(uint32_t v) { return (long long)(int)v; }
+
+// The three roles of the kernel for P planes and D scale digits.
+// A ring: groups of D tiles (the digits of one plane of one column); a tile is
+// 128 rows x 64 k, 64 bytes per row, 64-byte swizzle.
+template <int P, int D>
+__device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, const TcSmem& L, uint32_t tmem,
+                                         volatile uint32_t* misc, int passes, int tpass, int q0, int q1, int W) {
+  const int NS = p.nstage;
+  const int NG = p.nslot / D;  // A groups in the ring
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* full = bars;
   uint64_t* sfree = bars + NS;
   uint64_t* afull = bars + 2 * NS;
-  uint64_t* afree = afull + NA;
-  uint64_t* accfull = afree + NA;
+  uint64_t* afree = afull + p.nslot;
+  uint64_t* accfull = afree + p.nslot;
   uint64_t* accfree = accfull + 1;
   uint64_t* fin = accfree + 1;
-  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L.misc);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  int D = 1;
-  if (p.tq) D = (int)__ldg(reinterpret_cast<const unsigned*>(p.header + kDigitsOffset));
-  bool bad = D < 1 || D > kTcMaxDigits;
-  int passes = 1, tpass = 16;
-  tc_passes(bad ? 1 : D, p.m16, &passes, &tpass);
-  bad = bad || tpass > p.xcap || passes > p.passes_cap;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&sfree[i], 1);
-    }
-    for (int j = 0; j < NA; ++j) {
-      mbar_init(&afull[j], kDecWarps);
-      mbar_init(&afree[j], 1);
-    }
-    mbar_init(accfull, 1);
-    mbar_init(accfree, kDecWarps);
-    mbar_init(fin, 1);
-    misc[kMiscAbort] = 0u;
-    misc[kMiscLast] = 0u;
-    if (bad && blockIdx.x == 0) atomicOr(&g_dev_error, TERN_DEVERR_FORMAT);
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tc::tmem_alloc(smem_u32((const void*)&misc[kMiscTmem]), kTmemCols);
-    tc::tmem_relinquish();
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tmem = misc[kMiscTmem];
-
   const int cols = p.cols;
-  const long long W = (long long)p.tiles * passes * cols;
   const int G = p.grid;
-  long long q0 = W * blockIdx.x / G, q1 = W * (blockIdx.x + 1) / G;
-  if (bad) q1 = q0;
+  constexpr uint32_t kGroupBytes = (uint32_t)D * kSlotBytes;
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
-    if (lane == 0) {
-      const int ngc = p.tq ? (p.group >= 64 ? 1 : 64 / p.group) : 0;
-      const int groups = p.tq ? p.k / p.group : 0;
-      long long i = 0;
-      for (long long q = q0; q < q1; ++q, ++i) {
-        const int s = (int)(i % NS);
-        if (i >= NS && !tc_wait(&sfree[s], (uint32_t)((i / NS) - 1) & 1u, misc)) break;
-        if (misc[kMiscAbort]) break;
-        const int unit = (int)(q / cols), col = (int)(q % cols);
-        const int tile = unit / passes, pass = unit % passes;
-        const int nrt = min(4, p.row_tiles - 4 * tile);
-        const uint32_t scb = (uint32_t)ngc * P * 64u;
-        const uint32_t bytes = (uint32_t)nrt * (P * kPlaneColBytes + scb) + 4u * tpass * 16u;
-        const uint32_t st = smem_u32(smem + L.stages + (size_t)s * L.stage_bytes);
-        mbar_arrive_expect_tx(&full[s], bytes);
-        for (int r4 = 0; r4 < nrt; ++r4) {
-          const int rt = 4 * tile + r4;
-          bulk_g2s_plain(st + r4 * P * kPlaneColBytes, p.trit + ((size_t)rt * cols + col) * P * kPlaneColBytes,
-                         P * kPlaneColBytes, &full[s]);
-          if (p.tq) {
-            const int g0 = (col * kColK2) / p.group;
-            bulk_g2s_plain(st + L.raw_bytes + r4 * scb, p.scale + ((size_t)rt * groups + g0) * P * kTileRows, scb,
-                           &full[s]);
-          }
+    // lane 0 waits for a free stage and posts the byte count; lanes 0-3 then
+    // copy the four row tiles' trits, lanes 4-7 their scales and lanes 8-11
+    // the activation chunks, so the copies are issued side by side
+    const int ngc = p.tq ? (p.group >= 64 ? 1 : 64 / p.group) : 0;
+    const int groups = p.tq ? p.k / p.group : 0;
+    const uint32_t scb = (uint32_t)ngc * P * 64u;
+    // positions advance one column at a time: (tile, pass, col) and the
+    // stage ring index and phase are stepped, never divided
+    int col = q0 % cols, unit = q0 / cols;
+    int tile = unit / passes, pass = unit % passes;
+    int s = 0;
+    uint32_t ph = 0;
+    for (int q = q0, i = 0; q < q1; ++q, ++i) {
+      uint32_t go = 1;
+      const int nrt = min(4, p.row_tiles - 4 * tile);
+      const uint32_t st = smem_u32(smem + L.stages) + (uint32_t)s * L.stage_bytes;
+      if (lane == 0) {
+        if (i >= NS && !tc_wait(&sfree[s], ph ^ 1u, misc)) go = 0;
+        if (misc[kMiscAbort]) go = 0;
+        if (go) mbar_arrive_expect_tx(&full[s], (uint32_t)nrt * (P * kPlaneColBytes + scb) + 4u * tpass * 16u);
+      }
+      go = __shfl_sync(0xffffffffu, go, 0);
+      if (!go) break;
+      if (lane < 4) {
+        if (lane < nrt)
+          bulk_g2s_plain(st + lane * P * kPlaneColBytes,
+                         p.trit + ((size_t)(4 * tile + lane) * cols + col) * (P * kPlaneColBytes), P * kPlaneColBytes,
+                         &full[s]);
+      } else if (lane < 8) {
+        const int r4 = lane - 4;
+        if (p.tq && r4 < nrt)
+          bulk_g2s_plain(st + L.raw_bytes + r4 * scb,
+                         p.scale + ((size_t)(4 * tile + r4) * groups + (col * kColK2) / p.group) * P * kTileRows, scb,
+                         &full[s]);
+      } else if (lane < 12) {
+        const int w = lane - 8;
+        bulk_g2s_plain(st + L.raw_bytes + L.sc_bytes + w * tpass * 16,
+                       p.xp + (((size_t)col * 4 + w) * p.mp + (size_t)pass * tpass) * 16, tpass * 16u, &full[s]);
+      }
+      if (++col == cols) {
+        col = 0;
+        if (++pass == passes) {
+          pass = 0;
+          ++tile;
         }
-        const int t0 = pass * tpass;
-        for (int w = 0; w < 4; ++w)
-          bulk_g2s_plain(st + L.raw_bytes + L.sc_bytes + w * tpass * 16,
-                         p.xp + (((size_t)col * 4 + w) * p.mp + t0) * 16, tpass * 16u, &full[s]);
+      }
+      if (++s == NS) {
+        s = 0;
+        ph ^= 1u;
       }
     }
     __syncwarp();
@@ -265,40 +269,50 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     if (lane == 0) {
       const uint32_t idesc = tc::idesc_i8_s32(tpass);
       const uint32_t slots = smem_u32(smem + L.slots);
-      long long i = 0, sc = 0;
-      int seg = 0;
-      for (long long q = q0; q < q1; ++q, ++i) {
+      int col = q0 % cols, s = 0, j = 0, seg = 0;
+      uint32_t ph = 0, aph = 0;
+      for (int q = q0; q < q1; ++q) {
         if (misc[kMiscAbort]) break;
-        const int col = (int)(q % cols);
         const bool first = q == q0 || col == 0;
         const bool last = q == q1 - 1 || col == cols - 1;
-        const int s = (int)(i % NS);
         if (first && seg > 0) {
           tc_wait(accfree, (uint32_t)(seg - 1) & 1u, misc);
           tc::fence_after_sync();
         }
-        tc_wait(&full[s], (uint32_t)(i / NS) & 1u, misc);
-        const uint32_t xs = smem_u32(smem + L.stages + (size_t)s * L.stage_bytes + L.raw_bytes + L.sc_bytes);
+        tc_wait(&full[s], ph, misc);
+        const uint32_t xs = smem_u32(smem + L.stages) + (uint32_t)s * L.stage_bytes + L.raw_bytes + L.sc_bytes;
+        const uint64_t bd0 = tc::smem_desc(xs, tpass * 16, 128);
+        const uint64_t bd1 = tc::smem_desc(xs + 2 * tpass * 16, tpass * 16, 128);
 #pragma unroll
         for (int pl = 0; pl < P; ++pl) {
-          for (int d = 0; d < D; ++d, ++sc) {
-            const int j = (int)(sc % NA);
-            tc_wait(&afull[j], (uint32_t)(sc / NA) & 1u, misc);
-            tc::fence_after_sync();
-            const uint32_t a0 = slots + (uint32_t)j * kSlotBytes;
+          tc_wait(&afull[j], aph, misc);
+          tc::fence_after_sync();
+          const uint32_t a0 = slots + (uint32_t)j * kGroupBytes;
+          // the D accumulators are independent: interleave them so that
+          // consecutive instructions do not wait on one another
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-              const uint64_t ad = tc::smem_desc(a0 + kk * 2 * kChunkStride, kChunkStride, 128);
-              const uint64_t bd = tc::smem_desc(xs + kk * 2 * tpass * 16, tpass * 16, 128);
-              tc::mma_i8(tmem + (uint32_t)(d * tpass), ad, bd, idesc, (first && pl == 0 && kk == 0) ? 0u : 1u);
-            }
-            tc::commit(&afree[j]);
+          for (int d = 0; d < D; ++d)
+            tc::mma_i8(tmem + (uint32_t)(d * tpass), tc::smem_desc_sw64(a0 + (uint32_t)d * kSlotBytes, 512), bd0, idesc,
+                       first && pl == 0 ? 0u : 1u);
+#pragma unroll
+          for (int d = 0; d < D; ++d)
+            tc::mma_i8(tmem + (uint32_t)(d * tpass), tc::smem_desc_sw64(a0 + (uint32_t)d * kSlotBytes + 32, 512), bd1,
+                       idesc, 1u);
+          tc::commit(&afree[j]);
+          if (++j == NG) {
+            j = 0;
+            aph ^= 1u;
           }
         }
         tc::commit(&sfree[s]);
         if (last) {
           tc::commit(accfull);
           ++seg;
+        }
+        if (++col == cols) col = 0;
+        if (++s == NS) {
+          s = 0;
+          ph ^= 1u;
         }
       }
       // every MMA issued has completed before tensor memory is released
@@ -314,80 +328,81 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     __syncwarp();
   } else {
     // ------------------------------------------------ decoders + epilogue
-    const int ew = warp - 2, q4 = warp & 3, h = ew >> 2;
-    const int r = 32 * q4 + lane;  // row of the 128-row tile = tensor-memory lane
+    // warp (q4, c): rows 32 q4 .. 32 q4 + 31 (tensor-memory lane quarter
+    // warp % 4), chunk c (16 k) of every column, and a quarter of the tokens
+    // in the epilogue
+    const int ew = warp - 2, q4 = warp & 3, c = ew >> 2;
+    const int r = 32 * q4 + lane;
     const int ngc = p.tq ? (p.group >= 64 ? 1 : 64 / p.group) : 0;
-    const int gla = p.group >= 64 ? 0 : (32 * h) / max(p.group, 1);
-    const int glb = p.group >= 64 ? 0 : (32 * h + 16) / max(p.group, 1);
-    const uint32_t slots = smem_u32(smem + L.slots) + (uint32_t)r * kChunkBytes + (uint32_t)(2 * h) * kChunkStride;
+    const int gl = p.tq && p.group < 64 ? (16 * c) / p.group : 0;
+    // A tiles in the 64-byte swizzled K-major layout: row r at 64 r, its
+    // 16-byte chunk c at chunk position c ^ ((r >> 1) & 3)
+    const uint32_t slots = smem_u32(smem + L.slots) + (uint32_t)r * 64u + (uint32_t)((c ^ ((r >> 1) & 3)) * 16);
     const uint32_t taddr = tmem + ((uint32_t)(32 * q4) << 16);
-    long long i = 0, sc = 0;
-    int seg = 0;
-    for (long long q = q0; q < q1; ++q, ++i) {
-      const int unit = (int)(q / cols), col = (int)(q % cols);
+    int col = q0 % cols, unit = q0 / cols, s = 0, j = 0, seg = 0, gc = 0;
+    uint32_t ph = 0, aph = 0;
+    for (int q = q0; q < q1; ++q) {
       const bool last = q == q1 - 1 || col == cols - 1;
-      const int s = (int)(i % NS);
-      tc_wait(&full[s], (uint32_t)(i / NS) & 1u, misc);
-      const uint32_t st = smem_u32(smem + L.stages + (size_t)s * L.stage_bytes);
-      const uint32_t raw = st + (uint32_t)(q4 * P * kPlaneColBytes + lane * kChunkBytes + 8 * h);
-      const uint32_t scs = st + L.raw_bytes + (uint32_t)(q4 * ngc * P * 64 + lane * 2);
+      tc_wait(&full[s], ph, misc);
+      const uint32_t st = smem_u32(smem + L.stages) + (uint32_t)s * L.stage_bytes;
+      const uint32_t raw = st + (uint32_t)(q4 * P * kPlaneColBytes + lane * kChunkBytes + 4 * c);
+      const uint32_t scs = st + L.raw_bytes + (uint32_t)((q4 * ngc + gl) * P * 64 + lane * 2);
+      if (++s == NS) {
+        s = 0;
+        ph ^= 1u;
+      }
 #pragma unroll
-      for (int pl = 0; pl < P; ++pl) {
-        const uint2 wv = lds64(raw + pl * kPlaneColBytes);
-        uint32_t la[kTcMaxDigits], lb[kTcMaxDigits];
+      for (int pl = 0; pl < P; ++pl, ++gc) {
+        const uint32_t w = lds32(raw + pl * kPlaneColBytes);
+        uint32_t lut[D];
         if (p.tq) {
-          const uint32_t ha = lds16(scs + (uint32_t)((gla * P + pl) * 64));
-          scale_luts(ha, D, la);
-          if (glb != gla) {
-            scale_luts(lds16(scs + (uint32_t)((glb * P + pl) * 64)), D, lb);
-          } else {
-#pragma unroll
-            for (int d = 0; d < kTcMaxDigits; ++d) lb[d] = la[d];
-          }
+          scale_luts<D>(lds16(scs + (uint32_t)(pl * 64)), lut);
         } else {
 #pragma unroll
-          for (int d = 0; d < kTcMaxDigits; ++d) la[d] = lb[d] = d == 0 ? 0x00FF0100u : 0u;
+          for (int d = 0; d < D; ++d) lut[d] = 0x00FF0100u;
         }
+        const uint32_t lo = w & 0x33333333u, hi = (w >> 2) & 0x33333333u;
+        const uint32_t lo2 = lo >> 16, hi2 = hi >> 16;
+        if (gc >= NG) tc_wait(&afree[j], aph ^ 1u, misc);
+        const uint32_t a = slots + (uint32_t)j * kGroupBytes;
 #pragma unroll
-        for (int d = 0; d < kTcMaxDigits; ++d) {
-          if (d < D) {
-            const int j = (int)(sc % NA);
-            if (sc >= NA) tc_wait(&afree[j], (uint32_t)((sc / NA) - 1) & 1u, misc);
-            const uint32_t a = slots + (uint32_t)j * kSlotBytes;
-            decode_word(wv.x, la[d], a);
-            decode_word(wv.y, lb[d], a + kChunkStride);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&afull[j]);
-            ++sc;
-          }
+        for (int d = 0; d < D; ++d)
+          sts128(a + (uint32_t)d * kSlotBytes, __byte_perm(lut[d], 0u, lo), __byte_perm(lut[d], 0u, lo2),
+                 __byte_perm(lut[d], 0u, hi), __byte_perm(lut[d], 0u, hi2));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[j]);
+        if (++j == NG) {
+          j = 0;
+          aph ^= 1u;
         }
+      }
+      const int ucur = unit;
+      if (++col == cols) {
+        col = 0;
+        ++unit;
       }
       if (!last) continue;
       // ------------------------------------------------ segment epilogue
-      const int tile = unit / passes, pass = unit % passes;
+      const int tile = ucur / passes, pass = ucur % passes;
       // the tile's whole K range lies in this CTA's range
-      const bool owned = col == cols - 1 && q0 <= (long long)unit * cols;
+      const bool owned = col == 0 && q0 <= ucur * cols;
       tc_wait(accfull, (uint32_t)seg & 1u, misc);
       tc::fence_after_sync();
       const int n = tile * kTcRows + r;
-      const int tokh = tpass >> 1, tb = h * tokh, t0 = pass * tpass;
-      for (int c8 = 0; c8 < tokh; c8 += 8) {
-        long long acc[8];
+      const int tq4 = tpass >> 2, tb = c * tq4, t0 = pass * tpass;
+      for (int c4 = 0; c4 < tq4; c4 += 4) {
+        long long acc[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) acc[jj] = 0;
+        for (int d = 0; d < D; ++d) {
+          uint32_t v[4];
+          tc::ld_x4_sync(taddr + (uint32_t)(d * tpass + tb + c4), v);
 #pragma unroll
-        for (int d = 0; d < kTcMaxDigits; ++d) {
-          if (d < D) {
-            uint32_t v[8];
-            tc::ld_x8_sync(taddr + (uint32_t)(d * tpass + tb + c8), v);
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) acc[jj] += (long long)(int)v[jj] << (7 * d);
-          }
+          for (int jj = 0; jj < 4; ++jj) acc[jj] += to_ll(v[jj]) << (7 * d);
         }
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const int t = t0 + tb + c8 + jj;
+        for (int jj = 0; jj < 4; ++jj) {
+          const int t = t0 + tb + c4 + jj;
           if (t < p.m && n < p.n) {
             if (owned) {
               store_y(p, t, n, acc[jj]);
@@ -406,25 +421,83 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         __threadfence();
         named_sync_decoders();
         if (ew == 0 && lane == 0) {
-          const long long qa = (long long)unit * cols, qb = qa + cols - 1;
+          const long long qa = (long long)ucur * cols, qb = qa + cols - 1;
           const long long ca = ((qa + 1) * G - 1) / W, cb = ((qb + 1) * G - 1) / W;
-          const unsigned old = atomicAdd(p.cnt + unit, 1u);
+          const unsigned old = atomicAdd(p.cnt + ucur, 1u);
           misc[kMiscLast] = (old + 1u == (unsigned)(cb - ca + 1)) ? 1u : 0u;
         }
         named_sync_decoders();
         if (misc[kMiscLast]) {
           __threadfence();
-          for (int tt = tb; tt < tb + tokh; ++tt) {
+          for (int tt = tb; tt < tb + tq4; ++tt) {
             const int t = t0 + tt;
             if (t < p.m && n < p.n) {
               const unsigned long long v = atomicExch(p.part + (size_t)t * p.n_pad + n, 0ull);
               store_y(p, t, n, (long long)v);
             }
           }
-          if (ew == 0 && lane == 0) atomicExch(p.cnt + unit, 0u);
+          if (ew == 0 && lane == 0) atomicExch(p.cnt + ucur, 0u);
         }
       }
     }
+  }
+}
+
+template <int P>
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmTcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const TcSmem L = tc_smem(p);
+  const int NS = p.nstage, NA = p.nslot;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L.misc);
+  const int warp = threadIdx.x >> 5;
+
+  int D = 1;
+  if (p.tq) D = (int)__ldg(reinterpret_cast<const unsigned*>(p.header + kDigitsOffset));
+  bool bad = D < 1 || D > kTcMaxDigits || (P > 1 && !p.tq) || NA / (D < 1 ? 1 : D) < 1;
+  int passes = 1, tpass = 16;
+  tc_passes(bad ? 1 : D, p.m16, &passes, &tpass);
+  bad = bad || tpass > p.xcap || passes > p.passes_cap;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&bars[i], 1);       // full
+      mbar_init(&bars[NS + i], 1);  // sfree
+    }
+    for (int j = 0; j < NA; ++j) {
+      mbar_init(&bars[2 * NS + j], kDecWarps);  // afull
+      mbar_init(&bars[2 * NS + NA + j], 1);     // afree
+    }
+    mbar_init(&bars[2 * NS + 2 * NA], 1);              // accfull
+    mbar_init(&bars[2 * NS + 2 * NA + 1], kDecWarps);  // accfree
+    mbar_init(&bars[2 * NS + 2 * NA + 2], 1);          // fin
+    misc[kMiscAbort] = 0u;
+    misc[kMiscLast] = 0u;
+    if (bad && blockIdx.x == 0) atomicOr(&g_dev_error, TERN_DEVERR_FORMAT);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(smem_u32((const void*)&misc[kMiscTmem]), kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = misc[kMiscTmem];
+
+  // positions fit in 32 bits (the host checks tiles x 4 passes x columns)
+  const int W = p.tiles * passes * p.cols;
+  const int G = p.grid;
+  const int q0 = (int)((long long)W * blockIdx.x / G);
+  const int q1 = bad ? q0 : (int)((long long)W * (blockIdx.x + 1) / G);
+
+  switch (D) {
+    case 1: tc_roles<P, 1>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
+    case 2: tc_roles<P, 2>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
+    case 3: tc_roles<P, 3>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
+    case 4: tc_roles<P, 4>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
+    case 5: tc_roles<P, 5>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
+    default: tc_roles<P, 6>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
   }
 
   tc::fence_before_sync();

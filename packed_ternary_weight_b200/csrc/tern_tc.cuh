@@ -36,6 +36,16 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
+// Shared-memory matrix descriptor, 64-byte swizzle, K-major: rows of 64 bytes,
+// 8-row atoms of 512 bytes (16-byte chunk c of row r stored at chunk
+// c ^ ((r >> 1) & 3)); stride byte offset between 8-row groups, leading byte
+// offset unused (1), swizzle mode 4 at bits 61-63. The atom base must be
+// 512-byte aligned; a K offset inside the 64-byte row is added to the start.
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t addr, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | (1ull << 16) | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) |
+         (4ull << 61);
+}
+
 // Instruction descriptor of kind::i8 with signed A and B, int32 accumulator,
 // both operands K-major, M = 128 rows, N columns (16..256, multiple of 16).
 __host__ __device__ constexpr uint32_t idesc_i8_s32(int n) {
@@ -69,6 +79,16 @@ __device__ __forceinline__ void ld_x8_sync(uint32_t taddr, uint32_t (&v)[8]) {
       "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
       : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+      : "r"(taddr)
+      : "memory");
+}
+
+// Four consecutive 32-bit columns of this warp's lane quarter, as ld_x8_sync.
+__device__ __forceinline__ void ld_x4_sync(uint32_t taddr, uint32_t (&v)[4]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3])
       : "r"(taddr)
       : "memory");
 }
