@@ -6,9 +6,9 @@ projections (q/o 2560x2560, k/v 640x2560, gate/up 6912x2560, down
 2560x6912), batch 1, single ternary plane with a per-tensor scale, int8
 per-token absmax activations, fp32 output, each GEMV with its own seeded
 weights and activations. One step = the layer set's 210 GEMVs, which have no
-data dependencies on one another: one grouped launch per projection shape
-(30 GEMVs each), every GEMV quantising its bf16 activation per token inside
-the kernel (521 MB of packed weights, so every step streams from HBM: inputs
+data dependencies on one another: one grouped launch per input width (the
+180 GEMVs with K = 2560, then the 30 down projections), every GEMV quantising
+its bf16 activation per token inside the kernel (521 MB of packed weights, so every step streams from HBM: inputs
 larger than L2). The same GEMVs run in decode order -- per layer [q,k,v] ->
 o -> [gate,up] -> down, each launch waiting for the previous one -- are
 reported alongside as "decode_chain".
@@ -175,8 +175,12 @@ def run_ours(args, rank, world):
     indep = {nm: grouped([L for L in layers if L["name"] == nm]) for nm, _, _ in synth.BITNET_2B_SHAPES}
 
     # the step: the layer set's 210 independent GEMVs, one grouped launch per
-    # projection shape (activations quantised per token inside each GEMV)
-    step_launches = [indep[nm] for nm, _, _ in synth.BITNET_2B_SHAPES]
+    # input width K (q,k,v,o,gate,up share K = 2560: 180 GEMVs; down: 30),
+    # activations quantised per token inside each GEMV
+    by_k = {}
+    for L in layers:
+        by_k.setdefault(L["k"], []).append(L)
+    step_launches = [grouped(Ls) for _, Ls in sorted(by_k.items())]
 
     def step():
         for g in step_launches:
@@ -334,9 +338,9 @@ def run_ours(args, rank, world):
         "data": "synthetic (seeded ternary weights P(-1)=P(+1)=0.3, bf16 N(0,1) activations)",
         "config": {"workload": WORKLOAD, "layers": args.layers, "gemvs_per_step": len(layers),
                    "launches_per_step": len(step_launches),
-                   "order": "one launch per projection shape carrying the 30 layers' copies of it as independent "
-                            "GEMVs (the layer set's GEMVs have no data dependencies); decode-order figures in "
-                            "decode_chain",
+                   "order": "one grouped launch per input width K (the 180 GEMVs with K = 2560, then the 30 "
+                            "down projections) as independent GEMVs (the layer set's GEMVs have no data "
+                            "dependencies); decode-order figures in decode_chain, per-shape launches in per_shape",
                    "l2": "inputs larger than L2 (packed weights per step %.1f MB vs 126 MB L2)" % (
                        sum(L["wbytes"] for L in layers) / 1e6),
                    "parallelism": "replicas" if world > 1 else "single GPU"},

@@ -163,7 +163,7 @@ tern_status tern_gemm_batched(const tern_desc* desc, const void* d_packed, int32
  * and v projections of a decode step, or gate and up). The pages state one
  * GEMV per projection (QORA-LLM-2B, "SubLN Pattern"); running independent
  * ones together is a launch-level choice of this library.
- *   count       1..32 problems; descs[i] must share fmt, k, planes, group and
+ *   count       1..256 problems; descs[i] must share fmt, k, planes, group and
  *               flags (n may differ).
  *   d_packed[i], d_x[i] ([K]), d_xscale[i] (TERN_ACT_INT8, else ignored and may
  *               be NULL), d_y[i] ([n_i]): as tern_gemv, one per problem.

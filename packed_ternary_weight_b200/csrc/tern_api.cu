@@ -2,6 +2,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstddef>
 #include <cstdint>
 
 #include "tern_internal.h"
@@ -125,7 +126,8 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
 // over the SMs by K splits in the row-group kernel).
 bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, int sms, Gemv2wParams& p) {
   if (L.fmt == TERN_FMT_BT3) return false;
-  int begin[kMaxProblems + 1];
+  if (nprob > kMaxProblemsW) return false;
+  int begin[kMaxProblemsW + 1];
   begin[0] = 0;
   for (int i = 0; i < nprob; ++i) begin[i + 1] = begin[i] + row_tiles[i];
   const int T = begin[nprob];
@@ -155,6 +157,7 @@ bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, in
     const int t0 = (int)((long long)T * c / p.grid), t1 = (int)((long long)T * (c + 1) / p.grid);
     xs = std::max(xs, prob_of(t1 - 1) - prob_of(t0) + 1);
   }
+  if (xs > kMaxSlotsW) return false;
   p.xslots = xs;
   const int colb = L.planes * kPlaneColBytes;
   p.stage_cols = std::max(p.gcols, (6144 / colb) / p.gcols * p.gcols);
@@ -164,8 +167,10 @@ bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, in
   for (const auto& sh : kShapes) {
     p.nw = sh[0];
     p.nstage = sh[1];
-    // the kernel adds its shared copy of the problem table
-    if (gemv2w_smem_bytes(p, xmode) + sizeof(Gemv2wProblem) * kMaxProblems + 4 * (kMaxProblems + 1) <= 227 * 1024)
+    // the kernel adds its shared copy of the parameter block's head and of
+    // its problems
+    if (gemv2w_smem_bytes(p, xmode) + offsetof(Gemv2wParams, prob) + sizeof(Gemv2wProblem) * kMaxSlotsW <=
+        227 * 1024)
       return true;
   }
   return false;
@@ -447,10 +452,10 @@ extern "C" tern_status tern_gemv(const tern_desc* desc, const void* d_packed, te
 extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, const void* const* d_packed,
                                          tern_act act, const void* const* d_x, const float* const* d_xscale,
                                          tern_out out, void* const* d_y, void* stream) {
-  if (count < 1 || count > kMaxProblems || !descs || !d_packed || !d_x || !d_y) return TERN_EINVAL;
+  if (count < 1 || count > kMaxProblemsW || !descs || !d_packed || !d_x || !d_y) return TERN_EINVAL;
   if (act == TERN_ACT_INT8 && !d_xscale) return TERN_EINVAL;
-  Layout L[kMaxProblems];
-  int rt[kMaxProblems];
+  static thread_local Layout L[kMaxProblemsW];
+  int rt[kMaxProblemsW];
   for (int i = 0; i < count; ++i) {
     tern_status st = check_one(&descs[i], d_packed[i], act, d_x[i], d_xscale ? d_xscale[i] : nullptr, out, d_y[i],
                                &L[i]);
@@ -466,7 +471,8 @@ extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, 
   const int sms = device_sms();
   const bool pdl = (descs[0].flags & TERN_F_PDL) != 0;
   {
-    Gemv2wParams w{};
+    static thread_local Gemv2wParams w;
+    w = Gemv2wParams{};
     if (plan_gemv2w(L[0], rt, count, xmode, sms, w)) {
       w.out_bf16 = out == TERN_OUT_BF16;
       bool vec = L[0].k % 16 == 0;
@@ -489,32 +495,38 @@ extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, 
       return rc == 0 ? TERN_OK : TERN_ECUDA;
     }
   }
-  const Plan2 pl = plan_gemv2(L[0], rt, count, 1, xmode, sms, false);
-  if (!pl.ok) return TERN_EUNSUPPORTED;
-  Gemv2Params p{};
-  fill_common(p, L[0], pl, 1, out);
-  p.nprob = count;
-  int cta = 0;
-  bool vec = L[0].k % 16 == 0;
-  for (int i = 0; i < count; ++i) {
-    const uint8_t* base = static_cast<const uint8_t*>(d_packed[i]);
-    Gemv2Problem& q = p.prob[i];
-    q.trit = base + L[i].trit_offset;
-    q.scale = p.tq ? reinterpret_cast<const uint16_t*>(base + L[i].scale_offset) : nullptr;
-    q.x = d_x[i];
-    q.xscale = d_xscale ? d_xscale[i] : nullptr;
-    q.y = d_y[i];
-    q.n = L[i].n;
-    q.row_tiles = L[i].row_tiles;
-    q.cta_begin = cta;
-    q.tensor_scale = descs[i].tensor_scale;
-    cta += (L[i].row_tiles + pl.wpc - 1) / pl.wpc;
-    vec = vec && aligned16(q.x);
+  // the row-group kernel takes up to kMaxProblems problems per launch
+  for (int c0 = 0; c0 < count; c0 += kMaxProblems) {
+    const int nc = std::min(kMaxProblems, count - c0);
+    const Plan2 pl = plan_gemv2(L[c0], rt + c0, nc, 1, xmode, sms, false);
+    if (!pl.ok) return TERN_EUNSUPPORTED;
+    Gemv2Params p{};
+    fill_common(p, L[c0], pl, 1, out);
+    p.nprob = nc;
+    int cta = 0;
+    bool vec = L[0].k % 16 == 0;
+    for (int j = 0; j < nc; ++j) {
+      const int i = c0 + j;
+      const uint8_t* base = static_cast<const uint8_t*>(d_packed[i]);
+      Gemv2Problem& q = p.prob[j];
+      q.trit = base + L[i].trit_offset;
+      q.scale = p.tq ? reinterpret_cast<const uint16_t*>(base + L[i].scale_offset) : nullptr;
+      q.x = d_x[i];
+      q.xscale = d_xscale ? d_xscale[i] : nullptr;
+      q.y = d_y[i];
+      q.n = L[i].n;
+      q.row_tiles = L[i].row_tiles;
+      q.cta_begin = cta;
+      q.tensor_scale = descs[i].tensor_scale;
+      cta += (L[i].row_tiles + pl.wpc - 1) / pl.wpc;
+      vec = vec && aligned16(q.x);
+    }
+    p.x_vec = vec;
+    const int rc = L[0].fmt == TERN_FMT_BT3 ? launch_gemv3(p, pdl, stream) : launch_gemv2(p, xmode, pdl, stream);
+    if (rc < 0) return TERN_EUNSUPPORTED;
+    if (rc != 0) return TERN_ECUDA;
   }
-  p.x_vec = vec;
-  const int rc = L[0].fmt == TERN_FMT_BT3 ? launch_gemv3(p, pdl, stream) : launch_gemv2(p, xmode, pdl, stream);
-  if (rc < 0) return TERN_EUNSUPPORTED;
-  return rc == 0 ? TERN_OK : TERN_ECUDA;
+  return TERN_OK;
 }
 
 extern "C" tern_status tern_device_error(void* stream) {

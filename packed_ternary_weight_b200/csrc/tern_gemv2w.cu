@@ -27,6 +27,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <cstddef>
 #include <type_traits>
 
 #include "tern_gemv_common.cuh"
@@ -160,8 +161,25 @@ __device__ __forceinline__ long long fold_fp16_exact(uint16_t h, int S) {
 // XM: activation mode; P: planes; WG: words (16 k) per scale group, 0 = one
 // per-tensor scale (BitNet).
 template <int XM, int P, int WG>
-__global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ Gemv2wParams p) {
+__global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ Gemv2wParams pg) {
   extern __shared__ __align__(128) uint8_t smem[];
+  // The parameter block is copied to shared memory in two parallel rounds of
+  // parameter reads (scalars and problem boundaries, then this CTA's problems):
+  // each dependent round of parameter reads costs on the order of a
+  // microsecond at launch (every SM misses at once), so nothing below reads
+  // the parameter space again. Only the members before `prob` are valid in
+  // the shared copy; the problems live in `sprob`.
+  constexpr int kHeadBytes = (int)offsetof(Gemv2wParams, prob);
+  static_assert(kHeadBytes % 4 == 0 && sizeof(Gemv2wProblem) % 4 == 0, "copied as 32-bit words");
+  __shared__ __align__(16) unsigned char shead[kHeadBytes];
+  __shared__ __align__(16) Gemv2wProblem sprob[kMaxSlotsW];
+  {
+    const int* src = reinterpret_cast<const int*>(&pg);
+    int* dst = reinterpret_cast<int*>(shead);
+    for (int i = threadIdx.x; i < kHeadBytes / 4; i += blockDim.x) dst[i] = src[i];
+  }
+  __syncthreads();
+  const Gemv2wParams& p = *reinterpret_cast<const Gemv2wParams*>(shead);
   constexpr bool kTQ = WG > 0;
   constexpr bool kBf = XM == kXBf16;
   const Plan2w sp = plan2w(p, XM);
@@ -172,12 +190,9 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
   // the planner keeps tiles x CTAs and columns x warps below 2^31). The tiles'
   // problem boundaries are searched in shared memory, and only the problems
   // of this CTA's tiles are copied there (slot s = problem qa + s).
-  __shared__ int stb[kMaxProblems + 1];
-  __shared__ Gemv2wProblem sprob[kMaxProblems];
-  if (threadIdx.x <= p.nprob) stb[threadIdx.x] = p.tile_begin[threadIdx.x];
+  const int* stb = p.tile_begin;
   const int t0 = (int)((unsigned)(p.tiles_total * blockIdx.x) / gridDim.x);
   const int t1 = (int)((unsigned)(p.tiles_total * (blockIdx.x + 1)) / gridDim.x);
-  __syncthreads();
   auto prob_of = [&](int t) {  // the last problem whose first tile is <= t
     int lo = 0, hi = p.nprob - 1;
     while (lo < hi) {
@@ -186,8 +201,13 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
     }
     return lo;
   };
-  const int qa = prob_of(t0), nslots = prob_of(t1 - 1) - qa + 1;
-  if (threadIdx.x < nslots) sprob[threadIdx.x] = p.prob[qa + threadIdx.x];
+  const int qa = prob_of(t0), nslots = min(kMaxSlotsW, prob_of(t1 - 1) - qa + 1);  // the host keeps it <= 16
+  {  // slot s = problem qa + s
+    constexpr int kPw = (int)(sizeof(Gemv2wProblem) / 4);
+    const int* src = reinterpret_cast<const int*>(&pg.prob[qa]);
+    int* dst = reinterpret_cast<int*>(sprob);
+    for (int i = threadIdx.x; i < nslots * kPw; i += blockDim.x) dst[i] = src[i];
+  }
   __syncthreads();
   const int gcols = p.gcols;
   const int cg = (t1 - t0) * cols / gcols;  // granules in this CTA
@@ -248,6 +268,10 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
     }
   };
   pdl_launch_dependents();
+  // weights depend on no preceding kernel: with a programmatic dependent
+  // launch the first stages are requested before the dependency wait
+  if (p.early_w && lane == 0)
+    for (int i = 0; i < nst; ++i) issue_next();
 
   // ---- activations of every problem this CTA touches (after the producer of
   // x). Each warp requests its first weight stages only once its activation
@@ -274,6 +298,10 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
       const int f = threadIdx.x + i * nthr;
       xr[i] = f < nflat ? chunk_load(f) : make_uint4(0, 0, 0, 0);
     }
+    // the activation loads are on their way: request the first weight stages
+    // now, so that the ring fills while the activations are staged
+    if (!p.early_w && lane == 0)
+      for (int i = 0; i < nst; ++i) issue_next();
     unsigned* amax = reinterpret_cast<unsigned*>(mx);  // token maxima (bits of non-negative floats)
     if (threadIdx.x < nslots) amax[threadIdx.x] = 0u;
     __syncthreads();
@@ -297,9 +325,6 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
         const int f = f0 + lane;
         chunk_max(f, f < nflat ? chunk_load(f) : make_uint4(0, 0, 0, 0));
       }
-      __syncwarp();
-      if (lane == 0)
-        for (int i = 0; i < nst; ++i) issue_next();
       __syncthreads();
     }
     // int8 image (per-token quantisation with the rule of tern_quantize_act:
@@ -330,11 +355,6 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
       if (f < nflat) put(f, xr[i]);
     }
     for (int f = threadIdx.x + kXR * nthr; f < nflat; f += nthr) put(f, chunk_load(f));
-    if constexpr (!kQ8) {
-      __syncwarp();
-      if (lane == 0)
-        for (int i = 0; i < nst; ++i) issue_next();
-    }
     if (threadIdx.x < nslots) {
       float sx;
       if constexpr (kQ8) {
@@ -363,6 +383,8 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
     }
     __syncthreads();
   } else {
+    if (!p.early_w && lane == 0)
+      for (int i = 0; i < nst; ++i) issue_next();
     for (int s = 0; s < nslots; ++s) {
       uint8_t* sl = slot_ptr(s);
       gemv_common::stage_x_bf16_image(static_cast<const uint16_t*>(sprob[s].x), p.k, p.group, 0, sp.kx,
@@ -370,8 +392,6 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
                                       reinterpret_cast<long long*>(sl + sp.sum_off),
                                       reinterpret_cast<float*>(sl + sp.sx_off));
     }
-    if (lane == 0)
-      for (int i = 0; i < nst; ++i) issue_next();
     __syncthreads();
   }
   if constexpr (!kTQ) {
@@ -619,7 +639,9 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
 
 // ------------------------------------------------------------------ launch
 template <int XM, int P, int WG>
-static int launch_w(const Gemv2wParams& p, bool pdl, void* stream) {
+static int launch_w(const Gemv2wParams& p0, bool pdl, void* stream) {
+  Gemv2wParams p = p0;
+  p.early_w = pdl ? 1 : 0;
   const Plan2w sp = plan2w(p, XM);
   auto kern = gemv2w_kernel<XM, P, WG>;
   // at least half of an SM's shared memory, so that CTAs never share an SM

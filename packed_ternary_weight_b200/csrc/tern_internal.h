@@ -46,7 +46,9 @@ tern_status layout_of(const tern_desc* d, Layout* L);
 //            exact int8 path (same result as tern_quantize_act + kXInt8).
 enum XMode : int { kXInt8 = 0, kXBf16 = 1, kXBf16Q8 = 2 };
 
-constexpr int kMaxProblems = 32;  // independent GEMVs in one grouped launch
+constexpr int kMaxProblems = 32;   // independent GEMVs in one launch of the row-group kernel
+constexpr int kMaxProblemsW = 256; // ... of the one-CTA-per-SM kernel (parameter block < 32 KB)
+constexpr int kMaxSlotsW = 16;     // problems one CTA of that kernel may touch
 constexpr int kMaxCluster = 16;   // K-splits reduced through one thread-block cluster
 
 struct Gemv2Problem {
@@ -109,8 +111,9 @@ struct Gemv2wParams {
   int stage_cols, nstage;   // per-warp ring: columns per stage, stages
   int xslots;               // activation images resident per CTA
   int x_vec;                // activations may be read with 16-byte loads
-  int tile_begin[kMaxProblems + 1];  // first tile of each problem; [nprob] = tiles_total
-  Gemv2wProblem prob[kMaxProblems];
+  int early_w;              // set at launch: weights may be requested before the dependency wait
+  int tile_begin[kMaxProblemsW + 1];  // first tile of each problem; [nprob] = tiles_total
+  Gemv2wProblem prob[kMaxProblemsW];  // last member: the kernel copies only its own problems
 };
 
 // Batched GEMM on the tensor cores (tcgen05 kind::i8), m >= 16 tokens. The
