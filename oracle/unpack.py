@@ -23,10 +23,12 @@ Format (all little-endian):
 * TQ scales: fp16 scale of (T, group G, plane p, row r) at
   scale_offset + ((T*groups + G)*P + p)*64 + 2*r.
 * Balanced ternary d = 3: a column is 80 consecutive k of a 32-row tile, 1632
-  bytes at trit_offset + (T*cols + c)*1632. Its first 1536 bytes are three
-  digit planes (p = 0, 1, 2 for the trits of weight 1, 3, 9), 16 bytes per row
-  at p*512 + 16*r; byte i holds five base-3 digits u_j = t + 1 (first digit
-  least significant) for k = 80c + 16j + i, j = 0..4. The last 96 bytes hold the
+  bytes at trit_offset + (T*cols + c)*1632. Its first 1536 bytes hold, per row
+  r, 16 byte triples: byte b (0..2) of triple i at b*512 + 16*r + i. Every byte
+  holds five base-3 digits u = t + 1 (first digit least significant); the 15
+  digits of triple i, byte 0 first, are the trits t0, t1, t2 (weights 1, 3, 9)
+  of k = 80c + i, then of k = 80c + 16 + i, ..., then of k = 80c + 64 + i
+  (weight j of the triple, j = 0..4, is k = 80c + 16j + i). The last 96 bytes hold the
   scale indices of the column's five groups of 16: byte d (0..2) of row r, at
   1536 + 32*d + r, holds base-3 digit d of the index of group 5c + j as its
   digit j. Padding trits are 0 (digit 1), padding indices 0.
@@ -103,11 +105,13 @@ def _unpack_bt3(buf: np.ndarray, h: dict):
     n, k, T, C = h["n"], h["k"], h["row_tiles"], h["cols"]
     raw = np.asarray(buf, dtype=np.uint8)[h["trit_offset"]:h["trit_offset"] + h["trit_bytes"]]
     col = raw.reshape(T, C, 1632)
-    planes = col[:, :, :1536].reshape(T, C, 3, 32, 16)            # [T][c][p][r][i]
-    dig = _base3_digits(planes)                                   # [T][c][p][r][i][j]
+    tri = col[:, :, :1536].reshape(T, C, 3, 32, 16)               # [T][c][b][r][i]
+    dig = _base3_digits(tri)                                      # [T][c][b][r][i][q]
+    # digit s = 5b + q of the triple; trit p of weight j is digit 3j + p
+    dig = dig.transpose(0, 1, 3, 4, 2, 5).reshape(T, C, 32, 16, 5, 3)  # [T][c][r][i][j][p]
     t = (dig - 1).astype(np.int8)
     # k = 80c + 16j + i
-    t = t.transpose(2, 0, 3, 1, 5, 4).reshape(3, T * 32, C * 80)
+    t = t.transpose(5, 0, 2, 1, 4, 3).reshape(3, T * 32, C * 80)
     ib = col[:, :, 1536:].reshape(T, C, 3, 32)                   # [T][c][d][r]
     idig = _base3_digits(ib)                                      # [T][c][d][r][j]
     idx = idig[:, :, 0] + 3 * idig[:, :, 1] + 9 * idig[:, :, 2]   # [T][c][r][j]

@@ -3,23 +3,27 @@
 // log-spaced scale codebook; weight = cb[idx] * (9 t2 + 3 t1 + t0)), bf16
 // activations.
 //
-// Layout of one 80-k column of a 32-row tile (the packer's): three digit
-// planes of 16 bytes per row, byte i holding the digits u = t + 1 of
-// k = 80c + 16j + i as its base-3 digit j (j = 0..4), then three bytes per row
-// holding the base-3 digits of the five groups' codebook indices. Digit j of
-// the 16 bytes of a row is exactly group 5c + j.
+// Layout of one 80-k column of a 32-row tile (the packer's): per row, 16 byte
+// triples; triple i holds the digits u = t + 1 of the five weights
+// k = 80c + 16j + i (j = 0..4), weight by weight (u0, u1, u2 of weight j are
+// base-3 digits 3j .. 3j+2 of the triple, five digits per byte, first digit
+// least significant), byte b of every triple in the b-th 16-byte chunk of the
+// row; then three bytes per row holding the base-3 digits of the five groups'
+// codebook indices. Weight j of the 16 triples of a row is group 5c + j.
 //
 // Work split, weight stream, K-splits and persistence follow the 2-bit kernel:
 // one warp per 32-row tile and K-split, per-warp rings of shared-memory stages
 // filled by 1-D bulk async copies on mbarriers, splits reduced in a
 // thread-block cluster, persistent CTAs when K is not split.
 //
-// Decode (per lane = one row, per 4 bytes of a plane): the bytes are spread
-// into two 16-bit lanes each and their five digits extracted with the exact
-// reciprocal floor(v / 3) = (171 v) >> 9 (v <= 242), both lanes at once.
-// U = u0 + 3 u1 + 9 u2 = level + 13 in 0..26 is formed in byte lanes and
-// dotted with the 24-bit fixed-point image of the activations (same as the
-// 2-bit bf16 path) with byte dot-products, so the group sum is
+// Decode (per lane = one row, per 4 triples): the 12 bytes are spread into
+// 16-bit lanes (two triples per 32-bit register) and the five levels
+// U = u0 + 3 u1 + 9 u2 = level + 13 in 0..26 read with exact multiply-shift
+// divisions, both lanes at once (byte 0 = U0 + 27 h1; byte 1 = l1 + 3 U2 +
+// 81 h3; byte 2 = l3 + 9 U4; U1 = h1 + 9 l1, U3 = h3 + 3 l3), about 0.8
+// integer operations per trit. The levels, four per register in byte lanes,
+// are dotted with the 24-bit fixed-point image of the activations (same as
+// the 2-bit bf16 path) with byte dot-products, so the group sum is
 // sum U q - 13 sum q, exact in integers; each group is then scaled once,
 // cb[idx] * 2^(E-22), and accumulated in fp32.
 #include <cuda_bf16.h>
@@ -80,6 +84,25 @@ __device__ __forceinline__ void digits5(uint32_t v, uint32_t (&d)[5]) {
     v = q;
   }
   d[4] = v;
+}
+
+// The five levels of the triples held in the 16-bit lanes of b0, b1, b2 (the
+// triples' bytes 0, 1, 2; every byte <= 242). Exact in both lanes:
+// floor(v / 27) = (19 v) >> 9 (v <= 242), floor(v / 3) = (171 v) >> 9,
+// floor(v / 9) = (57 v) >> 9; no lane carries into the other (products < 2^16,
+// differences >= 0).
+__device__ __forceinline__ void triple_levels(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t (&U)[5]) {
+  constexpr uint32_t kM = 0x007F007Fu;
+  const uint32_t h1 = ((b0 * 19u) >> 9) & kM;  // u0 + 3 u1 of weight 1
+  U[0] = b0 - 27u * h1;
+  const uint32_t r = ((b1 * 171u) >> 9) & kM;  // b1 / 3
+  const uint32_t l1 = b1 - 3u * r;             // u2 of weight 1
+  const uint32_t h3 = ((r * 19u) >> 9) & kM;   // u0 of weight 3
+  U[2] = r - 27u * h3;
+  U[4] = ((b2 * 57u) >> 9) & kM;
+  const uint32_t l3 = b2 - 9u * U[4];          // u1 + 3 u2 of weight 3
+  U[1] = h1 + 9u * l1;
+  U[3] = h3 + 3u * l3;
 }
 
 __device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {
@@ -223,19 +246,12 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
           const uint4 b2 = lds128<2 * kPlaneColBytes>(col + lane * 16);
           auto word_u = [&](auto wi_c, uint32_t w0, uint32_t w1, uint32_t w2) {
             constexpr int w = decltype(wi_c)::value;
-            uint32_t l0[5], h0[5], l1[5], h1[5], l2[5], h2[5];
-            digits5(w0 & 0x00FF00FFu, l0);
-            digits5((w0 >> 8) & 0x00FF00FFu, h0);
-            digits5(w1 & 0x00FF00FFu, l1);
-            digits5((w1 >> 8) & 0x00FF00FFu, h1);
-            digits5(w2 & 0x00FF00FFu, l2);
-            digits5((w2 >> 8) & 0x00FF00FFu, h2);
+            uint32_t ue[5], uo[5];
+            triple_levels(w0 & 0x00FF00FFu, w1 & 0x00FF00FFu, w2 & 0x00FF00FFu, ue);  // triples 4w, 4w+2
+            triple_levels((w0 >> 8) & 0x00FF00FFu, (w1 >> 8) & 0x00FF00FFu, (w2 >> 8) & 0x00FF00FFu,
+                          uo);  // triples 4w+1, 4w+3
 #pragma unroll
-            for (int j = 0; j < 5; ++j) {
-              const uint32_t ul = l0[j] + 3u * l1[j] + 9u * l2[j];  // bytes 0, 2 in 16-bit lanes
-              const uint32_t uh = h0[j] + 3u * h1[j] + 9u * h2[j];  // bytes 1, 3
-              U[w][j] = ul | (uh << 8);
-            }
+            for (int j = 0; j < 5; ++j) U[w][j] = ue[j] | (uo[j] << 8);
           };
           word_u(std::integral_constant<int, 0>{}, b0.x, b1.x, b2.x);
           word_u(std::integral_constant<int, 1>{}, b0.y, b1.y, b2.y);

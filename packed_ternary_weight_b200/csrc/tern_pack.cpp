@@ -19,10 +19,15 @@
 //
 // Balanced ternary d = 3 (Entrit card, "Quantization details"): digits
 // u = t + 1 are packed five per byte in base 3 (first digit least
-// significant). A column covers 80 k of a 32-row tile: three digit planes of
-// 16 bytes per row, byte i holding k = 80c + 16j + i as its digit j, so digit j
-// of the 16 bytes is exactly group 5c + j of 16 weights; then three bytes per
-// row holding the base-3 digits of the five groups' codebook indices.
+// significant). A column covers 80 k of a 32-row tile. Per row it holds 16
+// byte triples: triple i carries the 15 trits of the five weights
+// k = 80c + 16j + i (j = 0..4, one weight of each of the column's five groups
+// of 16), weight by weight (t0, t1, t2 of weight j are trits 3j, 3j+1, 3j+2 of
+// the triple, trits 5b..5b+4 in byte b); byte b of triple i sits at
+// b * 512 + 16 r + i. Then three bytes per row holding the base-3 digits of the
+// five groups' codebook indices. Keeping the three trits of a weight together
+// lets the decoder read a weight's level U = u0 + 3 u1 + 9 u2 with a few
+// divisions by 3, 9 and 27 instead of extracting every digit.
 #include <cmath>
 #include <cstring>
 #include <vector>
@@ -181,19 +186,22 @@ static tern_status pack_bt3(const Layout& L, const int8_t* trits, const uint8_t*
   for (int T = 0; T < L.row_tiles; ++T) {
     for (int c = 0; c < L.cols; ++c) {
       uint8_t* col = base + ((size_t)T * L.cols + c) * kBt3ColBytes;
-      for (int p = 0; p < 3; ++p)
-        for (int r = 0; r < kTileRows; ++r) {
-          const int n = T * kTileRows + r;
-          for (int i = 0; i < 16; ++i) {
+      for (int r = 0; r < kTileRows; ++r) {
+        const int n = T * kTileRows + r;
+        for (int i = 0; i < 16; ++i) {
+          unsigned dig[15];  // the triple's trits, weight-major
+          for (int j = 0; j < 5; ++j) {
+            const int k = c * kColK3 + 16 * j + i;
+            for (int p = 0; p < 3; ++p)
+              dig[3 * j + p] = (n < N && k < K) ? (unsigned)(trits[((size_t)p * N + n) * K + k] + 1) : 1u;
+          }
+          for (int b = 0; b < 3; ++b) {
             unsigned v = 0, pw = 1;
-            for (int j = 0; j < 5; ++j, pw *= 3) {
-              const int k = c * kColK3 + 16 * j + i;
-              const unsigned u = (n < N && k < K) ? (unsigned)(trits[((size_t)p * N + n) * K + k] + 1) : 1u;
-              v += u * pw;
-            }
-            col[p * kPlaneColBytes + r * kChunkBytes + i] = (uint8_t)v;
+            for (int q = 0; q < 5; ++q, pw *= 3) v += dig[5 * b + q] * pw;
+            col[b * kPlaneColBytes + r * kChunkBytes + i] = (uint8_t)v;
           }
         }
+      }
       for (int dgt = 0; dgt < 3; ++dgt)
         for (int r = 0; r < kTileRows; ++r) {
           const int n = T * kTileRows + r;

@@ -103,8 +103,10 @@ def test_bitnet_bytes_by_hand():
 
 def test_bt3_bytes_by_hand():
     # one row, K = 16 (one group): t0[3] = +1 (digit 2), everything else 0
-    # (digit 1). Byte i holds k = 16 j + i as digit j, so byte 3 of plane 0 is
-    # 2 + 3 + 9 + 27 + 81 = 122 and every other byte is 1+3+9+27+81 = 121.
+    # (digit 1). Triple i holds the trits of k = 16 j + i (j = 0..4), weight by
+    # weight, five digits per byte: triple 3 starts with the digits 2, 1, 1 of
+    # k = 3, so its byte 0 is 2 + 3 + 9 + 27 + 81 = 122 and every other byte is
+    # 1 + 3 + 9 + 27 + 81 = 121.
     # The group's index 14 = 2 + 1*3 + 1*9: index byte d holds digit d of it as
     # digit 0 and 0 (padding groups) elsewhere -> 2, 1, 1.
     t = np.zeros((3, 1, 16), np.int8)
@@ -121,6 +123,29 @@ def test_bt3_bytes_by_hand():
     assert np.array_equal(buf[128:128 + 108].view("<f4"), cb)
     u = oracle.unpack(buf)
     assert np.array_equal(u["trits"], t) and u["idx"].tolist() == [[14]]
+
+
+def test_bt3_triple_order_by_hand():
+    # one row, K = 32 (two groups): t1[0] = -1 and t2[16] = +1, everything else
+    # 0. Triple 0 carries k = 0, 16, 32, 48, 64 (the last three are padding,
+    # digits 1 1 1). Its 15 digits, weight by weight (t0, t1, t2):
+    #   k = 0: 1 0 1 | k = 16: 1 1 2 | padding: 1 1 1, 1 1 1, 1 1 1
+    # byte 0 = digits 1 0 1 1 1 (s = 0..4)   -> 1 + 0*3 + 1*9 + 1*27 + 1*81 = 118
+    # byte 1 = digits 2 1 1 1 1 (s = 5..9)   -> 2 + 3 + 9 + 27 + 81 = 122
+    # byte 2 = digits 1 1 1 1 1 (s = 10..14) -> 121
+    # (a plane-major layout, five k of one plane per byte, would give 121, 120
+    # and 124 instead)
+    t = np.zeros((3, 1, 32), np.int8)
+    t[1, 0, 0] = -1
+    t[2, 0, 16] = 1
+    idx = np.array([[0, 26]], np.uint8)
+    d = tern.make_desc("bt3", 1, 32, 3, 16)
+    buf = tern.pack(d, t, scale_idx=idx, codebook=synth.codebook27())
+    col = buf[256:]
+    assert (col[0], col[512], col[1024]) == (118, 122, 121)
+    assert col[1] == 121 and col[512 + 1] == 121 and col[1024 + 15] == 121
+    u = oracle.unpack(buf)
+    assert np.array_equal(u["trits"], t) and u["idx"].tolist() == [[0, 26]]
 
 
 # ------------------------------------------------------------------ sizes
