@@ -125,7 +125,8 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
 // the launch has at least four tiles per SM (smaller launches are spread
 // over the SMs by K splits in the row-group kernel).
 bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, int sms, Gemv2wParams& p) {
-  if (L.fmt == TERN_FMT_BT3) return false;
+  const bool bt3 = L.fmt == TERN_FMT_BT3;
+  if (bt3 && xmode != kXBf16) return false;
   if (nprob > kMaxProblemsW) return false;
   int begin[kMaxProblemsW + 1];
   begin[0] = 0;
@@ -142,6 +143,7 @@ bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, in
   p.group = L.group;
   p.groups = L.groups;
   p.cols = L.cols;
+  p.bt3 = bt3;
   p.gcols = (tq && L.group >= 64) ? L.group / 64 : 1;
   p.nprob = nprob;
   p.tiles_total = T;
@@ -159,7 +161,7 @@ bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, in
   }
   if (xs > kMaxSlotsW) return false;
   p.xslots = xs;
-  const int colb = L.planes * kPlaneColBytes;
+  const int colb = bt3 ? kBt3ColBytes : L.planes * kPlaneColBytes;
   p.stage_cols = std::max(p.gcols, (6144 / colb) / p.gcols * p.gcols);
   // (warps, stages): sixteen warps with two 6 KB stages each measured best on
   // the BitNet-2B layer set; fewer when the activation images need the room

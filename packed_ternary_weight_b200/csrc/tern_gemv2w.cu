@@ -57,6 +57,7 @@ struct Plan2w {
 //           integer paths: int8 x [kx] | int32 sums (BitNet: prefix sums per column [cols+1];
 //                          TQ: per group [groups]) | fp32 token scale
 //           bf16 path:     high, middle, low bytes [kx] each | int64 group sums | fp32 2^(E-22) per group
+//                          (| fp32 codebook [27] for balanced ternary d = 3)
 //   red   [nw][2][32] partial row sums of shared tiles (8 bytes each)
 //   cnt   [nw] arrival counters of shared tiles
 //   misc  per-warp maxima [xslots][nw] for the in-kernel quantisation
@@ -64,13 +65,18 @@ __host__ __device__ inline Plan2w plan2w(const Gemv2wParams& p, int xmode) {
   Plan2w s{};
   const bool tq = p.tq != 0;
   const bool bf = xmode == kXBf16;
-  s.kx = p.cols * kColK2;
+  s.kx = p.cols * (p.bt3 ? kColK3 : kColK2);
   const int gps = tq ? (p.stage_cols * kColK2 + p.group - 1) / p.group : 0;
-  s.stage_bytes = (int)align_up((size_t)p.stage_cols * p.planes * kPlaneColBytes + (size_t)gps * p.planes * 64, 128);
+  const size_t colb = p.bt3 ? (size_t)kBt3ColBytes : (size_t)p.planes * kPlaneColBytes;
+  s.stage_bytes = (int)align_up((size_t)p.stage_cols * colb + (size_t)gps * p.planes * 64, 128);
   if (bf) {
+    // the image covers whole columns: d = 3 pads K to a multiple of 80, so it
+    // holds kx / 16 groups (TQ: K is a multiple of 64, kx = K)
+    const size_t gimg = p.bt3 ? (size_t)s.kx / 16 : (size_t)p.groups;
     s.sum_off = 3 * (size_t)s.kx;
-    s.sx_off = s.sum_off + 8 * (size_t)p.groups;  // here: 2^(E-22) per group
-    s.slot_bytes = align_up(s.sx_off + 4 * (size_t)p.groups, 128);
+    s.sx_off = s.sum_off + 8 * gimg;  // here: 2^(E-22) per group
+    // d = 3: the 27-entry codebook follows the per-group multipliers
+    s.slot_bytes = align_up(s.sx_off + 4 * gimg + (p.bt3 ? 27 * 4 : 0), 128);
   } else {
     s.sum_off = s.kx;
     s.sx_off = align_up(s.sum_off + 4 * (size_t)(tq ? p.groups : p.cols + 1), 16);
@@ -148,6 +154,12 @@ __device__ void prefix_columns(int* sums, int cols) {
   }
 }
 
+__device__ __forceinline__ uint32_t lds_u8w(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ long long fold_fp16_exact(uint16_t h, int S) {
   const int ex = (h >> 10) & 0x1F, man = h & 0x3FF;
   int mm = ex ? man + 1024 : man;
@@ -159,7 +171,8 @@ __device__ __forceinline__ long long fold_fp16_exact(uint16_t h, int S) {
 }  // namespace
 
 // XM: activation mode; P: planes; WG: words (16 k) per scale group, 0 = one
-// per-tensor scale (BitNet).
+// per-tensor scale (BitNet), -1 = balanced ternary d = 3 (base-3 columns of
+// 80 k with the group indices inside, group 16, bf16 activations, P = 3).
 template <int XM, int P, int WG>
 __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ Gemv2wParams pg) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -181,7 +194,10 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
   __syncthreads();
   const Gemv2wParams& p = *reinterpret_cast<const Gemv2wParams*>(shead);
   constexpr bool kTQ = WG > 0;
+  constexpr bool kB3 = WG < 0;
   constexpr bool kBf = XM == kXBf16;
+  static_assert(!kB3 || (kBf && P == 3), "balanced ternary: bf16 activations, three digit planes");
+  constexpr int kColB = kB3 ? kBt3ColBytes : P * kPlaneColBytes;  // bytes per tile column
   const Plan2w sp = plan2w(p, XM);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = p.nw, nst = p.nstage, sc = p.stage_cols, cols = p.cols;
@@ -243,7 +259,7 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
     const int T = t0 + rp - stb[qp];
     const int slot = islot;
     islot = islot + 1 == nst ? 0 : islot + 1;
-    const uint32_t tb = (uint32_t)ncols * P * kPlaneColBytes;
+    const uint32_t tb = (uint32_t)ncols * kColB;
     uint8_t* dst = ring + (size_t)slot * sp.stage_bytes;
     uint32_t sb = 0;
     int ga = 0;
@@ -253,7 +269,7 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
       sb = (uint32_t)(gb - ga) * P * 64;
     }
     mbar_arrive_expect_tx(&bars[slot], tb + sb);
-    bulk_g2s(dst, pq.trit + ((size_t)T * cols + ccp) * P * kPlaneColBytes, tb, &bars[slot], pol);
+    bulk_g2s(dst, pq.trit + ((size_t)T * cols + ccp) * kColB, tb, &bars[slot], pol);
     if constexpr (kTQ)
       bulk_g2s(dst + (size_t)sc * P * kPlaneColBytes,
                reinterpret_cast<const uint8_t*>(pq.scale) + ((size_t)T * p.groups + ga) * P * 64, sb, &bars[slot],
@@ -387,6 +403,12 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
       for (int i = 0; i < nst; ++i) issue_next();
     for (int s = 0; s < nslots; ++s) {
       uint8_t* sl = slot_ptr(s);
+      if constexpr (kB3) {
+        // the codebook from the packed header (the trit stream starts right after it)
+        if (threadIdx.x < 27)
+          reinterpret_cast<float*>(sl + sp.sx_off + (size_t)sp.kx / 4)[threadIdx.x] =
+              reinterpret_cast<const float*>(sprob[s].trit - kHeaderBytes + kCodebookOffset)[threadIdx.x];
+      }
       gemv_common::stage_x_bf16_image(static_cast<const uint16_t*>(sprob[s].x), p.k, p.group, 0, sp.kx,
                                       reinterpret_cast<int8_t*>(sl), sl + sp.kx, sl + 2 * (size_t)sp.kx,
                                       reinterpret_cast<long long*>(sl + sp.sum_off),
@@ -394,7 +416,7 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
     }
     __syncthreads();
   }
-  if constexpr (!kTQ) {
+  if constexpr (!kTQ && !kB3) {  // single plane: column sums -> prefix sums
     for (int s = warp; s < nslots; s += nw) prefix_columns(reinterpret_cast<int*>(slot_ptr(s) + sp.sum_off), cols);
     __syncthreads();
   }
@@ -575,7 +597,7 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
       }
     };
     auto load_w = [&](int j, uint4* wv) {
-      const uint32_t wc = st32 + (uint32_t)(j * P * kPlaneColBytes);
+      const uint32_t wc = st32 + (uint32_t)(j * kColB);
       wv[0] = lds128<0>(wc);
       if constexpr (P > 1) wv[1] = lds128<kPlaneColBytes>(wc);
       if constexpr (P > 2) wv[2] = lds128<2 * kPlaneColBytes>(wc);
@@ -590,11 +612,63 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
         xw[3] = lds128<48>(xc);
       }
     };
+    // balanced ternary d = 3: one 80-k column of this lane's row (16 byte
+    // triples in wv[0..2], the five group indices in three bytes after the
+    // digit chunks), five groups of 16 folded with their codebook scales
+    auto column3 = [&](const uint4* wv, int cc) {
+      const uint32_t cbase = st32 - (uint32_t)(lane * 16) + (uint32_t)((cc - ccc) * kColB);
+      uint32_t ia[5], ib[5];
+      gemv_common::digits5(lds_u8w(cbase + 3 * kPlaneColBytes + lane) |
+                               (lds_u8w(cbase + 3 * kPlaneColBytes + 32 + lane) << 16),
+                           ia);
+      gemv_common::digits5(lds_u8w(cbase + 3 * kPlaneColBytes + 64 + lane), ib);
+      uint32_t U[4][5];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t w0 = w == 0 ? wv[0].x : w == 1 ? wv[0].y : w == 2 ? wv[0].z : wv[0].w;
+        const uint32_t w1 = w == 0 ? wv[1].x : w == 1 ? wv[1].y : w == 2 ? wv[1].z : wv[1].w;
+        const uint32_t w2 = w == 0 ? wv[2].x : w == 1 ? wv[2].y : w == 2 ? wv[2].z : wv[2].w;
+        uint32_t ue[5], uo[5];
+        gemv_common::triple_levels(w0 & 0x00FF00FFu, w1 & 0x00FF00FFu, w2 & 0x00FF00FFu, ue);
+        gemv_common::triple_levels((w0 >> 8) & 0x00FF00FFu, (w1 >> 8) & 0x00FF00FFu, (w2 >> 8) & 0x00FF00FFu, uo);
+#pragma unroll
+        for (int j = 0; j < 5; ++j) U[w][j] = ue[j] | (uo[j] << 8);
+      }
+      const float* cbk = gmul + sp.kx / 16;  // the codebook follows the kx / 16 group multipliers
+#pragma unroll
+      for (int j = 0; j < 5; ++j) {
+        const uint32_t xo = (uint32_t)(cc * kColK3 + 16 * j);
+        const uint4 hv = lds128<0>(x32 + xo), mv = lds128<0>(x32 + (uint32_t)sp.kx + xo),
+                    lv = lds128<0>(x32 + 2u * (uint32_t)sp.kx + xo);
+        int H = 0;
+        unsigned M = 0, L = 0;
+        H = dp4a_us(U[0][j], (int)hv.x, H);
+        H = dp4a_us(U[1][j], (int)hv.y, H);
+        H = dp4a_us(U[2][j], (int)hv.z, H);
+        H = dp4a_us(U[3][j], (int)hv.w, H);
+        M = dp4a_uu(U[0][j], mv.x, M);
+        M = dp4a_uu(U[1][j], mv.y, M);
+        M = dp4a_uu(U[2][j], mv.z, M);
+        M = dp4a_uu(U[3][j], mv.w, M);
+        L = dp4a_uu(U[0][j], lv.x, L);
+        L = dp4a_uu(U[1][j], lv.y, L);
+        L = dp4a_uu(U[2][j], lv.z, L);
+        L = dp4a_uu(U[3][j], lv.w, L);
+        const int g = cc * kBt3Groups + j;
+        const long long S = ((long long)H * 65536 + (long long)M * 256 + L) - 13ll * gsum64[g];
+        const uint32_t idx = (ia[j] & 0xFFFFu) + 3u * (ia[j] >> 16) + 9u * ib[j];
+        yacc = fmaf(cbk[idx] * gmul[g], __ll2float_rn(S), yacc);
+      }
+    };
     auto column = [&](const uint4* wv, const uint4* xw, int cc) {
-      word_step(std::integral_constant<int, 0>{}, wv, xw, cc);
-      word_step(std::integral_constant<int, 1>{}, wv, xw, cc);
-      word_step(std::integral_constant<int, 2>{}, wv, xw, cc);
-      word_step(std::integral_constant<int, 3>{}, wv, xw, cc);
+      if constexpr (kB3) {
+        column3(wv, cc);
+      } else {
+        word_step(std::integral_constant<int, 0>{}, wv, xw, cc);
+        word_step(std::integral_constant<int, 1>{}, wv, xw, cc);
+        word_step(std::integral_constant<int, 2>{}, wv, xw, cc);
+        word_step(std::integral_constant<int, 3>{}, wv, xw, cc);
+      }
     };
     // two columns per trip, each one's shared loads issued a column ahead
     // (the load after the last column re-reads it and is not used)
@@ -679,6 +753,7 @@ size_t gemv2w_smem_bytes(const Gemv2wParams& p, int xmode) { return plan2w(p, xm
   }
 
 int launch_gemv2w(const Gemv2wParams& p, int xmode, bool pdl, void* stream) {
+  if (p.bt3) return (xmode == kXBf16 && p.planes == 3) ? launch_w<kXBf16, 3, -1>(p, pdl, stream) : -1;
   if (!p.tq) {
     if (p.planes != 1) return -1;
     if (xmode == kXInt8) return launch_w<kXInt8, 1, 0>(p, pdl, stream);

@@ -41,6 +41,8 @@ int read_clear_dev_error_gemv3(void* stream, unsigned* out) { return read_clear_
 namespace {
 
 using gemv_common::align_up;
+using gemv_common::digits5;
+using gemv_common::triple_levels;
 
 struct Smem3 {
   size_t bars, ring, xa, xb, xc, gsum, gmult, cb, red, total;
@@ -73,36 +75,6 @@ __host__ __device__ inline Smem3 smem3_plan(const Gemv2Params& p) {
   off = align_up(off + ((p.cluster && p.ks > 1) ? (size_t)p.ks * p.wpc * 32 * 4 : 0), 16);
   s.total = off;
   return s;
-}
-
-// Five base-3 digits of the two values (each <= 242) held in the 16-bit lanes of v.
-__device__ __forceinline__ void digits5(uint32_t v, uint32_t (&d)[5]) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t q = ((v * 171u) >> 9) & 0x007F007Fu;  // floor(v / 3) in both lanes
-    d[j] = v - 3u * q;
-    v = q;
-  }
-  d[4] = v;
-}
-
-// The five levels of the triples held in the 16-bit lanes of b0, b1, b2 (the
-// triples' bytes 0, 1, 2; every byte <= 242). Exact in both lanes:
-// floor(v / 27) = (19 v) >> 9 (v <= 242), floor(v / 3) = (171 v) >> 9,
-// floor(v / 9) = (57 v) >> 9; no lane carries into the other (products < 2^16,
-// differences >= 0).
-__device__ __forceinline__ void triple_levels(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t (&U)[5]) {
-  constexpr uint32_t kM = 0x007F007Fu;
-  const uint32_t h1 = ((b0 * 19u) >> 9) & kM;  // u0 + 3 u1 of weight 1
-  U[0] = b0 - 27u * h1;
-  const uint32_t r = ((b1 * 171u) >> 9) & kM;  // b1 / 3
-  const uint32_t l1 = b1 - 3u * r;             // u2 of weight 1
-  const uint32_t h3 = ((r * 19u) >> 9) & kM;   // u0 of weight 3
-  U[2] = r - 27u * h3;
-  U[4] = ((b2 * 57u) >> 9) & kM;
-  const uint32_t l3 = b2 - 9u * U[4];          // u1 + 3 u2 of weight 3
-  U[1] = h1 + 9u * l1;
-  U[3] = h3 + 3u * l3;
 }
 
 __device__ __forceinline__ uint32_t lds_u8(uint32_t addr) {

@@ -105,6 +105,7 @@ struct Gemv2wParams {
   int nprob, tiles_total;
   int grid;                 // CTAs (at most one per SM)
   int tq, k, planes, group, groups, cols;
+  int bt3;                  // balanced ternary d = 3 columns (80 k, 1632 bytes per tile column)
   int gcols;                // columns per granule of the warp ranges (a whole scale group)
   int out_bf16;
   int nw;                   // warps per CTA

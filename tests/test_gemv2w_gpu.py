@@ -147,3 +147,39 @@ def test_bf16_deterministic(tern):
     for r in runs[1:]:
         for a, b in zip(runs[0], r):
             assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+def bt3_check(layers, ys, xbits, nrows, outs16=None):
+    for i, (lay, y, x) in enumerate(zip(layers, ys, xbits)):
+        rows = sample_rows(lay.n, nrows, i)
+        w = oracle.dequantize("bt3", lay.trits[:, rows], 16, idx=lay.idx[rows], codebook=lay.codebook)
+        check_bf16(y[rows], oracle.gemv_bf16(w, x)[0])
+        if outs16 is not None:
+            assert np.array_equal(outs16[i].view(np.uint16), synth.f32_to_bf16_bits(y))
+
+
+def test_bt3_llama_q_x8(tern):
+    # balanced ternary d = 3 in the one-CTA-per-SM kernel: 8 x 128 row tiles
+    layers = [synth.bt3_layer(4096, 4096, seed=5900 + i) for i in range(8)]
+    (ys,), xbits = run_grouped(tern, layers, tern.ACT_BF16)
+    (y16,), _ = run_grouped(tern, layers, tern.ACT_BF16, out=tern.OUT_BF16)
+    bt3_check(layers, ys, xbits, 256, y16)
+
+
+def test_bt3_down_long_k_x5(tern):
+    # K = 14336: the largest activation image per problem
+    layers = [synth.bt3_layer(4096, 14336, seed=5950 + i) for i in range(5)]
+    (ys,), xbits = run_grouped(tern, layers, tern.ACT_BF16)
+    bt3_check(layers, ys, xbits, 128)
+
+
+def test_bt3_ragged_mix(tern):
+    # rows not multiples of 32, K not a multiple of 80 (padded last column),
+    # problems much smaller than a CTA's share next to large ones
+    ns = [70, 20000, 33, 1500, 9000]
+    layers = [synth.bt3_layer(n, 1040, seed=6000 + i) for i, n in enumerate(ns)]
+    (ys,), xbits = run_grouped(tern, layers, tern.ACT_BF16)
+    bt3_check(layers, ys, xbits, 1024)
+    runs, _ = run_grouped(tern, layers, tern.ACT_BF16, reps=2)
+    for a, b in zip(runs[0], runs[1]):
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
