@@ -56,7 +56,9 @@ def parse():
                          "Llama-3.1-8B shapes; tq2p: the batched sweep (per-shape tables only)")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--profile", default=None,
-                    help="run only one case eagerly for a profiler: step | <shape>_indep | <shape>_chain")
+                    help="run only one case eagerly for a profiler: step | <shape>_indep | <shape>_chain "
+                         "(headline workload); with --config tq3p|bt3|tq2p|single: <shape>:<m> (the copies "
+                         "launched one after another) or <shape>:1:indep (one grouped launch)")
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--ceiling", action="store_true",
                     help="measure the read ceiling (tern_stream_read) for a few access shapes and exit")
@@ -346,7 +348,7 @@ def run_ours(args, rank, world):
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": committed_traffic(step_bytes / len(step_launches)),
+                     "traffic": committed_traffic(),
                      "kernel": "gemv2w_kernel<bf16->int8 in-kernel, 1 plane, per-tensor scale> (one CTA per SM)",
                      "peak_kind": peak_kind,
                      "achieved_basis": "algorithmic bytes of the step's GEMV launches (weights, bf16 activations, "
@@ -424,11 +426,12 @@ def run_config(args):
                     tern.gemm_batched(d, pkc, m, act, xin, sin, tern.OUT_F32, y, ws, stream)
 
             indep = None
-            if m == 1:   # grouped launches of up to 32 independent GEMVs
-                indep = [tern.Grouped([d] * len(packs[i:i + 32]), packs[i:i + 32], act,
-                                      [xin.view(-1)] * len(packs[i:i + 32]),
-                                      None if sin is None else [sin] * len(packs[i:i + 32]), tern.OUT_F32,
-                                      [y.view(-1) for y in ys[i:i + 32]]) for i in range(0, copies, 32)]
+            if m == 1:   # grouped launches of up to 256 independent GEMVs
+                G = 256
+                indep = [tern.Grouped([d] * len(packs[i:i + G]), packs[i:i + G], act,
+                                      [xin.view(-1)] * len(packs[i:i + G]),
+                                      None if sin is None else [sin] * len(packs[i:i + G]), tern.OUT_F32,
+                                      [y.view(-1) for y in ys[i:i + G]]) for i in range(0, copies, G)]
 
             def timed(fn):
                 with torch.cuda.stream(stream):
@@ -448,6 +451,17 @@ def run_config(args):
                     torch.cuda.synchronize()
                 return e0.elapsed_time(e1) / reps
 
+            if args.profile:
+                case = f"{lay.name}:{m}"
+                if args.profile in (case, case + ":indep"):
+                    fn = (lambda: [g.launch(stream) for g in indep]) if args.profile.endswith(":indep") else chain
+                    with torch.cuda.stream(stream):
+                        for _ in range(args.reps):
+                            fn()
+                    torch.cuda.synchronize()
+                    assert tern.device_error(stream) == tern.OK
+                    return None
+                continue
             ms_c = timed(chain)
             row = dict(shape=f"{lay.name} {lay.n}x{lay.k}", m=m, bytes_per_gemv=algo, copies=copies,
                        chain_us_per_gemv=round(ms_c * 1e3 / copies, 3),
@@ -503,18 +517,26 @@ def run_ceiling(args):
             "best": max(r["gbs"] for r in rows)}
 
 
-def committed_traffic(algo_bytes_per_launch):
-    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
-    p = os.path.join(ROOT, "profiles", "gemv2_traffic.json")
+def committed_traffic():
+    """DRAM bytes (read + written) per launch of the step from a committed ncu summary, if the summary
+    was taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "gemv2w_bitnet2b_step_traffic.txt")
     if not os.path.exists(p):
         return None
+    vals = {}
     with open(p) as f:
-        d = json.load(f)
-    src = os.path.join(ROOT, "packed_ternary_weight_b200", "csrc", "tern_gemv2.cu")
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                key, val = line.split(":", 1)
+                vals[key.strip()] = val.strip()
+    src = os.path.join(ROOT, "packed_ternary_weight_b200", "csrc", "tern_gemv2w.cu")
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if d.get("source_sha256_16") != h:
+    if vals.get("kernel_source_sha256_16") != h:
         return None
-    return d.get("dram_bytes_per_launch_scaled")
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
 
 
 # ---------------------------------------------------------- CPU baseline
