@@ -29,9 +29,10 @@ Format (all little-endian):
   digits of triple i, byte 0 first, are the trits t0, t1, t2 (weights 1, 3, 9)
   of k = 80c + i, then of k = 80c + 16 + i, ..., then of k = 80c + 64 + i
   (weight j of the triple, j = 0..4, is k = 80c + 16j + i). The last 96 bytes hold the
-  scale indices of the column's five groups of 16: byte d (0..2) of row r, at
-  1536 + 32*d + r, holds base-3 digit d of the index of group 5c + j as its
-  digit j. Padding trits are 0 (digit 1), padding indices 0.
+  scale indices of the column's five groups of 16 as one more triple per row:
+  byte b (0..2) of row r at 1536 + 32*b + r, five base-3 digits each; digit
+  3j + q of the triple (byte 0 first) is base-3 digit q of the index of group
+  5c + j. Padding trits are 0 (digit 1), padding indices 0.
 """
 from __future__ import annotations
 
@@ -112,9 +113,10 @@ def _unpack_bt3(buf: np.ndarray, h: dict):
     t = (dig - 1).astype(np.int8)
     # k = 80c + 16j + i
     t = t.transpose(5, 0, 2, 1, 4, 3).reshape(3, T * 32, C * 80)
-    ib = col[:, :, 1536:].reshape(T, C, 3, 32)                   # [T][c][d][r]
-    idig = _base3_digits(ib)                                      # [T][c][d][r][j]
-    idx = idig[:, :, 0] + 3 * idig[:, :, 1] + 9 * idig[:, :, 2]   # [T][c][r][j]
+    ib = col[:, :, 1536:].reshape(T, C, 3, 32)                   # [T][c][b][r]
+    idig = _base3_digits(ib)                                      # [T][c][b][r][q]
+    idig = idig.transpose(0, 1, 3, 2, 4).reshape(T, C, 32, 5, 3)  # [T][c][r][j][digit]
+    idx = idig[..., 0] + 3 * idig[..., 1] + 9 * idig[..., 2]      # [T][c][r][j]
     idx = idx.transpose(0, 2, 1, 3).reshape(T * 32, C * 5)        # group = 5c + j
     return t[:, :n, :k].copy(), idx[:n, : k // 16].astype(np.uint8)
 

@@ -162,13 +162,15 @@ bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, in
   if (xs > kMaxSlotsW) return false;
   p.xslots = xs;
   const int colb = bt3 ? kBt3ColBytes : L.planes * kPlaneColBytes;
-  p.stage_cols = std::max(p.gcols, (6144 / colb) / p.gcols * p.gcols);
-  // (warps, stages): sixteen warps with two 6 KB stages each measured best on
-  // the BitNet-2B layer set; fewer when the activation images need the room
-  static const int kShapes[][2] = {{16, 2}, {12, 2}, {8, 3}, {8, 2}, {4, 3}, {4, 2}};
+  // (warps, stages, stage bytes): sixteen warps with two 6 KB stages each
+  // measured best on the BitNet-2B layer set; when the activation images need
+  // the room (long K), smaller stages keep sixteen warps before fewer warps
+  static const int kShapes[][3] = {{16, 2, 6144}, {16, 2, 4096}, {16, 2, 3072}, {12, 2, 4096},
+                                   {8, 3, 4096},  {8, 2, 4096},  {4, 3, 4096},  {4, 2, 4096}};
   for (const auto& sh : kShapes) {
     p.nw = sh[0];
     p.nstage = sh[1];
+    p.stage_cols = std::max(p.gcols, (sh[2] / colb) / p.gcols * p.gcols);
     // the kernel adds its shared copy of the parameter block's head and of
     // its problems
     if (gemv2w_smem_bytes(p, xmode) + offsetof(Gemv2wParams, prob) + sizeof(Gemv2wProblem) * kMaxSlotsW <=

@@ -56,8 +56,8 @@ struct Plan2w {
 //   xs    [xslots] activation slots:
 //           integer paths: int8 x [kx] | int32 sums (BitNet: prefix sums per column [cols+1];
 //                          TQ: per group [groups]) | fp32 token scale
-//           bf16 path:     high, middle, low bytes [kx] each | int64 group sums | fp32 2^(E-22) per group
-//                          (| fp32 codebook [27] for balanced ternary d = 3)
+//           bf16 path:     high, middle, low bytes [kx] each | per group {sum h, sum m, sum l,
+//                          2^(E-22)} (16 bytes) (| fp32 codebook [27] for balanced ternary d = 3)
 //   red   [nw][2][32] partial row sums of shared tiles (8 bytes each)
 //   cnt   [nw] arrival counters of shared tiles
 //   misc  per-warp maxima [xslots][nw] for the in-kernel quantisation
@@ -73,10 +73,9 @@ __host__ __device__ inline Plan2w plan2w(const Gemv2wParams& p, int xmode) {
     // the image covers whole columns: d = 3 pads K to a multiple of 80, so it
     // holds kx / 16 groups (TQ: K is a multiple of 64, kx = K)
     const size_t gimg = p.bt3 ? (size_t)s.kx / 16 : (size_t)p.groups;
-    s.sum_off = 3 * (size_t)s.kx;
-    s.sx_off = s.sum_off + 8 * gimg;  // here: 2^(E-22) per group
-    // d = 3: the 27-entry codebook follows the per-group multipliers
-    s.slot_bytes = align_up(s.sx_off + 4 * gimg + (p.bt3 ? 27 * 4 : 0), 128);
+    s.sum_off = 3 * (size_t)s.kx;       // 16-byte group records {sum h, sum m, sum l, 2^(E-22)}
+    s.sx_off = s.sum_off + 16 * gimg;   // d = 3: the 27-entry codebook
+    s.slot_bytes = align_up(s.sx_off + (p.bt3 ? 27 * 4 : 0), 128);
   } else {
     s.sum_off = s.kx;
     s.sx_off = align_up(s.sum_off + 4 * (size_t)(tq ? p.groups : p.cols + 1), 16);
@@ -406,13 +405,12 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
       if constexpr (kB3) {
         // the codebook from the packed header (the trit stream starts right after it)
         if (threadIdx.x < 27)
-          reinterpret_cast<float*>(sl + sp.sx_off + (size_t)sp.kx / 4)[threadIdx.x] =
+          reinterpret_cast<float*>(sl + sp.sx_off)[threadIdx.x] =
               reinterpret_cast<const float*>(sprob[s].trit - kHeaderBytes + kCodebookOffset)[threadIdx.x];
       }
-      gemv_common::stage_x_bf16_image(static_cast<const uint16_t*>(sprob[s].x), p.k, p.group, 0, sp.kx,
-                                      reinterpret_cast<int8_t*>(sl), sl + sp.kx, sl + 2 * (size_t)sp.kx,
-                                      reinterpret_cast<long long*>(sl + sp.sum_off),
-                                      reinterpret_cast<float*>(sl + sp.sx_off));
+      gemv_common::stage_x_bf16_chains(static_cast<const uint16_t*>(sprob[s].x), p.k, p.group, 0, sp.kx,
+                                       reinterpret_cast<int8_t*>(sl), sl + sp.kx, sl + 2 * (size_t)sp.kx,
+                                       reinterpret_cast<int4*>(sl + sp.sum_off));
     }
     __syncthreads();
   }
@@ -533,8 +531,8 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
         reinterpret_cast<const uint16_t*>(ring + (size_t)slot * sp.stage_bytes + (size_t)sc * P * kPlaneColBytes);
     const int ga_stage = kTQ ? ccc * kColK2 / p.group : 0;
     const int* gsum = reinterpret_cast<const int*>(sl + sp.sum_off);
-    const long long* gsum64 = reinterpret_cast<const long long*>(sl + sp.sum_off);
-    const float* gmul = reinterpret_cast<const float*>(sl + sp.sx_off);
+    const int4* grec = reinterpret_cast<const int4*>(sl + sp.sum_off);  // bf16: per-group chain sums
+    const float* cbk = reinterpret_cast<const float*>(sl + sp.sx_off);   // d = 3: codebook
     // one 16-k word (index WI of the column) of every plane
     // xw: the column's four activation words (integer paths, loaded ahead)
     auto word_step = [&](auto wi_c, const uint4* wv, const uint4* xw, int cc) {
@@ -586,9 +584,11 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
             if constexpr (!kBf) {
               acc64 += fold_fp16_exact(h, gsum[gl] - fold_int(acc[q]));
             } else {
-              const int H = fold_int(acc[q]), Mi = fold_u(accm[q]), L = fold_u(accl[q]);
-              const long long S = gsum64[gl] - ((long long)H * 65536 + (long long)Mi * 256 + L);
-              yacc = fmaf(__half2float(__ushort_as_half(h)) * gmul[gl], __ll2float_rn(S), yacc);
+              // sum t q = sum q - sum F q, chain by chain (small integers)
+              const int4 r = grec[gl];
+              const float S = gemv_common::chains_to_float(r.x - fold_int(acc[q]), r.y - fold_u(accm[q]),
+                                                           r.z - fold_u(accl[q]));
+              yacc = fmaf(__half2float(__ushort_as_half(h)) * __int_as_float(r.w), S, yacc);
             }
 #pragma unroll
             for (int f = 0; f < 4; ++f) acc[q][f] = accm[q][f] = accl[q][f] = 0;
@@ -617,11 +617,11 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
     // digit chunks), five groups of 16 folded with their codebook scales
     auto column3 = [&](const uint4* wv, int cc) {
       const uint32_t cbase = st32 - (uint32_t)(lane * 16) + (uint32_t)((cc - ccc) * kColB);
-      uint32_t ia[5], ib[5];
-      gemv_common::digits5(lds_u8w(cbase + 3 * kPlaneColBytes + lane) |
-                               (lds_u8w(cbase + 3 * kPlaneColBytes + 32 + lane) << 16),
-                           ia);
-      gemv_common::digits5(lds_u8w(cbase + 3 * kPlaneColBytes + 64 + lane), ib);
+      // the five groups' codebook indices: one more triple, same order as the trits
+      uint32_t ix[5];
+      gemv_common::triple_levels(lds_u8w(cbase + 3 * kPlaneColBytes + lane),
+                                 lds_u8w(cbase + 3 * kPlaneColBytes + 32 + lane),
+                                 lds_u8w(cbase + 3 * kPlaneColBytes + 64 + lane), ix);
       uint32_t U[4][5];
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
@@ -634,7 +634,6 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
 #pragma unroll
         for (int j = 0; j < 5; ++j) U[w][j] = ue[j] | (uo[j] << 8);
       }
-      const float* cbk = gmul + sp.kx / 16;  // the codebook follows the kx / 16 group multipliers
 #pragma unroll
       for (int j = 0; j < 5; ++j) {
         const uint32_t xo = (uint32_t)(cc * kColK3 + 16 * j);
@@ -655,9 +654,11 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
         L = dp4a_uu(U[2][j], lv.z, L);
         L = dp4a_uu(U[3][j], lv.w, L);
         const int g = cc * kBt3Groups + j;
-        const long long S = ((long long)H * 65536 + (long long)M * 256 + L) - 13ll * gsum64[g];
-        const uint32_t idx = (ia[j] & 0xFFFFu) + 3u * (ia[j] >> 16) + 9u * ib[j];
-        yacc = fmaf(cbk[idx] * gmul[g], __ll2float_rn(S), yacc);
+        // sum (U - 13) q chain by chain: |H'| < 2^15, |256 M' + L'| < 2^24, so
+        // the sum is rounded once, as an exact int64 conversion would be
+        const int4 r = grec[g];
+        const float S = gemv_common::chains_to_float(H - 13 * r.x, (int)M - 13 * r.y, (int)L - 13 * r.z);
+        yacc = fmaf(cbk[ix[j]] * __int_as_float(r.w), S, yacc);
       }
     };
     auto column = [&](const uint4* wv, const uint4* xw, int cc) {

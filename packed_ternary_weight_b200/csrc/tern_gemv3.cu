@@ -8,8 +8,8 @@
 // k = 80c + 16j + i (j = 0..4), weight by weight (u0, u1, u2 of weight j are
 // base-3 digits 3j .. 3j+2 of the triple, five digits per byte, first digit
 // least significant), byte b of every triple in the b-th 16-byte chunk of the
-// row; then three bytes per row holding the base-3 digits of the five groups'
-// codebook indices. Weight j of the 16 triples of a row is group 5c + j.
+// row; then one more triple per row holding the five groups' codebook indices
+// in the same order. Weight j of the 16 triples of a row is group 5c + j.
 //
 // Work split, weight stream, K-splits and persistence follow the 2-bit kernel:
 // one warp per 32-row tile and K-split, per-warp rings of shared-memory stages
@@ -41,7 +41,6 @@ int read_clear_dev_error_gemv3(void* stream, unsigned* out) { return read_clear_
 namespace {
 
 using gemv_common::align_up;
-using gemv_common::digits5;
 using gemv_common::triple_levels;
 
 struct Smem3 {
@@ -207,10 +206,11 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
         for (int cc = 0; cc < ncs; ++cc) {
           const uint32_t col = st32 + (uint32_t)(cc * kBt3ColBytes);
           const uint32_t kx = (uint32_t)((cs + cc - c0) * kColK3);
-          // scale indices of the column's five groups (three bytes of base-3 digits)
-          uint32_t ia[5], ib[5];
-          digits5(lds_u8(col + 3 * kPlaneColBytes + lane) | (lds_u8(col + 3 * kPlaneColBytes + 32 + lane) << 16), ia);
-          digits5(lds_u8(col + 3 * kPlaneColBytes + 64 + lane), ib);
+          // scale indices of the column's five groups: one more triple, same
+          // order as the trits
+          uint32_t ix[5];
+          triple_levels(lds_u8(col + 3 * kPlaneColBytes + lane), lds_u8(col + 3 * kPlaneColBytes + 32 + lane),
+                        lds_u8(col + 3 * kPlaneColBytes + 64 + lane), ix);
           // U = u0 + 3 u1 + 9 u2 in byte lanes, for the 4 words x 5 digit positions
           uint32_t U[4][5];
           const uint4 b0 = lds128<0>(col + lane * 16);
@@ -249,8 +249,7 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
             L = dp4a_uu(U[3][j], lv.w, L);
             const int g = (int)(kx >> 4) + j;  // group within the split
             const long long S = ((long long)H * 65536 + (long long)M * 256 + L) - 13ll * gsum[g];
-            const uint32_t idx = (ia[j] & 0xFFFFu) + 3u * (ia[j] >> 16) + 9u * ib[j];
-            yacc = fmaf(lds_f32(cb32 + 4u * idx) * gmul[g], __ll2float_rn(S), yacc);
+            yacc = fmaf(lds_f32(cb32 + 4u * ix[j]) * gmul[g], __ll2float_rn(S), yacc);
           }
         }
         fence_proxy_async_smem();

@@ -59,6 +59,56 @@ __device__ inline void stage_x_bf16_image(const uint16_t* x, int K, int g, int k
   }
 }
 
+// As stage_x_bf16_image, but instead of the exact sum of q per group it writes
+// one 16-byte record per group: the sums of the high (signed), middle and low
+// byte chains, {sum h, sum m, sum l, bits of 2^(E-22)}, so that a group's
+// sum of w * q can be formed as 65536 * (H - c sum h) + 256 * (M - c sum m) +
+// (L - c sum l) from small integers (q = 65536 h + 256 m + l exactly).
+__device__ inline void stage_x_bf16_chains(const uint16_t* x, int K, int g, int k0, int kr, int8_t* xh, uint8_t* xm,
+                                           uint8_t* xl, int4* rec) {
+  const int gr = kr / g;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int grp = warp; grp < gr; grp += nw) {
+    const int kb = grp * g;
+    float amax = 0.f;
+    for (int kk = kb + lane; kk < kb + g; kk += 32) {
+      const int k = k0 + kk;
+      const float v = k < K ? __uint_as_float((uint32_t)x[k] << 16) : 0.f;
+      amax = fmaxf(amax, fabsf(v));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const int e = amax > 0.f ? ilogbf(amax) : 0;
+    const int sh = 22 - e;
+    const float up1 = ldexpf(1.0f, sh > 100 ? 100 : sh), up2 = ldexpf(1.0f, sh > 100 ? sh - 100 : 0);
+    int sh_ = 0, sm = 0, sl = 0;
+    for (int kk = kb + lane; kk < kb + g; kk += 32) {
+      const int k = k0 + kk;
+      const float v = k < K ? __uint_as_float((uint32_t)x[k] << 16) : 0.f;
+      const int q = __float2int_rn(__fmul_rn(__fmul_rn(v, up1), up2));  // |q| < 2^23
+      const int h = q >> 16, m = (q >> 8) & 0xFF, l = q & 0xFF;
+      sh_ += h;
+      sm += m;
+      sl += l;
+      xh[kk] = (int8_t)h;
+      xm[kk] = (uint8_t)m;
+      xl[kk] = (uint8_t)l;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      sh_ += __shfl_xor_sync(0xffffffffu, sh_, o);
+      sm += __shfl_xor_sync(0xffffffffu, sm, o);
+      sl += __shfl_xor_sync(0xffffffffu, sl, o);
+    }
+    if (lane == 0) rec[grp] = make_int4(sh_, sm, sl, __float_as_int(amax > 0.f ? ldexpf(1.0f, e - 22) : 0.f));
+  }
+}
+
+// 65536 a + 256 b + c as fp32, rounded once when |256 b + c| < 2^24 and |a| < 2^24.
+__device__ __forceinline__ float chains_to_float(int a, int b, int c) {
+  return fmaf(__int2float_rn(a), 65536.0f, fmaf(__int2float_rn(b), 256.0f, __int2float_rn(c)));
+}
+
 // Five base-3 digits of the two values (each <= 242) held in the 16-bit lanes of v.
 __device__ __forceinline__ void digits5(uint32_t v, uint32_t (&d)[5]) {
 #pragma unroll

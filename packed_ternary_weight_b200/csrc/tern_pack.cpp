@@ -24,8 +24,9 @@
 // k = 80c + 16j + i (j = 0..4, one weight of each of the column's five groups
 // of 16), weight by weight (t0, t1, t2 of weight j are trits 3j, 3j+1, 3j+2 of
 // the triple, trits 5b..5b+4 in byte b); byte b of triple i sits at
-// b * 512 + 16 r + i. Then three bytes per row holding the base-3 digits of the
-// five groups' codebook indices. Keeping the three trits of a weight together
+// b * 512 + 16 r + i. Then one more triple per row (bytes at 1536 + 32 b + r)
+// holding the five groups' codebook indices in the same order (digit q of
+// index j is trit 3j + q). Keeping the three trits of a weight together
 // lets the decoder read a weight's level U = u0 + 3 u1 + 9 u2 with a few
 // divisions by 3, 9 and 27 instead of extracting every digit.
 #include <cmath>
@@ -202,18 +203,24 @@ static tern_status pack_bt3(const Layout& L, const int8_t* trits, const uint8_t*
           }
         }
       }
-      for (int dgt = 0; dgt < 3; ++dgt)
-        for (int r = 0; r < kTileRows; ++r) {
-          const int n = T * kTileRows + r;
-          unsigned v = 0, pw = 1;
-          for (int j = 0; j < 5; ++j, pw *= 3) {
-            const int g = c * kBt3Groups + j;
-            unsigned id = (n < N && g < G) ? idx[(size_t)n * G + g] : 0u;
-            for (int q = 0; q < dgt; ++q) id /= 3;
-            v += (id % 3) * pw;
-          }
-          col[3 * kPlaneColBytes + dgt * kTileRows + r] = (uint8_t)v;
+      // the five groups' codebook indices (3 base-3 digits each) as one more
+      // triple per row, index by index: digit q of index j is trit 3j + q
+      for (int r = 0; r < kTileRows; ++r) {
+        const int n = T * kTileRows + r;
+        unsigned dig[15];
+        for (int j = 0; j < 5; ++j) {
+          const int g = c * kBt3Groups + j;
+          const unsigned id = (n < N && g < G) ? idx[(size_t)n * G + g] : 0u;
+          dig[3 * j] = id % 3;
+          dig[3 * j + 1] = (id / 3) % 3;
+          dig[3 * j + 2] = id / 9;
         }
+        for (int b = 0; b < 3; ++b) {
+          unsigned v = 0, pw = 1;
+          for (int q = 0; q < 5; ++q, pw *= 3) v += dig[5 * b + q] * pw;
+          col[3 * kPlaneColBytes + b * kTileRows + r] = (uint8_t)v;
+        }
+      }
     }
   }
   return TERN_OK;

@@ -107,8 +107,9 @@ def test_bt3_bytes_by_hand():
     # weight, five digits per byte: triple 3 starts with the digits 2, 1, 1 of
     # k = 3, so its byte 0 is 2 + 3 + 9 + 27 + 81 = 122 and every other byte is
     # 1 + 3 + 9 + 27 + 81 = 121.
-    # The group's index 14 = 2 + 1*3 + 1*9: index byte d holds digit d of it as
-    # digit 0 and 0 (padding groups) elsewhere -> 2, 1, 1.
+    # The group's index 14 = 2 + 1*3 + 1*9: the index triple holds its digits
+    # 2, 1, 1 first and 0 for the padding groups: byte 0 = 2 + 1*3 + 1*9 = 14,
+    # bytes 1 and 2 = 0.
     t = np.zeros((3, 1, 16), np.int8)
     t[0, 0, 3] = 1
     idx = np.array([[14]], np.uint8)
@@ -119,7 +120,7 @@ def test_bt3_bytes_by_hand():
     col = buf[256:]
     assert col[3] == 122 and col[0] == 121 and col[15] == 121
     assert col[512] == 121 and col[1024 + 7] == 121
-    assert col[1536] == 2 and col[1536 + 32] == 1 and col[1536 + 64] == 1
+    assert col[1536] == 14 and col[1536 + 32] == 0 and col[1536 + 64] == 0
     assert np.array_equal(buf[128:128 + 108].view("<f4"), cb)
     u = oracle.unpack(buf)
     assert np.array_equal(u["trits"], t) and u["idx"].tolist() == [[14]]
@@ -144,6 +145,9 @@ def test_bt3_triple_order_by_hand():
     col = buf[256:]
     assert (col[0], col[512], col[1024]) == (118, 122, 121)
     assert col[1] == 121 and col[512 + 1] == 121 and col[1024 + 15] == 121
+    # index triple: index 0 (digits 0 0 0), index 26 (digits 2 2 2), padding 0:
+    # byte 0 = digits 0 0 0 2 2 -> 2*27 + 2*81 = 216; byte 1 = digits 2 0 0 0 0 -> 2
+    assert (col[1536], col[1536 + 32], col[1536 + 64]) == (216, 2, 0)
     u = oracle.unpack(buf)
     assert np.array_equal(u["trits"], t) and u["idx"].tolist() == [[0, 26]]
 
