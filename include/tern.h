@@ -115,13 +115,18 @@ tern_status tern_pack(const tern_desc* desc, const int8_t* trits, const uint16_t
                       size_t* out_used);
 
 /*
- * Workspace needed by tern_gemv / tern_gemm_batched for `m` tokens (0 for
- * most layers: K-splits normally reduce inside a thread-block cluster; only a
- * very long K needs more splits than a cluster holds and a workspace).
- * The workspace holds per-block arrival counters and split partial sums. It
- * must be zero-filled before its first use; every call resets the counters
- * to zero, so the workspace can be reused by later calls without clearing.
- * Calls that may run at the same time need separate workspaces.
+ * Workspace needed by tern_gemv / tern_gemm_batched for `m` tokens.
+ *   m < 16: 0 for most layers (K-splits normally reduce inside a thread-block
+ *     cluster; only a very long K needs more splits than a cluster holds).
+ *   m >= 16 (2-bit formats, TERN_ACT_INT8 or TERN_ACT_BF16_Q8): the tensor-
+ *     core path needs arrival counters and exact int64 partial sums for the
+ *     row tiles that several CTAs share (sized for 256 tokens), the
+ *     activations in MMA order and, for bf16 input, their int8 quantisation.
+ * The workspace must be 256-byte aligned and zero-filled before its first
+ * use; every call leaves its counters and partial sums at zero again, so the
+ * workspace can be reused by later calls (with any m up to the m it was sized
+ * for) without clearing. Calls that may run at the same time need separate
+ * workspaces.
  */
 tern_status tern_workspace_size(const tern_desc* desc, int32_t m, size_t* bytes);
 
@@ -153,6 +158,12 @@ tern_status tern_gemv(const tern_desc* desc, const void* d_packed, tern_act act,
  * Y = X W^T for m tokens (m >= 1), the weights read once for all tokens.
  *   d_x [m][K] (int8 or bf16 bits), d_xscale float [m] for TERN_ACT_INT8,
  *   d_y [m][N]. For TERN_ACT_INT8 the result is bit-identical to the oracle.
+ * For m >= 16 with the 2-bit formats and int8 (or in-kernel quantised bf16)
+ * activations the product runs on the tensor cores (tcgen05 int8 MMA, up to
+ * 256 tokens per launch); the fp16 group scales are split into small integer
+ * digits folded into the int8 weight operand, so the result stays exact.
+ * That path needs the workspace tern_workspace_size(desc, m) reports
+ * (TERN_ENOSPACE without it).
  */
 tern_status tern_gemm_batched(const tern_desc* desc, const void* d_packed, int32_t m, tern_act act,
                               const void* d_x, const float* d_xscale, tern_out out, void* d_y,

@@ -199,10 +199,11 @@ PlanTc plan_tc(const Layout& L, int mb, int xmode, int sms) {
   PlanTc t{};
   const bool tq = L.fmt == TERN_FMT_TQ;
   if (L.fmt == TERN_FMT_BT3 || (xmode != kXInt8 && xmode != kXBf16Q8) || mb < 1 || mb > kTcMaxTokens) return t;
-  // every digit accumulator stays below 2^31: planes * 127 * 127 * K; the
-  // kernel's positions (128-row tiles x token passes x columns) fit in 31 bits
-  if ((long long)L.planes * 127 * 127 * L.k >= (1ll << 31)) return t;
-  if ((long long)(L.row_tiles + 3) / 4 * kTcMaxDigits * L.cols >= (1ll << 31)) return t;
+  // every digit accumulator stays below 2^31: 127 * 127 * K (the planes share
+  // one int8 operand); the kernel's positions (128-row tiles x token passes x
+  // columns) fit in 31 bits
+  if ((long long)127 * 127 * L.k >= (1ll << 31)) return t;
+  if ((long long)(L.row_tiles + 3) / 4 * kTcMaxMerged * L.cols >= (1ll << 31)) return t;
   GemmTcParams& p = t.p;
   p.tq = tq;
   p.n = L.n;
@@ -216,9 +217,9 @@ PlanTc plan_tc(const Layout& L, int mb, int xmode, int sms) {
   p.m = mb;
   p.m16 = (mb + 15) & ~15;
   int mp = 0, xcap = 0, pcap = 0;
-  for (int d = 1; d <= (tq ? kTcMaxDigits : 1); ++d) {
+  for (int d7 = 1; d7 <= (tq ? kTcMaxDigits : 1); ++d7) {
     int ps, tp;
-    tc_passes(d, p.m16, &ps, &tp);
+    tc_passes(tc_merged_digits(L.planes, d7), p.m16, &ps, &tp);
     mp = std::max(mp, ps * tp);
     xcap = std::max(xcap, tp);
     pcap = std::max(pcap, ps);
@@ -235,7 +236,7 @@ PlanTc plan_tc(const Layout& L, int mb, int xmode, int sms) {
     return o;
   };
   int pmax = 0, tdummy = 0;
-  tc_passes(kTcMaxDigits, kTcMaxTokens, &pmax, &tdummy);
+  tc_passes(kTcMaxMerged, kTcMaxTokens, &pmax, &tdummy);
   t.cnt_off = take((size_t)p.tiles * pmax * 4);
   t.part_off = take((size_t)kTcMaxTokens * p.n_pad * 8);
   t.xp_off = take((size_t)t.kchunks * mp * 16);
@@ -246,7 +247,7 @@ PlanTc plan_tc(const Layout& L, int mb, int xmode, int sms) {
   t.total = off;
   // A ring of twelve 8 KB tiles (two groups at the largest digit count); as
   // many input stages in flight as the rest of shared memory holds, up to 12
-  p.nslot = 2 * kTcMaxDigits;
+  p.nslot = 2 * kTcMaxMerged;
   p.nstage = 12;
   while (p.nstage > 2 && gemm_tc_smem_bytes(p) > 227 * 1024) --p.nstage;
   t.ok = gemm_tc_smem_bytes(p) <= 227 * 1024;

@@ -11,20 +11,25 @@
 // one integer per row and token; applying a different fp16 scale to every 32
 // columns would cost several CUDA-core instructions per accumulator element
 // and K step. Instead the scale goes into the A operand: u = |s| / 2^-24 is an
-// integer below 2^40, written in D base-128 digits u_d (D from the packed
-// header: the largest scale's digit count). For digit d the A tile holds
-// sign(s) * t * u_d, which fits int8 because t is -1, 0 or +1 and u_d <= 127;
-// one tensor-memory int32 accumulator per digit then sums every group and
-// plane of the K range, and the exact result is sum_d 128^d * acc_d, formed in
-// int64 once per output. (|acc_d| <= P * 127 * 127 * K stays below 2^31 for
-// the shapes the host admits.) The tensor cores do D times the algorithmic
-// MACs; the CUDA cores only decode.
+// integer below 2^40, written in D' base-2^b digits u_d with b = 7 for one
+// plane, 6 for two, 5 for three or four (D' = ceil(7 D / b), D the packed
+// header's count of 7-bit digits of the largest scale). The A tile of digit d
+// holds sum_p sign(s_p) * t_p * u_{p,d}: at most P (2^b - 1) <= 127 in
+// magnitude, so the planes merge into one int8 operand. One tensor-memory
+// int32 accumulator per digit then sums every group and plane of the K range,
+// and the exact result is sum_d 2^(b d) * acc_d, formed in int64 once per
+// output (|acc_d| <= 127 * 127 * K < 2^31 for the shapes the host admits).
+// The tensor cores do D' times the algorithmic MACs of one plane; the CUDA
+// cores only decode.
 //
-// Decode. A 2-bit code selects one of three bytes {0, a, -a} of a per-digit
-// lookup word by byte permutation (PRMT), four weights per instruction. The
-// selector nibbles come from masking the packed word, which yields the 16
-// weights of a word in the order 0,8,1,9,...,7,15; the activations are staged
-// in the same order (tc_prep_x), so every dot product sees matching pairs.
+// Decode. A 2-bit code selects one of three bytes {beta, beta + a, beta - a}
+// of a per-(plane, digit) lookup word by byte permutation (PRMT), four weights
+// per instruction; the planes' bias bytes beta add up to 128, so the planes'
+// words add without carries between bytes and one XOR with 0x80 per byte
+// leaves the signed sum (one plane: beta = 0, no XOR). The selector nibbles
+// come from masking the packed word, which yields the 16 weights of a word in
+// the order 0,8,1,9,...,7,15; the activations are staged in the same order
+// (tc_prep_x), so every dot product sees matching pairs.
 //
 // Pipeline (one CTA per SM, persistent). Work = (128-row tile, token pass) x
 // 64-k columns; CTA c takes the contiguous range [W c / G, W (c+1) / G).
@@ -32,9 +37,9 @@
 //              activations into a ring of stages (mbarrier transaction counts);
 //   warp 1     allocates tensor memory; one thread issues tcgen05.mma and
 //              commits completion to mbarriers;
-//   warps 2-17 decode A tiles (the D digit tiles of one plane of one column
-//              form a group of the shared ring; one warp per 32 rows and
-//              16-k chunk), then drain the accumulators: a tile whose whole K range
+//   warps 2-17 decode A tiles (the D' digit tiles of one column form a group
+//              of the shared ring; one warp per 32 rows and 16-k chunk), then
+//              drain the accumulators: a tile whose whole K range
 //              lies in this CTA is written directly; a tile cut between CTAs is
 //              summed exactly in an int64 workspace with atomic adds and
 //              finished by the last CTA to arrive (integer sums, so the order
@@ -148,24 +153,31 @@ __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint3
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
 
-// Per-digit lookup words of one fp16 scale h: byte 1 = sign(s) * u_d (code
-// 01, t = +1), byte 2 = its negation (code 10, t = -1), byte 0 zero (code 00);
-// byte 3 is never selected (code 11 does not occur). u_d * 0x00FF0100 puts u_d
-// in byte 1 and -u_d mod 256 in byte 2; a negative scale swaps the two bytes.
-template <int D>
-__device__ __forceinline__ void scale_luts(uint32_t h, uint32_t (&lut)[D]) {
+// Digit width and per-plane bias of the merged A operand for P planes.
+template <int P>
+constexpr int kDigitBits = P == 1 ? 7 : (P == 2 ? 6 : 5);
+template <int P>
+__device__ __forceinline__ uint32_t plane_bias(int pl) {
+  if constexpr (P == 1) return 0u;
+  if constexpr (P == 2) return 64u;
+  if constexpr (P == 3) return pl == 2 ? 42u : 43u;
+  return 32u;
+}
+
+// u = |s| / 2^-24 of an fp16 scale (below 2^40) and the byte permutation that
+// applies its sign (a negative scale swaps the +t and -t bytes).
+__device__ __forceinline__ uint64_t scale_units(uint32_t h, uint32_t& sel) {
   const uint32_t ex = (h >> 10) & 31u, man = h & 1023u;
-  const uint32_t sel = (h & 0x8000u) ? 0x3120u : 0x3210u;
-  if constexpr (D <= 4) {
-    // the largest scale has at most 4 digits, so every u is below 2^28
-    const uint32_t u = ex ? (1024u | man) << (ex - 1u) : man;
-#pragma unroll
-    for (int d = 0; d < D; ++d) lut[d] = __byte_perm(((u >> (7 * d)) & 127u) * 0x00FF0100u, 0u, sel);
-  } else {
-    const uint64_t u = ex ? (uint64_t)(1024u | man) << (ex - 1u) : (uint64_t)man;
-#pragma unroll
-    for (int d = 0; d < D; ++d) lut[d] = __byte_perm((uint32_t)((u >> (7 * d)) & 127u) * 0x00FF0100u, 0u, sel);
-  }
+  sel = (h & 0x8000u) ? 0x3120u : 0x3210u;
+  return ex ? (uint64_t)(1024u | man) << (ex - 1u) : (uint64_t)man;
+}
+
+// Lookup word of one plane and digit: byte 0 = beta (code 00, t = 0), byte 1 =
+// beta + a (code 01, t = +1), byte 2 = beta - a (code 10, t = -1), a = sign(s)
+// * ud; byte 3 is never selected (code 11 does not occur). ud * 0x00FF0100
+// puts ud in byte 1 and -ud mod 256 in byte 2 (its borrow lands in byte 3).
+__device__ __forceinline__ uint32_t digit_lut(uint32_t ud, uint32_t beta, uint32_t sel) {
+  return __byte_perm(ud * 0x00FF0100u + beta * 0x00010101u, 0u, sel);
 }
 
 // y = fl32(fl32(acc * 2^-24) * s_x) for the group-scaled sum (acc counts 2^-24,
@@ -189,9 +201,9 @@ __device__ __forceinline__ void store_y(const GemmTcParams& p, int t, int n, lon
 
 __device__ __forceinline__ long long to_ll(uint32_t v) { return (long long)(int)v; }
 
-// The three roles of the kernel for P planes and D scale digits.
-// A ring: groups of D tiles (the digits of one plane of one column); a tile is
-// 128 rows x 64 k, 64 bytes per row, 64-byte swizzle.
+// The three roles of the kernel for P planes and D merged scale digits.
+// A ring: groups of D tiles (the digits of one column); a tile is 128 rows x
+// 64 k, 64 bytes per row, 64-byte swizzle.
 template <int P, int D>
 __device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, const TcSmem& L, uint32_t tmem,
                                          volatile uint32_t* misc, int passes, int tpass, int q0, int q1, int W) {
@@ -283,8 +295,7 @@ __device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, c
         const uint32_t xs = smem_u32(smem + L.stages) + (uint32_t)s * L.stage_bytes + L.raw_bytes + L.sc_bytes;
         const uint64_t bd0 = tc::smem_desc(xs, tpass * 16, 128);
         const uint64_t bd1 = tc::smem_desc(xs + 2 * tpass * 16, tpass * 16, 128);
-#pragma unroll
-        for (int pl = 0; pl < P; ++pl) {
+        {
           tc_wait(&afull[j], aph, misc);
           tc::fence_after_sync();
           const uint32_t a0 = slots + (uint32_t)j * kGroupBytes;
@@ -293,7 +304,7 @@ __device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, c
 #pragma unroll
           for (int d = 0; d < D; ++d)
             tc::mma_i8(tmem + (uint32_t)(d * tpass), tc::smem_desc_sw64(a0 + (uint32_t)d * kSlotBytes, 512), bd0, idesc,
-                       first && pl == 0 ? 0u : 1u);
+                       first ? 0u : 1u);
 #pragma unroll
           for (int d = 0; d < D; ++d)
             tc::mma_i8(tmem + (uint32_t)(d * tpass), tc::smem_desc_sw64(a0 + (uint32_t)d * kSlotBytes + 32, 512), bd1,
@@ -351,31 +362,54 @@ __device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, c
         s = 0;
         ph ^= 1u;
       }
+      // the column's word of every plane, its scale and selector nibbles
+      uint32_t lo[P], lo2[P], hi[P], hi2[P], sel[P];
+      uint64_t u[P];
 #pragma unroll
-      for (int pl = 0; pl < P; ++pl, ++gc) {
+      for (int pl = 0; pl < P; ++pl) {
         const uint32_t w = lds32(raw + pl * kPlaneColBytes);
-        uint32_t lut[D];
         if (p.tq) {
-          scale_luts<D>(lds16(scs + (uint32_t)(pl * 64)), lut);
+          u[pl] = scale_units(lds16(scs + (uint32_t)(pl * 64)), sel[pl]);
         } else {
-#pragma unroll
-          for (int d = 0; d < D; ++d) lut[d] = 0x00FF0100u;
+          u[pl] = 1u;
+          sel[pl] = 0x3210u;
         }
-        const uint32_t lo = w & 0x33333333u, hi = (w >> 2) & 0x33333333u;
-        const uint32_t lo2 = lo >> 16, hi2 = hi >> 16;
-        if (gc >= NG) tc_wait(&afree[j], aph ^ 1u, misc);
-        const uint32_t a = slots + (uint32_t)j * kGroupBytes;
+        lo[pl] = w & 0x33333333u;
+        hi[pl] = (w >> 2) & 0x33333333u;
+        lo2[pl] = lo[pl] >> 16;
+        hi2[pl] = hi[pl] >> 16;
+      }
+      if (gc >= NG) tc_wait(&afree[j], aph ^ 1u, misc);
+      const uint32_t a = slots + (uint32_t)j * kGroupBytes;
+      constexpr int kB = kDigitBits<P>;
+      constexpr uint32_t kMask = (1u << kB) - 1u;
 #pragma unroll
-        for (int d = 0; d < D; ++d)
-          sts128(a + (uint32_t)d * kSlotBytes, __byte_perm(lut[d], 0u, lo), __byte_perm(lut[d], 0u, lo2),
-                 __byte_perm(lut[d], 0u, hi), __byte_perm(lut[d], 0u, hi2));
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[j]);
-        if (++j == NG) {
-          j = 0;
-          aph ^= 1u;
+      for (int d = 0; d < D; ++d) {
+        uint32_t o0 = 0, o1 = 0, o2 = 0, o3 = 0;
+#pragma unroll
+        for (int pl = 0; pl < P; ++pl) {
+          const uint32_t ud = (uint32_t)(u[pl] >> (kB * d)) & kMask;
+          const uint32_t lut = digit_lut(ud, plane_bias<P>(pl), sel[pl]);
+          o0 += __byte_perm(lut, 0u, lo[pl]);
+          o1 += __byte_perm(lut, 0u, lo2[pl]);
+          o2 += __byte_perm(lut, 0u, hi[pl]);
+          o3 += __byte_perm(lut, 0u, hi2[pl]);
         }
+        if constexpr (P > 1) {  // remove the bias of 128 per byte
+          o0 ^= 0x80808080u;
+          o1 ^= 0x80808080u;
+          o2 ^= 0x80808080u;
+          o3 ^= 0x80808080u;
+        }
+        sts128(a + (uint32_t)d * kSlotBytes, o0, o1, o2, o3);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[j]);
+      ++gc;
+      if (++j == NG) {
+        j = 0;
+        aph ^= 1u;
       }
       const int ucur = unit;
       if (++col == cols) {
@@ -398,7 +432,7 @@ __device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, c
           uint32_t v[4];
           tc::ld_x4_sync(taddr + (uint32_t)(d * tpass + tb + c4), v);
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) acc[jj] += to_ll(v[jj]) << (7 * d);
+          for (int jj = 0; jj < 4; ++jj) acc[jj] += to_ll(v[jj]) << (kDigitBits<P> * d);
         }
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
@@ -452,9 +486,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L.misc);
   const int warp = threadIdx.x >> 5;
 
-  int D = 1;
-  if (p.tq) D = (int)__ldg(reinterpret_cast<const unsigned*>(p.header + kDigitsOffset));
-  bool bad = D < 1 || D > kTcMaxDigits || (P > 1 && !p.tq) || NA / (D < 1 ? 1 : D) < 1;
+  int D7 = 1;
+  if (p.tq) D7 = (int)__ldg(reinterpret_cast<const unsigned*>(p.header + kDigitsOffset));
+  const int D = tc_merged_digits(P, D7);  // digits of the merged A operand
+  bool bad = D7 < 1 || D7 > kTcMaxDigits || (P > 1 && !p.tq) || NA / (D < 1 ? 1 : D) < 1;
   int passes = 1, tpass = 16;
   tc_passes(bad ? 1 : D, p.m16, &passes, &tpass);
   bad = bad || tpass > p.xcap || passes > p.passes_cap;
@@ -497,7 +532,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     case 3: tc_roles<P, 3>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
     case 4: tc_roles<P, 4>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
     case 5: tc_roles<P, 5>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
-    default: tc_roles<P, 6>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
+    case 6: tc_roles<P, 6>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
+    case 7: tc_roles<P, 7>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
+    case 8: tc_roles<P, 8>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
+    default: tc_roles<P, 9>(p, smem, L, tmem, misc, passes, tpass, q0, q1, W); break;
   }
 
   tc::fence_before_sync();

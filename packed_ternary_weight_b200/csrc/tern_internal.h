@@ -123,7 +123,8 @@ struct Gemv2wParams {
 // sign(s) * t * u_d (int8), so one int32 accumulator per digit sums over all
 // groups and planes and the exact result is sum_d 128^d * acc_d (int64).
 constexpr int kTcRows = 128;       // weight rows per MMA tile (four 32-row tiles)
-constexpr int kTcMaxDigits = 6;    // fp16 magnitudes are below 2^40 units of 2^-24
+constexpr int kTcMaxDigits = 6;    // 7-bit digits: fp16 magnitudes are below 2^40 units of 2^-24
+constexpr int kTcMaxMerged = 9;    // merged digits (5 bits for three or four planes)
 constexpr int kTcMaxTokens = 256;  // tokens per launch (MMA N <= 256)
 
 struct GemmTcParams {
@@ -141,6 +142,13 @@ struct GemmTcParams {
   float tensor_scale;
   int nstage, nslot, grid;
 };
+
+// Digits of the merged A operand for P planes and D 7-bit digits of the
+// largest scale: b = 7 (one plane), 6 (two), 5 (three, four) bits per digit.
+TERN_HD inline int tc_merged_digits(int planes, int d7) {
+  const int b = planes == 1 ? 7 : (planes == 2 ? 6 : 5);
+  return (7 * d7 + b - 1) / b;
+}
 
 // Token passes for D digits: the D accumulators of one pass share the 512
 // tensor-memory columns. Host and device compute the same values.
