@@ -190,7 +190,7 @@ bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, in
 // in MMA order | (bf16 input) int8 activations and their scales.
 struct PlanTc {
   GemmTcParams p;
-  int kchunks;
+  int kchunks, mp;  // 16-k chunks; the largest passes x tokens per pass
   size_t cnt_off, part_off, xp_off, xq_off, sx_off, total;
   bool ok;
 };
@@ -216,16 +216,18 @@ PlanTc plan_tc(const Layout& L, int mb, int xmode, int sms) {
   p.n_pad = p.tiles * kTcRows;
   p.m = mb;
   p.m16 = (mb + 15) & ~15;
-  int mp = 0, xcap = 0, pcap = 0;
+  // every digit count the header may hold must have a shared-memory plan
+  int mp = 0, pcap = 0;
   for (int d7 = 1; d7 <= (tq ? kTcMaxDigits : 1); ++d7) {
     int ps, tp;
-    tc_passes(tc_merged_digits(L.planes, d7), p.m16, &ps, &tp);
+    const int dm = tc_merged_digits(L.planes, d7);
+    tc_passes(dm, p.m16, &ps, &tp);
+    TcLayout lay;
+    if (!tc_layout(L.planes, tq, p.group, dm, tp, &lay)) return t;
     mp = std::max(mp, ps * tp);
-    xcap = std::max(xcap, tp);
     pcap = std::max(pcap, ps);
   }
-  p.mp = mp;
-  p.xcap = xcap;
+  t.mp = mp;
   p.passes_cap = pcap;
   p.grid = (int)std::min<long long>(sms, (long long)p.tiles * p.cols);
   t.kchunks = L.cols * 4;
@@ -245,12 +247,7 @@ PlanTc plan_tc(const Layout& L, int mb, int xmode, int sms) {
     t.sx_off = take((size_t)mb * 4);
   }
   t.total = off;
-  // A ring of twelve 8 KB tiles (two groups at the largest digit count); as
-  // many input stages in flight as the rest of shared memory holds, up to 12
-  p.nslot = 2 * kTcMaxMerged;
-  p.nstage = 12;
-  while (p.nstage > 2 && gemm_tc_smem_bytes(p) > 227 * 1024) --p.nstage;
-  t.ok = gemm_tc_smem_bytes(p) <= 227 * 1024;
+  t.ok = true;
   return t;
 }
 
@@ -329,10 +326,11 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
                               const_cast<float*>(sx), stream) != 0)
             return TERN_ECUDA;
         }
-        if (launch_tc_prep_x(xq, mc, L.k, pc.kchunks, p.mp, ws + pc.xp_off, stream) != 0) return TERN_ECUDA;
         p.trit = base + L.trit_offset;
         p.scale = p.tq ? reinterpret_cast<const uint16_t*>(base + L.scale_offset) : nullptr;
         p.header = base;
+        if (launch_tc_prep_x(xq, mc, L.k, pc.kchunks, pc.kchunks * pc.mp, p, ws + pc.xp_off, stream) != 0)
+          return TERN_ECUDA;
         p.xp = ws + pc.xp_off;
         p.xscale = sx;
         p.y = static_cast<uint8_t*>(d_y) + (size_t)t0 * L.n * out_elem;

@@ -33,11 +33,17 @@
 //
 // Pipeline (one CTA per SM, persistent). Work = (128-row tile, token pass) x
 // 64-k columns; CTA c takes the contiguous range [W c / G, W (c+1) / G).
-//   warp 0     bulk async copies of each column's packed trits, scales and
-//              activations into a ring of stages (mbarrier transaction counts);
-//   warp 1     allocates tensor memory; one thread issues tcgen05.mma and
-//              commits completion to mbarriers;
-//   warps 2-17 decode A tiles (the D' digit tiles of one column form a group
+//   warp 0     bulk async copies into a ring of stages (mbarrier transaction
+//              counts); a stage holds up to C consecutive columns of the four
+//              row tiles' trits, their scale blocks and the activations, and
+//              is fetched by ONE copy instruction with a lane per stream
+//              (a bulk copy holds its warp for some hundreds of cycles
+//              whatever its size, so fewer and larger copies);
+//   warps 1-2  one thread each issues tcgen05.mma for half of the digit
+//              accumulators and commits completion to mbarriers (two issuing
+//              warps keep the tensor cores busier than one at small N);
+//              warp 1 also owns the tensor-memory allocation;
+//   warps 3-18 decode A tiles (the D' digit tiles of one column form a group
 //              of the shared ring; one warp per 32 rows and 16-k chunk), then
 //              drain the accumulators: a tile whose whole K range
 //              lies in this CTA is written directly; a tile cut between CTAs is
@@ -58,35 +64,11 @@ int read_clear_dev_error_gemm_tc(void* stream, unsigned* out) { return read_clea
 namespace {
 
 constexpr int kDecWarps = 16;
-constexpr int kThreads = 32 * (2 + kDecWarps);
-constexpr int kChunkStride = kTcRows * kChunkBytes;  // 2048: one 16-k chunk of a 128-row A tile
-constexpr int kSlotBytes = 4 * kChunkStride;         // one A tile: 128 rows x 64 k
+constexpr int kMmaWarps = 2;
+constexpr int kDec0 = 1 + kMmaWarps;  // first decoder warp
+constexpr int kThreads = 32 * (kDec0 + kDecWarps);
+constexpr int kSlotBytes = kTcSlotBytes;  // one A tile: 128 rows x 64 k
 constexpr int kTmemCols = 512;
-
-__host__ __device__ inline uint32_t up(uint32_t v, uint32_t a) { return (v + a - 1) / a * a; }
-
-struct TcSmem {
-  uint32_t bars, misc, stages, slots, total;
-  uint32_t raw_bytes, sc_bytes, x_bytes, stage_bytes;
-};
-
-// Shared memory: mbarriers | misc words | stages [nstage] (raw trits of four
-// row tiles, their scales, activations) | A slots [nslot].
-__host__ __device__ inline TcSmem tc_smem(const GemmTcParams& p) {
-  TcSmem s{};
-  const int ngc = p.tq ? (p.group >= 64 ? 1 : 64 / p.group) : 0;
-  s.raw_bytes = 4u * kPlaneColBytes * p.planes;
-  s.sc_bytes = up(4u * ngc * p.planes * 64u, 128);
-  s.x_bytes = up(64u * p.xcap, 128);
-  s.stage_bytes = s.raw_bytes + s.sc_bytes + s.x_bytes;
-  const uint32_t nbar = 2u * p.nstage + 2u * p.nslot + 3u;
-  s.bars = 0;
-  s.misc = up(nbar * 8u, 16);
-  s.stages = up(s.misc + 64u, 1024);
-  s.slots = up(s.stages + (uint32_t)p.nstage * s.stage_bytes, 1024);
-  s.total = s.slots + (uint32_t)p.nslot * kSlotBytes;
-  return s;
-}
 
 // misc words
 constexpr int kMiscTmem = 0, kMiscAbort = 1, kMiscLast = 2;
@@ -114,6 +96,28 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
   for (uint32_t it = 1;; ++it) {
     if (mbar_test(bar, parity)) return true;
     if ((it & 255u) == 0u) {
+      if (misc[kMiscAbort]) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
+        misc[kMiscAbort] = 1u;
+        return false;
+      }
+    }
+  }
+}
+
+// The same bounded wait for the sixteen decoder warps: they sleep between
+// tests, so that 512 waiting threads do not crowd the issue slots and the
+// shared-memory pipe that the single-thread producer and MMA roles need to
+// make progress (tight polling by all of them held the copy issue back until
+// the previous column had landed).
+__device__ __forceinline__ bool tc_wait_many(uint64_t* bar, uint32_t parity, volatile uint32_t* misc) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (mbar_test(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
       if (misc[kMiscAbort]) return false;
       if (global_timer_ns() - t0 > kWaitLimitNs) {
         atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
@@ -203,67 +207,79 @@ __device__ __forceinline__ long long to_ll(uint32_t v) { return (long long)(int)
 
 // The three roles of the kernel for P planes and D merged scale digits.
 // A ring: groups of D tiles (the digits of one column); a tile is 128 rows x
-// 64 k, 64 bytes per row, 64-byte swizzle.
+// 64 k, 64 bytes per row, 64-byte swizzle. Stage boundaries: a stage starts
+// at the CTA's first column and at every column that is a multiple of C (a new
+// tile or pass starts at column 0), so every role finds them by itself.
 template <int P, int D>
-__device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, const TcSmem& L, uint32_t tmem,
+__device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, const TcLayout& L, uint32_t tmem,
                                          volatile uint32_t* misc, int passes, int tpass, int q0, int q1, int W) {
-  const int NS = p.nstage;
-  const int NG = p.nslot / D;  // A groups in the ring
+  const int NS = L.NS, NG = L.NG, C = L.C;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* full = bars;
-  uint64_t* sfree = bars + NS;
-  uint64_t* afull = bars + 2 * NS;
-  uint64_t* afree = afull + p.nslot;
-  uint64_t* accfull = afree + p.nslot;
+  uint64_t* sfree = bars + kTcMaxStages;
+  uint64_t* afull = bars + 2 * kTcMaxStages;
+  uint64_t* afree = afull + kTcMaxSlots;
+  uint64_t* accfull = afree + kTcMaxSlots;
   uint64_t* accfree = accfull + 1;
   uint64_t* fin = accfree + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cols = p.cols;
   const int G = p.grid;
+  const int lg = p.tq ? 31 - __clz(p.group) : 0;  // groups are powers of two
   constexpr uint32_t kGroupBytes = (uint32_t)D * kSlotBytes;
+  constexpr int kMw = D >= 2 ? 2 : 1;  // MMA-issuing warps with work
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
-    // lane 0 waits for a free stage and posts the byte count; lanes 0-3 then
-    // copy the four row tiles' trits, lanes 4-7 their scales and lanes 8-11
-    // the activation chunks, so the copies are issued side by side
-    const int ngc = p.tq ? (p.group >= 64 ? 1 : 64 / p.group) : 0;
+    // lanes 0-3: the four row tiles' trits of the stage's columns, lanes 4-7
+    // their scale blocks, lane 8 the activations: one copy instruction
     const int groups = p.tq ? p.k / p.group : 0;
-    const uint32_t scb = (uint32_t)ngc * P * 64u;
-    // positions advance one column at a time: (tile, pass, col) and the
-    // stage ring index and phase are stepped, never divided
+    const size_t kchunks = (size_t)cols * 4;
     int col = q0 % cols, unit = q0 / cols;
     int tile = unit / passes, pass = unit % passes;
     int s = 0;
     uint32_t ph = 0;
-    for (int q = q0, i = 0; q < q1; ++q, ++i) {
-      uint32_t go = 1;
+    for (int q = q0, i = 0; q < q1; ++i) {
+      const int n = min(min(C - (col & (C - 1)), cols - col), q1 - q);
       const int nrt = min(4, p.row_tiles - 4 * tile);
       const uint32_t st = smem_u32(smem + L.stages) + (uint32_t)s * L.stage_bytes;
+      // scale blocks of the stage's columns; the last column may reach past
+      // K, where the trits are zero and no block exists
+      const int b0 = p.tq ? (col * 64) >> lg : 0;
+      const int nb = p.tq ? min(((col + n) * 64 - 1) >> lg, groups - 1) - b0 + 1 : 0;
+      uint32_t dst = 0, bytes = 0;
+      const uint8_t* src = nullptr;
+      if (lane < 4) {
+        if (lane < nrt) {
+          dst = st + (uint32_t)(lane * C * P * kPlaneColBytes);
+          src = p.trit + ((size_t)(4 * tile + lane) * cols + col) * (P * kPlaneColBytes);
+          bytes = (uint32_t)(n * P * kPlaneColBytes);
+        }
+      } else if (lane < 8) {
+        const int r4 = lane - 4;
+        if (p.tq && r4 < nrt) {
+          dst = st + L.raw_bytes + (uint32_t)(r4 * L.sgroups * P * 64);
+          src = reinterpret_cast<const uint8_t*>(p.scale + ((size_t)(4 * tile + r4) * groups + b0) * P * kTileRows);
+          bytes = (uint32_t)(nb * P * 64);
+        }
+      } else if (lane == 8) {
+        dst = st + L.raw_bytes + L.sc_bytes;
+        src = p.xp + ((size_t)pass * kchunks + (size_t)col * 4) * (size_t)tpass * 16;
+        bytes = (uint32_t)n * L.xcol_bytes;
+      }
+      uint32_t go = 1;
       if (lane == 0) {
         if (i >= NS && !tc_wait(&sfree[s], ph ^ 1u, misc)) go = 0;
         if (misc[kMiscAbort]) go = 0;
-        if (go) mbar_arrive_expect_tx(&full[s], (uint32_t)nrt * (P * kPlaneColBytes + scb) + 4u * tpass * 16u);
+        const uint32_t total = (uint32_t)(nrt * n * P * kPlaneColBytes + nrt * nb * P * 64) + (uint32_t)n * L.xcol_bytes;
+        if (go) mbar_arrive_expect_tx(&full[s], total);
       }
       go = __shfl_sync(0xffffffffu, go, 0);
       if (!go) break;
-      if (lane < 4) {
-        if (lane < nrt)
-          bulk_g2s_plain(st + lane * P * kPlaneColBytes,
-                         p.trit + ((size_t)(4 * tile + lane) * cols + col) * (P * kPlaneColBytes), P * kPlaneColBytes,
-                         &full[s]);
-      } else if (lane < 8) {
-        const int r4 = lane - 4;
-        if (p.tq && r4 < nrt)
-          bulk_g2s_plain(st + L.raw_bytes + r4 * scb,
-                         p.scale + ((size_t)(4 * tile + r4) * groups + (col * kColK2) / p.group) * P * kTileRows, scb,
-                         &full[s]);
-      } else if (lane < 12) {
-        const int w = lane - 8;
-        bulk_g2s_plain(st + L.raw_bytes + L.sc_bytes + w * tpass * 16,
-                       p.xp + (((size_t)col * 4 + w) * p.mp + (size_t)pass * tpass) * 16, tpass * 16u, &full[s]);
-      }
-      if (++col == cols) {
+      if (bytes != 0u) bulk_g2s_plain(dst, src, bytes, &full[s]);
+      q += n;
+      col += n;
+      if (col == cols) {
         col = 0;
         if (++pass == passes) {
           pass = 0;
@@ -276,60 +292,73 @@ __device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, c
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp < kDec0) {
     // ---------------------------------------------------------------- MMA
-    if (lane == 0) {
+    // warp 1 issues digits [0, dh), warp 2 digits [dh, D)
+    const int mw = warp - 1;
+    constexpr int dh = kMw == 2 ? (D + 1) / 2 : D;
+    if (lane == 0 && mw < kMw) {
+      const int da = mw == 0 ? 0 : dh, db = mw == 0 ? dh : D;
       const uint32_t idesc = tc::idesc_i8_s32(tpass);
       const uint32_t slots = smem_u32(smem + L.slots);
-      int col = q0 % cols, s = 0, j = 0, seg = 0;
+      int col = q0 % cols, s = 0, j = 0, seg = 0, cc = 0;
       uint32_t ph = 0, aph = 0;
       for (int q = q0; q < q1; ++q) {
         if (misc[kMiscAbort]) break;
         const bool first = q == q0 || col == 0;
         const bool last = q == q1 - 1 || col == cols - 1;
+        const bool sstart = q == q0 || (col & (C - 1)) == 0;
+        const bool send = q + 1 == q1 || ((col + 1) & (C - 1)) == 0 || col + 1 == cols;
         if (first && seg > 0) {
           tc_wait(accfree, (uint32_t)(seg - 1) & 1u, misc);
           tc::fence_after_sync();
         }
-        tc_wait(&full[s], ph, misc);
-        const uint32_t xs = smem_u32(smem + L.stages) + (uint32_t)s * L.stage_bytes + L.raw_bytes + L.sc_bytes;
+        if (sstart) {
+          tc_wait(&full[s], ph, misc);
+          cc = 0;
+        }
+        const uint32_t xs = smem_u32(smem + L.stages) + (uint32_t)s * L.stage_bytes + L.raw_bytes + L.sc_bytes +
+                            (uint32_t)cc * L.xcol_bytes;
         const uint64_t bd0 = tc::smem_desc(xs, tpass * 16, 128);
         const uint64_t bd1 = tc::smem_desc(xs + 2 * tpass * 16, tpass * 16, 128);
-        {
-          tc_wait(&afull[j], aph, misc);
-          tc::fence_after_sync();
-          const uint32_t a0 = slots + (uint32_t)j * kGroupBytes;
-          // the D accumulators are independent: interleave them so that
-          // consecutive instructions do not wait on one another
+        tc_wait(&afull[j], aph, misc);
+        tc::fence_after_sync();
+        const uint32_t a0 = slots + (uint32_t)j * kGroupBytes;
+        // this warp's accumulators are independent: interleave them so that
+        // consecutive instructions do not wait on one another
 #pragma unroll
-          for (int d = 0; d < D; ++d)
-            tc::mma_i8(tmem + (uint32_t)(d * tpass), tc::smem_desc_sw64(a0 + (uint32_t)d * kSlotBytes, 512), bd0, idesc,
-                       first ? 0u : 1u);
+        for (int d = 0; d < D; ++d)
+          if (d >= da && d < db)
+            tc::mma_i8(tmem + (uint32_t)(d * tpass), tc::smem_desc_sw64(a0 + (uint32_t)d * kSlotBytes, 512), bd0,
+                       idesc, first ? 0u : 1u);
 #pragma unroll
-          for (int d = 0; d < D; ++d)
-            tc::mma_i8(tmem + (uint32_t)(d * tpass), tc::smem_desc_sw64(a0 + (uint32_t)d * kSlotBytes + 32, 512), bd1,
-                       idesc, 1u);
-          tc::commit(&afree[j]);
-          if (++j == NG) {
-            j = 0;
-            aph ^= 1u;
+        for (int d = 0; d < D; ++d)
+          if (d >= da && d < db)
+            tc::mma_i8(tmem + (uint32_t)(d * tpass), tc::smem_desc_sw64(a0 + (uint32_t)d * kSlotBytes + 32, 512),
+                       bd1, idesc, 1u);
+        tc::commit(&afree[j]);
+        if (++j == NG) {
+          j = 0;
+          aph ^= 1u;
+        }
+        if (send) {
+          tc::commit(&sfree[s]);
+          if (++s == NS) {
+            s = 0;
+            ph ^= 1u;
           }
         }
-        tc::commit(&sfree[s]);
         if (last) {
           tc::commit(accfull);
           ++seg;
         }
+        ++cc;
         if (++col == cols) col = 0;
-        if (++s == NS) {
-          s = 0;
-          ph ^= 1u;
-        }
       }
       // every MMA issued has completed before tensor memory is released
       tc::commit(fin);
       const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(fin, 0u)) {
+      while (!mbar_test(fin, 0u)) {
         if (global_timer_ns() - t0 > kWaitLimitNs) {
           atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
           break;
@@ -342,23 +371,28 @@ __device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, c
     // warp (q4, c): rows 32 q4 .. 32 q4 + 31 (tensor-memory lane quarter
     // warp % 4), chunk c (16 k) of every column, and a quarter of the tokens
     // in the epilogue
-    const int ew = warp - 2, q4 = warp & 3, c = ew >> 2;
+    const int ew = warp - kDec0, q4 = warp & 3, c = ew >> 2;
     const int r = 32 * q4 + lane;
-    const int ngc = p.tq ? (p.group >= 64 ? 1 : 64 / p.group) : 0;
-    const int gl = p.tq && p.group < 64 ? (16 * c) / p.group : 0;
     // A tiles in the 64-byte swizzled K-major layout: row r at 64 r, its
     // 16-byte chunk c at chunk position c ^ ((r >> 1) & 3)
     const uint32_t slots = smem_u32(smem + L.slots) + (uint32_t)r * 64u + (uint32_t)((c ^ ((r >> 1) & 3)) * 16);
     const uint32_t taddr = tmem + ((uint32_t)(32 * q4) << 16);
-    int col = q0 % cols, unit = q0 / cols, s = 0, j = 0, seg = 0, gc = 0;
+    int col = q0 % cols, unit = q0 / cols, s = 0, j = 0, seg = 0, gc = 0, cc = 0, b0 = 0;
     uint32_t ph = 0, aph = 0;
     for (int q = q0; q < q1; ++q) {
       const bool last = q == q1 - 1 || col == cols - 1;
-      tc_wait(&full[s], ph, misc);
+      if (q == q0 || (col & (C - 1)) == 0) {
+        tc_wait_many(&full[s], ph, misc);
+        cc = 0;
+        b0 = p.tq ? (col * 64) >> lg : 0;
+      }
+      const bool send = q + 1 == q1 || ((col + 1) & (C - 1)) == 0 || col + 1 == cols;
       const uint32_t st = smem_u32(smem + L.stages) + (uint32_t)s * L.stage_bytes;
-      const uint32_t raw = st + (uint32_t)(q4 * P * kPlaneColBytes + lane * kChunkBytes + 4 * c);
-      const uint32_t scs = st + L.raw_bytes + (uint32_t)((q4 * ngc + gl) * P * 64 + lane * 2);
-      if (++s == NS) {
+      const uint32_t raw = st + (uint32_t)((q4 * C + cc) * P * kPlaneColBytes + lane * kChunkBytes + 4 * c);
+      const int blk = p.tq ? ((col * 64 + 16 * c) >> lg) - b0 : 0;  // scale block of this chunk in the stage
+      const uint32_t scs = st + L.raw_bytes + (uint32_t)((q4 * L.sgroups + blk) * P * 64 + lane * 2);
+      ++cc;
+      if (send && ++s == NS) {
         s = 0;
         ph ^= 1u;
       }
@@ -379,7 +413,7 @@ __device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, c
         lo2[pl] = lo[pl] >> 16;
         hi2[pl] = hi[pl] >> 16;
       }
-      if (gc >= NG) tc_wait(&afree[j], aph ^ 1u, misc);
+      if (gc >= NG) tc_wait_many(&afree[j], aph ^ 1u, misc);
       const uint32_t a = slots + (uint32_t)j * kGroupBytes;
       constexpr int kB = kDigitBits<P>;
       constexpr uint32_t kMask = (1u << kB) - 1u;
@@ -421,7 +455,7 @@ __device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, c
       const int tile = ucur / passes, pass = ucur % passes;
       // the tile's whole K range lies in this CTA's range
       const bool owned = col == 0 && q0 <= ucur * cols;
-      tc_wait(accfull, (uint32_t)seg & 1u, misc);
+      tc_wait_many(accfull, (uint32_t)seg & 1u, misc);
       tc::fence_after_sync();
       const int n = tile * kTcRows + r;
       const int tq4 = tpass >> 2, tb = c * tq4, t0 = pass * tpass;
@@ -480,32 +514,33 @@ __device__ __forceinline__ void tc_roles(const GemmTcParams& p, uint8_t* smem, c
 template <int P>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmTcParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  const TcSmem L = tc_smem(p);
-  const int NS = p.nstage, NA = p.nslot;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
-  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L.misc);
   const int warp = threadIdx.x >> 5;
 
   int D7 = 1;
   if (p.tq) D7 = (int)__ldg(reinterpret_cast<const unsigned*>(p.header + kDigitsOffset));
-  const int D = tc_merged_digits(P, D7);  // digits of the merged A operand
-  bool bad = D7 < 1 || D7 > kTcMaxDigits || (P > 1 && !p.tq) || NA / (D < 1 ? 1 : D) < 1;
+  bool bad = D7 < 1 || D7 > kTcMaxDigits || (P > 1 && !p.tq);
+  const int D = bad ? 1 : tc_merged_digits(P, D7);  // digits of the merged A operand
   int passes = 1, tpass = 16;
-  tc_passes(bad ? 1 : D, p.m16, &passes, &tpass);
-  bad = bad || tpass > p.xcap || passes > p.passes_cap;
+  tc_passes(D, p.m16, &passes, &tpass);
+  TcLayout L;
+  bad = !tc_layout(P, p.tq, p.group, D, tpass, &L) || bad || passes > p.passes_cap;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + L.misc);
+  const uint32_t nmw = D >= 2 ? 2u : 1u;  // MMA warps that commit
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(&bars[i], 1);       // full
-      mbar_init(&bars[NS + i], 1);  // sfree
+    for (int i = 0; i < L.NS; ++i) {
+      mbar_init(&bars[i], 1);                   // full
+      mbar_init(&bars[kTcMaxStages + i], nmw);  // sfree
     }
-    for (int j = 0; j < NA; ++j) {
-      mbar_init(&bars[2 * NS + j], kDecWarps);  // afull
-      mbar_init(&bars[2 * NS + NA + j], 1);     // afree
+    for (int j = 0; j < L.nslot; ++j) {
+      mbar_init(&bars[2 * kTcMaxStages + j], kDecWarps);            // afull
+      mbar_init(&bars[2 * kTcMaxStages + kTcMaxSlots + j], nmw);    // afree
     }
-    mbar_init(&bars[2 * NS + 2 * NA], 1);              // accfull
-    mbar_init(&bars[2 * NS + 2 * NA + 1], kDecWarps);  // accfree
-    mbar_init(&bars[2 * NS + 2 * NA + 2], 1);          // fin
+    uint64_t* acc = bars + 2 * kTcMaxStages + 2 * kTcMaxSlots;
+    mbar_init(acc, nmw);            // accfull
+    mbar_init(acc + 1, kDecWarps);  // accfree
+    mbar_init(acc + 2, nmw);        // fin
     misc[kMiscAbort] = 0u;
     misc[kMiscLast] = 0u;
     if (bad && blockIdx.x == 0) atomicOr(&g_dev_error, TERN_DEVERR_FORMAT);
@@ -547,14 +582,30 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   }
 }
 
-// Activations in MMA order: xp[(kc * mp + t) * 16 + j] = xq[t][16 kc + perm(j)]
-// with perm = 0,8,1,9,...,7,15 (the decode order of a packed word); zero for
-// tokens t >= m and columns k >= K.
-__global__ void tc_prep_x_kernel(const int8_t* __restrict__ xq, int m, int k, int kchunks, int mp, bool vec,
+// Activations in MMA order, pass-major so that the columns of one token pass
+// are contiguous: xp[((pass * kchunks + kc) * tpass + t) * 16 + j] =
+// xq[pass * tpass + t][16 kc + perm(j)] with perm = 0,8,1,9,...,7,15 (the
+// decode order of a packed word); zero for tokens >= m and columns k >= K.
+// The pass split follows the packed header's digit count, read here as in the
+// GEMM kernel (an invalid count is flagged there; here it only keeps the
+// writes inside the workspace).
+__global__ void tc_prep_x_kernel(const int8_t* __restrict__ xq, int m, int k, int kchunks, long long total_max,
+                                 int planes, int tq, const uint8_t* __restrict__ header, int m16, bool vec,
                                  uint8_t* __restrict__ xp) {
+  int D7 = 1;
+  if (tq) {
+    D7 = (int)__ldg(reinterpret_cast<const unsigned*>(header + kDigitsOffset));
+    if (D7 < 1 || D7 > kTcMaxDigits) D7 = 1;
+  }
+  int passes, tpass;
+  tc_passes(tc_merged_digits(planes, D7), m16, &passes, &tpass);
+  const long long total = (long long)passes * kchunks * tpass;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long long)kchunks * mp) return;
-  const int t = (int)(idx % mp), kc = (int)(idx / mp);
+  if (idx >= total || idx >= total_max) return;
+  const int tl = (int)(idx % tpass);
+  const long long rest = idx / tpass;
+  const int kc = (int)(rest % kchunks), pass = (int)(rest / kchunks);
+  const int t = pass * tpass + tl;
   uint4 v = make_uint4(0u, 0u, 0u, 0u);
   if (t < m) {
     const int k0 = kc * 16;
@@ -574,20 +625,16 @@ __global__ void tc_prep_x_kernel(const int8_t* __restrict__ xq, int m, int k, in
 
 template <int P>
 int launch_p(const GemmTcParams& p, void* stream) {
-  const TcSmem s = tc_smem(p);
   auto kern = gemm_tc_kernel<P>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s.total);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
   if (e != cudaSuccess) return (int)e;
-  kern<<<p.grid, kThreads, s.total, static_cast<cudaStream_t>(stream)>>>(p);
+  kern<<<p.grid, kThreads, kTcSmemBytes, static_cast<cudaStream_t>(stream)>>>(p);
   return (int)cudaGetLastError();
 }
 
 }  // namespace
 
-size_t gemm_tc_smem_bytes(const GemmTcParams& p) { return tc_smem(p).total; }
-
 int launch_gemm_tc(const GemmTcParams& p, void* stream) {
-  if (tc_smem(p).total > 227u * 1024u) return -1;
   switch (p.planes) {
     case 1: return launch_p<1>(p, stream);
     case 2: return launch_p<2>(p, stream);
@@ -597,13 +644,14 @@ int launch_gemm_tc(const GemmTcParams& p, void* stream) {
   }
 }
 
-int launch_tc_prep_x(const int8_t* xq, int m, int k, int kchunks, int mp, uint8_t* xp, void* stream) {
-  const long long total = (long long)kchunks * mp;
-  if (total == 0) return 0;
+int launch_tc_prep_x(const int8_t* xq, int m, int k, int kchunks, int total_max, const GemmTcParams& p, uint8_t* xp,
+                     void* stream) {
+  if (total_max <= 0) return 0;
   const bool vec = (reinterpret_cast<uintptr_t>(xq) & 15u) == 0 && k % 16 == 0;
   const int threads = 256;
-  const long long blocks = (total + threads - 1) / threads;
-  tc_prep_x_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(xq, m, k, kchunks, mp, vec, xp);
+  const long long blocks = ((long long)total_max + threads - 1) / threads;
+  tc_prep_x_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      xq, m, k, kchunks, total_max, p.planes, p.tq, p.header, p.m16, vec, xp);
   return (int)cudaGetLastError();
 }
 

@@ -119,28 +119,34 @@ struct Gemv2wParams {
 
 // Batched GEMM on the tensor cores (tcgen05 kind::i8), m >= 16 tokens. The
 // fp16 group scale s of every (plane, row, group) is an integer u = |s| / 2^-24
-// written in D base-128 digits u_d; the A operand of digit d holds
-// sign(s) * t * u_d (int8), so one int32 accumulator per digit sums over all
-// groups and planes and the exact result is sum_d 128^d * acc_d (int64).
+// written in D' digits of b bits (b = 7, 6, 5 for one, two, three or four
+// planes); the A operand of digit d holds sum_p sign(s_p) * t_p * u_{p,d}
+// (int8), so one int32 accumulator per digit sums over all groups and planes
+// and the exact result is sum_d 2^(b d) * acc_d (int64).
 constexpr int kTcRows = 128;       // weight rows per MMA tile (four 32-row tiles)
 constexpr int kTcMaxDigits = 6;    // 7-bit digits: fp16 magnitudes are below 2^40 units of 2^-24
 constexpr int kTcMaxMerged = 9;    // merged digits (5 bits for three or four planes)
 constexpr int kTcMaxTokens = 256;  // tokens per launch (MMA N <= 256)
+constexpr int kTcSmemBytes = 227 * 1024;   // dynamic shared memory of every launch
+constexpr int kTcSlotBytes = kTcRows * 64;  // one A tile: 128 rows x 64 k, int8
+constexpr int kTcMaxStages = 12;
+constexpr int kTcMaxSlots = 18;             // A tiles: groups of D' tiles (see tc_layout)
+constexpr int kTcMaxColsPerStage = 4;
 
 struct GemmTcParams {
   const uint8_t* trit;           // trit stream
   const uint16_t* scale;         // TQ scale stream, or nullptr
   const uint8_t* header;         // packed header (digit count at kDigitsOffset)
-  const uint8_t* xp;             // activations in MMA order [cols*4][mp][16] (workspace)
+  const uint8_t* xp;             // activations in MMA order [passes][cols*4][tpass][16] (workspace)
   const float* xscale;           // [m]
   void* y;                       // [m][n]
   unsigned long long* part;      // [m][n_pad] int64 partial sums (zero on entry and exit)
   unsigned* cnt;                 // [tiles][passes_cap] arrival counters (zero on entry and exit)
   int n, k, planes, group, cols, row_tiles, tiles, n_pad;
-  int m, m16, mp, xcap, passes_cap;
+  int m, m16, passes_cap;
   int tq, out_bf16;
   float tensor_scale;
-  int nstage, nslot, grid;
+  int grid;
 };
 
 // Digits of the merged A operand for P planes and D 7-bit digits of the
@@ -161,9 +167,41 @@ TERN_HD inline void tc_passes(int digits, int m16, int* passes, int* tpass) {
   *tpass = t;
 }
 
+// Shared-memory plan of one launch, from the merged digit count D and the
+// tokens per pass: mbarriers and misc words | input stages | A tiles (at the
+// top). A stage holds C consecutive 64-k columns of four row tiles (trits,
+// scale blocks, activations), so that one bulk-copy instruction per stage
+// fetches all of them; C is the widest of 4, 2, 1 that leaves three stages.
+struct TcLayout {
+  uint32_t bars, misc, stages, slots;  // byte offsets
+  uint32_t raw_bytes, sc_bytes, xcol_bytes, stage_bytes;
+  int C, NS, nslot, NG, sgroups;       // columns per stage, stages, A tiles, A groups, scale blocks per row tile
+};
+TERN_HD inline bool tc_layout(int planes, int tq, int group, int digits, int tpass, TcLayout* L) {
+  L->NG = digits <= 4 ? 4 : (digits <= 6 ? 3 : 2);
+  L->nslot = L->NG * digits;
+  L->bars = 0;
+  L->misc = (uint32_t)(2 * kTcMaxStages + 2 * kTcMaxSlots + 3) * 8u;
+  L->stages = 1024;
+  L->slots = (uint32_t)kTcSmemBytes - (uint32_t)L->nslot * kTcSlotBytes;
+  L->xcol_bytes = 4u * (uint32_t)tpass * 16u;
+  for (int C = kTcMaxColsPerStage; C >= 1; C >>= 1) {
+    const int sg = tq ? (64 * C >= group ? 64 * C / group : 1) : 0;
+    L->C = C;
+    L->sgroups = sg;
+    L->raw_bytes = 4u * (uint32_t)(C * planes * kPlaneColBytes);
+    L->sc_bytes = ((uint32_t)(4 * sg * planes * 64) + 127u) & ~127u;
+    L->stage_bytes = L->raw_bytes + L->sc_bytes + (((uint32_t)C * L->xcol_bytes + 127u) & ~127u);
+    const int ns = L->slots > L->stages ? (int)((L->slots - L->stages) / L->stage_bytes) : 0;
+    L->NS = ns < kTcMaxStages ? ns : kTcMaxStages;
+    if (L->NS >= 3) break;
+  }
+  return L->misc + 64u <= L->stages && L->nslot <= kTcMaxSlots && L->NS >= 2;
+}
+
 int launch_gemm_tc(const GemmTcParams& p, void* stream);  // -1: no kernel for this shape
-size_t gemm_tc_smem_bytes(const GemmTcParams& p);
-int launch_tc_prep_x(const int8_t* xq, int m, int k, int kchunks, int mp, uint8_t* xp, void* stream);
+int launch_tc_prep_x(const int8_t* xq, int m, int k, int kchunks, int total_max, const GemmTcParams& p, uint8_t* xp,
+                     void* stream);
 int read_clear_dev_error_gemm_tc(void* stream, unsigned* out);
 
 // Launchers return cudaError_t values as int (0 = success).
