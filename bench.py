@@ -529,7 +529,7 @@ def committed_traffic():
             if ":" in line and not line.startswith("#"):
                 key, val = line.split(":", 1)
                 vals[key.strip()] = val.strip()
-    src = os.path.join(ROOT, "packed_ternary_weight_b200", "csrc", "tern_gemv2w.cu")
+    src = os.path.join(ROOT, "packed_ternary_weight_b200", "csrc", "tern_gemv2w_kernel.cuh")
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     if vals.get("kernel_source_sha256_16") != h:
         return None

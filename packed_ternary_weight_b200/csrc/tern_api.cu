@@ -124,15 +124,20 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
 // shared memory allows next to the resident activation images. Applies when
 // the launch has at least four tiles per SM (smaller launches are spread
 // over the SMs by K splits in the row-group kernel).
-bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, int sms, Gemv2wParams& p) {
+// With mt > 1 tokens (one problem, integer activations) a launch of half a
+// tile per SM is enough: each tile carries mt tokens' work.
+bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, int sms, Gemv2wParams& p,
+                 int mt = 1) {
   const bool bt3 = L.fmt == TERN_FMT_BT3;
   if (bt3 && xmode != kXBf16) return false;
   if (nprob > kMaxProblemsW) return false;
+  if (mt > 1 && (nprob != 1 || bt3 || xmode == kXBf16 || mt > kMaxTokensW)) return false;
   int begin[kMaxProblemsW + 1];
   begin[0] = 0;
   for (int i = 0; i < nprob; ++i) begin[i + 1] = begin[i] + row_tiles[i];
   const int T = begin[nprob];
-  if (T < 4 * sms) return false;
+  if (T < (mt > 1 ? (sms + 1) / 2 : 4 * sms)) return false;
+  p.mt = mt;
   // the kernel's index arithmetic is 32-bit: tiles x CTAs and a CTA's
   // columns x warps stay below 2^31
   if ((long long)T * sms >= (1ll << 31) || ((long long)T / sms + 1) * L.cols * 16 >= (1ll << 31)) return false;
@@ -367,6 +372,36 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
   }
   const size_t in_elem = xmode == kXInt8 ? 1 : 2;
   const size_t out_elem = out == TERN_OUT_F32 ? 4 : 2;
+  if (m >= 2 && xmode != kXBf16 && L.fmt != TERN_FMT_BT3) {
+    // several tokens on the one-CTA-per-SM kernel, up to eight per pass over
+    // the weights (more tokens: passes of near-equal size, at least two
+    // tokens each), when the layer has half a tile per SM and the images fit
+    Gemv2wParams w{};
+    const int rt = L.row_tiles;
+    const int passes = (m + kMaxTokensW - 1) / kMaxTokensW;
+    if (plan_gemv2w(L, &rt, 1, xmode, sms, w, (m + passes - 1) / passes)) {
+      for (int c = 0, t0 = 0; c < passes; ++c) {
+        const int mc = (m - t0) / (passes - c);
+        if (mc != w.mt && !plan_gemv2w(L, &rt, 1, xmode, sms, w, mc)) return TERN_EUNSUPPORTED;
+        w.out_bf16 = out == TERN_OUT_BF16;
+        Gemv2wProblem& q = w.prob[0];
+        q.trit = base + L.trit_offset;
+        q.scale = w.tq ? reinterpret_cast<const uint16_t*>(base + L.scale_offset) : nullptr;
+        q.x = static_cast<const uint8_t*>(d_x) + (size_t)t0 * L.k * in_elem;
+        q.xscale = d_xscale ? d_xscale + t0 : nullptr;
+        q.y = static_cast<uint8_t*>(d_y) + (size_t)t0 * L.n * out_elem;
+        q.n = L.n;
+        q.row_tiles = L.row_tiles;
+        q.tensor_scale = desc->tensor_scale;
+        w.x_vec = aligned16(q.x) && L.k % 16 == 0;
+        const int rc = launch_gemv2w(w, xmode, pdl, stream);
+        if (rc < 0) return TERN_EUNSUPPORTED;
+        if (rc != 0) return TERN_ECUDA;
+        t0 += mc;
+      }
+      return TERN_OK;
+    }
+  }
   const int mt_max = gemv2_mt(xmode, m);
   for (int t0 = 0; t0 < m; t0 += mt_max) {
     const int mc = std::min(mt_max, m - t0);
@@ -536,6 +571,7 @@ extern "C" tern_status tern_device_error(void* stream) {
   unsigned v = 0;
   if (read_clear_dev_error_gemv2(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_gemv2w(stream, &v) != 0) return TERN_ECUDA;
+  if (read_clear_dev_error_gemv2w_mt(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_stream(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_gemv3(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_gemm_tc(stream, &v) != 0) return TERN_ECUDA;

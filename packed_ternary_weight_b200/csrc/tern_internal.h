@@ -49,6 +49,7 @@ enum XMode : int { kXInt8 = 0, kXBf16 = 1, kXBf16Q8 = 2 };
 constexpr int kMaxProblems = 32;   // independent GEMVs in one launch of the row-group kernel
 constexpr int kMaxProblemsW = 256; // ... of the one-CTA-per-SM kernel (parameter block < 32 KB)
 constexpr int kMaxSlotsW = 16;     // problems one CTA of that kernel may touch
+constexpr int kMaxTokensW = 8;     // tokens of one problem per launch of that kernel
 constexpr int kMaxCluster = 16;   // K-splits reduced through one thread-block cluster
 
 struct Gemv2Problem {
@@ -79,6 +80,7 @@ struct Gemv2Params {
   int stage_cols;           // columns per pipeline stage
   int nstage;               // stages per warp ring
   int x_vec;                // activations may be read with 16-byte loads
+  int mt;                   // tokens of the (single) problem sharing the weight stream, or 1
   void* ws_part;            // global fallback: partials [ks][m][row_tiles*32]
   unsigned* ws_cnt;         // global fallback: arrival counters [grid.x]
 };
@@ -112,6 +114,7 @@ struct Gemv2wParams {
   int stage_cols, nstage;   // per-warp ring: columns per stage, stages
   int xslots;               // activation images resident per CTA
   int x_vec;                // activations may be read with 16-byte loads
+  int mt;                   // tokens of the (single) problem sharing the weight stream, or 1
   int early_w;              // set at launch: weights may be requested before the dependency wait
   int tile_begin[kMaxProblemsW + 1];  // first tile of each problem; [nprob] = tiles_total
   Gemv2wProblem prob[kMaxProblemsW];  // last member: the kernel copies only its own problems
@@ -207,8 +210,10 @@ int read_clear_dev_error_gemm_tc(void* stream, unsigned* out);
 // Launchers return cudaError_t values as int (0 = success).
 int launch_gemv2(const Gemv2Params& p, int xmode, bool pdl, void* stream);  // -1: no kernel
 int launch_gemv2w(const Gemv2wParams& p, int xmode, bool pdl, void* stream);  // -1: no kernel
+int launch_gemv2w_mt(const Gemv2wParams& p, int xmode, bool pdl, void* stream);  // p.mt > 1
 size_t gemv2w_smem_bytes(const Gemv2wParams& p, int xmode);
 int read_clear_dev_error_gemv2w(void* stream, unsigned* out);
+int read_clear_dev_error_gemv2w_mt(void* stream, unsigned* out);
 int launch_quantize(const uint16_t* x, int m, int k, int8_t* xq, float* xs, void* stream);
 
 int read_clear_dev_error_gemv2(void* stream, unsigned* out);
