@@ -163,7 +163,12 @@ tern_status tern_gemv(const tern_desc* desc, const void* d_packed, tern_act act,
  * 256 tokens per launch); the fp16 group scales are split into small integer
  * digits folded into the int8 weight operand, so the result stays exact.
  * That path needs the workspace tern_workspace_size(desc, m) reports
- * (TERN_ENOSPACE without it).
+ * (TERN_ENOSPACE without it); from m = 9 it is taken whenever that workspace
+ * is given, and from m = 5 when the activations of a CUDA-core pass would
+ * crowd shared memory (long K). Otherwise, with 2..15 tokens, the weights are
+ * read once per pass of up to eight tokens on the CUDA cores; those kernels
+ * cover BitNet, TQ{1..4}P with g = 256, TQ2P with g = 32 and TQ3P with g = 64
+ * (TERN_EUNSUPPORTED for other plane and group combinations).
  */
 tern_status tern_gemm_batched(const tern_desc* desc, const void* d_packed, int32_t m, tern_act act,
                               const void* d_x, const float* d_xscale, tern_out out, void* d_y,

@@ -307,7 +307,18 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
   const int sms = device_sms();
   const uint8_t* base = static_cast<const uint8_t*>(d_packed);
   const bool pdl = (desc->flags & TERN_F_PDL) != 0;
-  if (m >= 16) {
+  // tensor cores from 16 tokens, and from 9 when a workspace is given (the
+  // CUDA-core path below takes more than eight tokens in two passes, slower
+  // than one tensor-core launch padded to 16 tokens); also from 5 when the
+  // CUDA-core pass's activation images leave room for fewer than 16 warps
+  // (long K)
+  bool use_tc = m >= 16 || (m >= 9 && d_ws);
+  if (!use_tc && m >= 5 && d_ws && xmode != kXBf16 && L.fmt != TERN_FMT_BT3) {
+    Gemv2wParams w{};
+    const int rt = L.row_tiles;
+    use_tc = plan_gemv2w(L, &rt, 1, xmode, sms, w, std::min(m, kMaxTokensW)) && w.nw < 16;
+  }
+  if (use_tc) {
     const int mb = std::min(m, kTcMaxTokens);
     const PlanTc tp = plan_tc(L, mb, xmode, sms);
     if (tp.ok) {
@@ -366,8 +377,8 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
       q.tensor_scale = desc->tensor_scale;
       w.x_vec = aligned16(d_x) && L.k % 16 == 0;
       const int rc = launch_gemv2w(w, xmode, pdl, stream);
-      if (rc < 0) return TERN_EUNSUPPORTED;
-      return rc == 0 ? TERN_OK : TERN_ECUDA;
+      if (rc >= 0) return rc == 0 ? TERN_OK : TERN_ECUDA;
+      // no kernel for this plane count and group size: the row-group kernel below
     }
   }
   const size_t in_elem = xmode == kXInt8 ? 1 : 2;
@@ -395,11 +406,12 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
         q.tensor_scale = desc->tensor_scale;
         w.x_vec = aligned16(q.x) && L.k % 16 == 0;
         const int rc = launch_gemv2w(w, xmode, pdl, stream);
+        if (rc < 0 && c == 0) break;  // no kernel for this plane count and group size: the row-group kernel below
         if (rc < 0) return TERN_EUNSUPPORTED;
         if (rc != 0) return TERN_ECUDA;
         t0 += mc;
+        if (c + 1 == passes) return TERN_OK;
       }
-      return TERN_OK;
     }
   }
   const int mt_max = gemv2_mt(xmode, m);
@@ -447,7 +459,7 @@ extern "C" tern_status tern_workspace_size(const tern_desc* desc, int32_t m, siz
   if (m < 0) return TERN_EINVAL;
   const int sms = device_sms();
   size_t need = 0;
-  if (m >= 16) {
+  if (m >= 2) {  // tensor-core paths (a few tokens: group accumulators; more: scale digits)
     for (int xmode = 0; xmode < 3; ++xmode) {
       const PlanTc tp = plan_tc(L, std::min<int>(m, kTcMaxTokens), xmode, sms);
       if (tp.ok) need = std::max(need, tp.total);
@@ -529,8 +541,8 @@ extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, 
       }
       w.x_vec = vec;
       const int rc = launch_gemv2w(w, xmode, pdl, stream);
-      if (rc < 0) return TERN_EUNSUPPORTED;
-      return rc == 0 ? TERN_OK : TERN_ECUDA;
+      if (rc >= 0) return rc == 0 ? TERN_OK : TERN_ECUDA;
+      // no kernel for this plane count and group size: the row-group kernel below
     }
   }
   // the row-group kernel takes up to kMaxProblems problems per launch

@@ -70,92 +70,20 @@ constexpr int kThreads = 32 * (kDec0 + kDecWarps);
 constexpr int kSlotBytes = kTcSlotBytes;  // one A tile: 128 rows x 64 k
 constexpr int kTmemCols = 512;
 
-// misc words
-constexpr int kMiscTmem = 0, kMiscAbort = 1, kMiscLast = 2;
-
-// Non-blocking test of a phase.
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait by polling (a suspended try_wait resumes too late for the
-// one-thread roles on the critical path). Gives up at once when another thread
-// of the CTA has already given up (misc[kMiscAbort]), so that a failure costs
-// about one time limit, not one per wait.
-__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* misc) {
-  if (mbar_test(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_test(bar, parity)) return true;
-    if ((it & 255u) == 0u) {
-      if (misc[kMiscAbort]) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
-        misc[kMiscAbort] = 1u;
-        return false;
-      }
-    }
-  }
-}
-
-// The same bounded wait for the sixteen decoder warps: they sleep between
-// tests, so that 512 waiting threads do not crowd the issue slots and the
-// shared-memory pipe that the single-thread producer and MMA roles need to
-// make progress (tight polling by all of them held the copy issue back until
-// the previous column had landed).
-__device__ __forceinline__ bool tc_wait_many(uint64_t* bar, uint32_t parity, volatile uint32_t* misc) {
-  if (mbar_test(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(64);
-    if (mbar_test(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (misc[kMiscAbort]) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
-        misc[kMiscAbort] = 1u;
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Bulk copy without a cache-policy hint (a tile's weights are read again by
-// its next token pass, so they should stay in L2).
-__device__ __forceinline__ void bulk_g2s_plain(uint32_t dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst_smem),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
-}
+using tc::kMiscAbort;
+using tc::kMiscLast;
+using tc::kMiscTmem;
+using tc::bulk_g2s_plain;
+using tc::mbar_arrive;
+using tc::mbar_test;
+using tc::tc_wait;
+using tc::tc_wait_many;
 
 __device__ __forceinline__ void named_sync_decoders() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kDecWarps) : "memory"); }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ uint32_t lds16(uint32_t a) {
-  unsigned short v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
-}
+using tc::lds16;
+using tc::lds32;
+using tc::sts128;
 
 // Digit width and per-plane bias of the merged A operand for P planes.
 template <int P>

@@ -93,5 +93,89 @@ __device__ __forceinline__ void ld_x4_sync(uint32_t taddr, uint32_t (&v)[4]) {
       : "memory");
 }
 
+// Words after the mbarriers of a tensor-core kernel: the tensor-memory base
+// address, the abort flag of its bounded waits, the last-arrival flag.
+constexpr int kMiscTmem = 0, kMiscAbort = 1, kMiscLast = 2;
+
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait by polling (a suspended try_wait resumes too late for the
+// one-thread roles on the critical path). Gives up at once when another thread
+// of the CTA has already given up (misc[kMiscAbort]), so that a failure costs
+// about one time limit, not one per wait.
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* misc) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test(bar, parity)) return true;
+    if ((it & 255u) == 0u) {
+      if (misc[kMiscAbort]) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
+        misc[kMiscAbort] = 1u;
+        return false;
+      }
+    }
+  }
+}
+
+// The same bounded wait for roles of many warps: they sleep between tests, so
+// that hundreds of waiting threads do not crowd the issue slots and the
+// shared-memory pipe that the single-thread producer and MMA roles need.
+__device__ __forceinline__ bool tc_wait_many(uint64_t* bar, uint32_t parity, volatile uint32_t* misc) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (mbar_test(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (misc[kMiscAbort]) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
+        misc[kMiscAbort] = 1u;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Bulk copy without a cache-policy hint (a tile's weights are read again by
+// its next token pass, so they should stay in L2).
+__device__ __forceinline__ void bulk_g2s_plain(uint32_t dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst_smem),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+
 }  // namespace tc
 }  // namespace tern

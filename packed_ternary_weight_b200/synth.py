@@ -169,7 +169,7 @@ def bt3_llama_layers():
 
 
 PREFILL_SHAPES = (("ffn_up", 14336, 4096), ("ffn_down", 4096, 14336))
-PREFILL_TOKENS = (1, 4, 16, 64, 256)
+PREFILL_TOKENS = (1, 2, 4, 8, 16, 64, 256)
 
 
 def tq2p_prefill_layers():

@@ -75,8 +75,9 @@ def check(tern, layer, m, act=None, rows=None, out=None):
         assert bad.size == 0, f"{len(bad)} mismatches, first {bad[:4].tolist()}"
 
 
-@pytest.mark.parametrize("m", [16, 17, 33, 64, 100, 256])
+@pytest.mark.parametrize("m", [9, 12, 15, 16, 17, 33, 64, 100, 256])
 def test_tq2p_g32_small_bit_exact(tern, m):
+    # from 9 tokens a call with a workspace runs on the tensor cores (padded to 16)
     check(tern, synth.tq_layer(300, 1024, 2, 32, seed=60 + m), m)
 
 
