@@ -88,7 +88,7 @@ __host__ __device__ inline Plan2w plan2w(const Gemv2wParams& p, int xmode) {
     s.sx_off = align_up(s.sum_off + 4 * (size_t)(tq ? p.groups : p.cols + 1), 16);
     s.slot_bytes = align_up(s.sx_off + 16, 128);
   }
-  const size_t nimg = p.mt > 1 ? (size_t)p.mt : (size_t)p.xslots;
+  const size_t nimg = p.mt > 1 ? (size_t)gemv2w_mt_pad(p.mt) : (size_t)p.xslots;
   size_t off = 0;
   s.bars = off;
   off = align_up(off + (size_t)p.nw * p.nstage * 8, 128);
@@ -229,9 +229,10 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
     return lo;
   };
   const int qa = prob_of(t0), nslots = min(kMaxSlotsW, prob_of(t1 - 1) - qa + 1);  // the host keeps it <= 16
-  // activation images: one per problem, or one per token of the single problem
+  // activation images: one per problem, or one per token of the single
+  // problem, padded to MT with zero images
   const int mt = MT > 1 ? p.mt : 1;
-  const int nimg = MT > 1 ? mt : nslots;
+  const int nimg = MT > 1 ? MT : nslots;
   {  // slot s = problem qa + s
     constexpr int kPw = (int)(sizeof(Gemv2wProblem) / 4);
     const int* src = reinterpret_cast<const int*>(&pg.prob[qa]);
@@ -319,6 +320,7 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
     const int nthr = blockDim.x;
     auto chunk_load = [&](int f) -> uint4 {
       const int s = f / nch, c = f - s * nch;
+      if (MT > 1 && s >= mt) return make_uint4(0u, 0u, 0u, 0u);  // padding token
       const void* xp = MT > 1 ? static_cast<const void*>(static_cast<const int8_t*>(sprob[0].x) +
                                                          (size_t)s * p.k * (kQ8 ? 2 : 1))
                               : sprob[s].x;
@@ -396,7 +398,7 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
         const float a = __uint_as_float(amax[threadIdx.x]);
         sx = a > 0.f ? __fdiv_rn(a, 127.0f) : 0.f;
       } else {
-        sx = MT > 1 ? sprob[0].xscale[threadIdx.x] : sprob[threadIdx.x].xscale[0];
+        sx = MT > 1 ? (threadIdx.x < mt ? sprob[0].xscale[threadIdx.x] : 0.f) : sprob[threadIdx.x].xscale[0];
       }
       *reinterpret_cast<float*>(slot_ptr(threadIdx.x) + sp.sx_off) = sx;
     }
@@ -515,7 +517,7 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
         v[t] = acc64t[t];
       } else {
         const int* pre = reinterpret_cast<const int*>(slot_ptr(t) + sp.sum_off);
-        v[t] = t < mt ? (long long)(pre[hi] - pre[lo] - acct[t][0]) : 0;
+        v[t] = (long long)(pre[hi] - pre[lo] - acct[t][0]);
       }
     }
     if (lo == 0 && hi == cols) {
@@ -640,17 +642,15 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
         const uint32_t xo = (uint32_t)(cc * kColK2 + wi * 16);
 #pragma unroll
         for (int t = 0; t < MT; ++t) {
-          if (t < mt) {
-            const int4 xv = u4_as_i4(lds128<0>(x32 + (uint32_t)t * (uint32_t)sp.slot_bytes + xo));
+          const int4 xv = u4_as_i4(lds128<0>(x32 + (uint32_t)t * (uint32_t)sp.slot_bytes + xo));
 #pragma unroll
-            for (int q = 0; q < P; ++q) {
-              int a = acct[t][q];
-              a = dp4a_ss((int)dg[q][0], xv.x, a);
-              a = dp4a_ss((int)dg[q][1], xv.y, a);
-              a = dp4a_ss((int)dg[q][2], xv.z, a);
-              a = dp4a_ss((int)dg[q][3], xv.w, a);
-              acct[t][q] = a;
-            }
+          for (int q = 0; q < P; ++q) {
+            int a = acct[t][q];
+            a = dp4a_ss((int)dg[q][0], xv.x, a);
+            a = dp4a_ss((int)dg[q][1], xv.y, a);
+            a = dp4a_ss((int)dg[q][2], xv.z, a);
+            a = dp4a_ss((int)dg[q][3], xv.w, a);
+            acct[t][q] = a;
           }
         }
         if constexpr (kTQ) {
@@ -662,18 +662,18 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
             const int gst = gl - ga_stage;
             int gsx[MT];  // each token's sum of x over the group
 #pragma unroll
-            for (int t = 0; t < MT; ++t)
-              gsx[t] = t < mt ? reinterpret_cast<const int*>(slot_ptr(t) + sp.sum_off)[gl] : 0;
+            for (int t = 0; t < MT; ++t) gsx[t] = reinterpret_cast<const int*>(slot_ptr(t) + sp.sum_off)[gl];
 #pragma unroll
             for (int q = 0; q < P; ++q) {
               const uint32_t h = sst[(gst * P + q) * kTileRows + lane];
               const int ex = (int)((h >> 10) & 0x1Fu), man = (int)(h & 0x3FFu);
               int mm = ex ? man + 1024 : man;
               if (h & 0x8000u) mm = -mm;
-              const long long scl = 1ll << (ex ? ex - 1 : 0);
+              const int sh = ex ? ex - 1 : 0;
 #pragma unroll
               for (int t = 0; t < MT; ++t) {
-                acc64t[t] += (long long)(mm * (gsx[t] - acct[t][q])) * scl;
+                // the integer product (exact in 32 bits) shifted to units of 2^-24
+                acc64t[t] += (long long)((unsigned long long)(long long)(mm * (gsx[t] - acct[t][q])) << sh);
                 acct[t][q] = 0;
               }
             }

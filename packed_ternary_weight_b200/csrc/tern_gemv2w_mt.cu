@@ -1,6 +1,7 @@
 // Launches of the one-CTA-per-SM decode GEMV for several tokens of one
-// problem (2..8 int8 tokens sharing one pass over the packed weights); the
-// kernel template is in tern_gemv2w_kernel.cuh.
+// problem (2..8 int8 tokens sharing one pass over the packed weights, padded
+// to 2, 4 or 8 with zero images); the kernel template is in
+// tern_gemv2w_kernel.cuh.
 #include "tern_gemv2w_kernel.cuh"
 
 namespace tern {
@@ -27,10 +28,15 @@ int launch_mt_fmt(const Gemv2wParams& p, bool pdl, void* stream) {
 
 int launch_gemv2w_mt(const Gemv2wParams& p, int xmode, bool pdl, void* stream) {
   if (p.bt3 || p.nprob != 1 || p.mt < 2 || p.mt > kMaxTokensW) return -1;
-  const bool four = p.mt <= 4;
-  if (xmode == kXInt8) return four ? launch_mt_fmt<kXInt8, 4>(p, pdl, stream) : launch_mt_fmt<kXInt8, 8>(p, pdl, stream);
-  if (xmode == kXBf16Q8)
-    return four ? launch_mt_fmt<kXBf16Q8, 4>(p, pdl, stream) : launch_mt_fmt<kXBf16Q8, 8>(p, pdl, stream);
+  const int mtp = gemv2w_mt_pad(p.mt);  // the kernel's token count (zero images beyond p.mt)
+  if (xmode == kXInt8) {
+    if (mtp == 2) return launch_mt_fmt<kXInt8, 2>(p, pdl, stream);
+    return mtp == 4 ? launch_mt_fmt<kXInt8, 4>(p, pdl, stream) : launch_mt_fmt<kXInt8, 8>(p, pdl, stream);
+  }
+  if (xmode == kXBf16Q8) {
+    if (mtp == 2) return launch_mt_fmt<kXBf16Q8, 2>(p, pdl, stream);
+    return mtp == 4 ? launch_mt_fmt<kXBf16Q8, 4>(p, pdl, stream) : launch_mt_fmt<kXBf16Q8, 8>(p, pdl, stream);
+  }
   return -1;
 }
 

@@ -50,6 +50,9 @@ constexpr int kMaxProblems = 32;   // independent GEMVs in one launch of the row
 constexpr int kMaxProblemsW = 256; // ... of the one-CTA-per-SM kernel (parameter block < 32 KB)
 constexpr int kMaxSlotsW = 16;     // problems one CTA of that kernel may touch
 constexpr int kMaxTokensW = 8;     // tokens of one problem per launch of that kernel
+// Activation images of a multi-token launch: the tokens padded to 2, 4 or 8
+// (the padding images are zero), so the kernel's token loops have no bounds.
+TERN_HD inline int gemv2w_mt_pad(int mt) { return mt <= 1 ? 1 : (mt <= 2 ? 2 : (mt <= 4 ? 4 : 8)); }
 constexpr int kMaxCluster = 16;   // K-splits reduced through one thread-block cluster
 
 struct Gemv2Problem {
