@@ -179,8 +179,10 @@ tern_status tern_gemm_batched(const tern_desc* desc, const void* d_packed, int32
  * and v projections of a decode step, or gate and up). The pages state one
  * GEMV per projection (QORA-LLM-2B, "SubLN Pattern"); running independent
  * ones together is a launch-level choice of this library.
- *   count       1..256 problems; descs[i] must share fmt, k, planes, group and
- *               flags (n may differ).
+ *   count       1..256 problems; descs[i] must share fmt, planes, group and
+ *               flags (n and k may differ; a launch with several k balances
+ *               its work by columns, and smaller launches run one kernel per
+ *               run of equal k).
  *   d_packed[i], d_x[i] ([K]), d_xscale[i] (TERN_ACT_INT8, else ignored and may
  *               be NULL), d_y[i] ([n_i]): as tern_gemv, one per problem.
  * Needs no workspace. Returns TERN_EUNSUPPORTED if K is too large to split

@@ -125,22 +125,29 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
 // the launch has at least four tiles per SM (smaller launches are spread
 // over the SMs by K splits in the row-group kernel).
 // With mt > 1 tokens (one problem, integer activations) a launch of half a
-// tile per SM is enough: each tile carries mt tokens' work.
+// tile per SM is enough: each tile carries mt tokens' work. L is the layout of
+// the widest problem (its K sizes the activation images); prob_cols gives
+// each problem's column count when K differs between problems (else NULL).
 bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, int sms, Gemv2wParams& p,
-                 int mt = 1) {
+                 int mt = 1, const int* prob_cols = nullptr) {
   const bool bt3 = L.fmt == TERN_FMT_BT3;
   if (bt3 && xmode != kXBf16) return false;
   if (nprob > kMaxProblemsW) return false;
   if (mt > 1 && (nprob != 1 || bt3 || xmode == kXBf16 || mt > kMaxTokensW)) return false;
   int begin[kMaxProblemsW + 1];
+  long long cbeg[kMaxProblemsW + 1];
   begin[0] = 0;
-  for (int i = 0; i < nprob; ++i) begin[i + 1] = begin[i] + row_tiles[i];
+  cbeg[0] = 0;
+  for (int i = 0; i < nprob; ++i) {
+    begin[i + 1] = begin[i] + row_tiles[i];
+    cbeg[i + 1] = cbeg[i] + (long long)row_tiles[i] * (prob_cols ? prob_cols[i] : L.cols);
+  }
   const int T = begin[nprob];
   if (T < (mt > 1 ? (sms + 1) / 2 : 4 * sms)) return false;
   p.mt = mt;
-  // the kernel's index arithmetic is 32-bit: tiles x CTAs and a CTA's
-  // columns x warps stay below 2^31
-  if ((long long)T * sms >= (1ll << 31) || ((long long)T / sms + 1) * L.cols * 16 >= (1ll << 31)) return false;
+  // the kernel's index arithmetic is 32-bit: all columns, and a CTA's columns
+  // x warps, stay below 2^31
+  if (cbeg[nprob] * 16 >= (1ll << 31) || (cbeg[nprob] / sms + L.cols) * 16 >= (1ll << 31)) return false;
   const bool tq = L.fmt == TERN_FMT_TQ;
   p.tq = tq;
   p.k = L.k;
@@ -153,15 +160,22 @@ bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, in
   p.nprob = nprob;
   p.tiles_total = T;
   p.grid = std::min(sms, T);
-  for (int i = 0; i <= nprob; ++i) p.tile_begin[i] = begin[i];
+  for (int i = 0; i <= nprob; ++i) {
+    p.tile_begin[i] = begin[i];
+    p.col_begin[i] = (int)cbeg[i];
+  }
   auto prob_of = [&](int t) {
     int q = 0;
     while (q + 1 < nprob && t >= begin[q + 1]) ++q;
     return q;
   };
+  // CTA tile ranges balance columns (the kernel computes the same ones); every
+  // CTA needs at least one tile
   int xs = 1;
   for (int c = 0; c < p.grid; ++c) {
-    const int t0 = (int)((long long)T * c / p.grid), t1 = (int)((long long)T * (c + 1) / p.grid);
+    const int t0 = gemv2w_cta_tile(p.tile_begin, p.col_begin, nprob, c, p.grid);
+    const int t1 = gemv2w_cta_tile(p.tile_begin, p.col_begin, nprob, c + 1, p.grid);
+    if (t1 <= t0) return false;
     xs = std::max(xs, prob_of(t1 - 1) - prob_of(t0) + 1);
   }
   if (xs > kMaxSlotsW) return false;
@@ -375,6 +389,9 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
       q.n = L.n;
       q.row_tiles = L.row_tiles;
       q.tensor_scale = desc->tensor_scale;
+      q.k = L.k;
+      q.cols = L.cols;
+      q.groups = L.groups;
       w.x_vec = aligned16(d_x) && L.k % 16 == 0;
       const int rc = launch_gemv2w(w, xmode, pdl, stream);
       if (rc >= 0) return rc == 0 ? TERN_OK : TERN_ECUDA;
@@ -404,6 +421,9 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
         q.n = L.n;
         q.row_tiles = L.row_tiles;
         q.tensor_scale = desc->tensor_scale;
+        q.k = L.k;
+        q.cols = L.cols;
+        q.groups = L.groups;
         w.x_vec = aligned16(q.x) && L.k % 16 == 0;
         const int rc = launch_gemv2w(w, xmode, pdl, stream);
         if (rc < 0 && c == 0) break;  // no kernel for this plane count and group size: the row-group kernel below
@@ -510,22 +530,31 @@ extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, 
     tern_status st = check_one(&descs[i], d_packed[i], act, d_x[i], d_xscale ? d_xscale[i] : nullptr, out, d_y[i],
                                &L[i]);
     if (st != TERN_OK) return st;
-    if (L[i].fmt != L[0].fmt || L[i].k != L[0].k || L[i].planes != L[0].planes || L[i].group != L[0].group ||
-        descs[i].flags != descs[0].flags)
+    // the group size matters for TQ only (BitNet: the whole row; d = 3: 16)
+    if (L[i].fmt != L[0].fmt || L[i].planes != L[0].planes ||
+        (L[0].fmt == TERN_FMT_TQ && L[i].group != L[0].group) || descs[i].flags != descs[0].flags)
       return TERN_EINVAL;
     rt[i] = L[i].row_tiles;
   }
   const int xmode = xmode_of(act);
-  tern_status st = supported_2bit(L[0], xmode);
-  if (st != TERN_OK) return st;
+  int widest = 0;  // the problem with the largest K sizes the activation images
+  bool all_vec = true;
+  for (int i = 0; i < count; ++i) {
+    tern_status st = supported_2bit(L[i], xmode);
+    if (st != TERN_OK) return st;
+    if (L[i].k > L[widest].k) widest = i;
+    all_vec = all_vec && L[i].k % 16 == 0;
+  }
   const int sms = device_sms();
   const bool pdl = (descs[0].flags & TERN_F_PDL) != 0;
   {
     static thread_local Gemv2wParams w;
     w = Gemv2wParams{};
-    if (plan_gemv2w(L[0], rt, count, xmode, sms, w)) {
+    int pcols[kMaxProblemsW];
+    for (int i = 0; i < count; ++i) pcols[i] = L[i].cols;
+    if (plan_gemv2w(L[widest], rt, count, xmode, sms, w, 1, pcols)) {
       w.out_bf16 = out == TERN_OUT_BF16;
-      bool vec = L[0].k % 16 == 0;
+      bool vec = all_vec;
       for (int i = 0; i < count; ++i) {
         const uint8_t* base = static_cast<const uint8_t*>(d_packed[i]);
         Gemv2wProblem& q = w.prob[i];
@@ -537,6 +566,9 @@ extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, 
         q.n = L[i].n;
         q.row_tiles = L[i].row_tiles;
         q.tensor_scale = descs[i].tensor_scale;
+        q.k = L[i].k;
+        q.cols = L[i].cols;
+        q.groups = L[i].groups;
         vec = vec && aligned16(q.x);
       }
       w.x_vec = vec;
@@ -545,16 +577,17 @@ extern "C" tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, 
       // no kernel for this plane count and group size: the row-group kernel below
     }
   }
-  // the row-group kernel takes up to kMaxProblems problems per launch
-  for (int c0 = 0; c0 < count; c0 += kMaxProblems) {
-    const int nc = std::min(kMaxProblems, count - c0);
+  // the row-group kernel takes up to kMaxProblems problems of one K per launch
+  for (int c0 = 0, nc = 0; c0 < count; c0 += nc) {
+    nc = 1;
+    while (c0 + nc < count && nc < kMaxProblems && L[c0 + nc].k == L[c0].k) ++nc;
     const Plan2 pl = plan_gemv2(L[c0], rt + c0, nc, 1, xmode, sms, false);
     if (!pl.ok) return TERN_EUNSUPPORTED;
     Gemv2Params p{};
     fill_common(p, L[c0], pl, 1, out);
     p.nprob = nc;
     int cta = 0;
-    bool vec = L[0].k % 16 == 0;
+    bool vec = L[c0].k % 16 == 0;
     for (int j = 0; j < nc; ++j) {
       const int i = c0 + j;
       const uint8_t* base = static_cast<const uint8_t*>(d_packed[i]);

@@ -9,8 +9,9 @@
 // Work split. The row tiles (32 rows) of all problems of the launch form one
 // list; CTA c takes the contiguous range [T*c/G, T*(c+1)/G) of it, so every SM
 // gets the same number of tiles to within one. Inside the CTA the columns of
-// that range (tiles x columns, in memory order) are split into equal
-// contiguous ranges, one per warp, in units of whole scale groups. A warp
+// that range (tiles x columns, in memory order; problems may differ in K, so
+// a tile has its own problem's column count) are split into equal contiguous
+// ranges, one per warp, in units of whole scale groups. A warp
 // therefore streams one contiguous stretch of each problem's packed bytes and
 // the warps of a CTA finish together to within one column. A tile that lies
 // inside one warp's range is finished by that warp; a tile cut by one or more
@@ -193,13 +194,15 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
   // the parameter space again. Only the members before `prob` are valid in
   // the shared copy; the problems live in `sprob`.
   constexpr int kHeadBytes = (int)offsetof(Gemv2wParams, prob);
-  static_assert(kHeadBytes % 4 == 0 && sizeof(Gemv2wProblem) % 4 == 0, "copied as 32-bit words");
+  // copied as 64-bit words: one word per thread covers the head in one round
+  static_assert(kHeadBytes % 8 == 0 && sizeof(Gemv2wProblem) % 8 == 0 && kHeadBytes <= 512 * 8,
+                "copied as 64-bit words, one round");
   __shared__ __align__(16) unsigned char shead[kHeadBytes];
   __shared__ __align__(16) Gemv2wProblem sprob[kMaxSlotsW];
   {
-    const int* src = reinterpret_cast<const int*>(&pg);
-    int* dst = reinterpret_cast<int*>(shead);
-    for (int i = threadIdx.x; i < kHeadBytes / 4; i += blockDim.x) dst[i] = src[i];
+    const long long* src = reinterpret_cast<const long long*>(&pg);
+    long long* dst = reinterpret_cast<long long*>(shead);
+    for (int i = threadIdx.x; i < kHeadBytes / 8; i += blockDim.x) dst[i] = src[i];
   }
   __syncthreads();
   const Gemv2wParams& p = *reinterpret_cast<const Gemv2wParams*>(shead);
@@ -211,15 +214,15 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
   constexpr int kColB = kB3 ? kBt3ColBytes : P * kPlaneColBytes;  // bytes per tile column
   const Plan2w sp = plan2w(p, XM);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nw = p.nw, nst = p.nstage, sc = p.stage_cols, cols = p.cols;
+  const int nw = p.nw, nst = p.nstage, sc = p.stage_cols;
 
   // ---- this CTA's tiles, and this warp's columns of them (32-bit arithmetic:
   // the planner keeps tiles x CTAs and columns x warps below 2^31). The tiles'
   // problem boundaries are searched in shared memory, and only the problems
   // of this CTA's tiles are copied there (slot s = problem qa + s).
   const int* stb = p.tile_begin;
-  const int t0 = (int)((unsigned)(p.tiles_total * blockIdx.x) / gridDim.x);
-  const int t1 = (int)((unsigned)(p.tiles_total * (blockIdx.x + 1)) / gridDim.x);
+  const int t0 = gemv2w_cta_tile(stb, p.col_begin, p.nprob, blockIdx.x, gridDim.x);
+  const int t1 = gemv2w_cta_tile(stb, p.col_begin, p.nprob, blockIdx.x + 1, gridDim.x);
   auto prob_of = [&](int t) {  // the last problem whose first tile is <= t
     int lo = 0, hi = p.nprob - 1;
     while (lo < hi) {
@@ -234,22 +237,48 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
   const int mt = MT > 1 ? p.mt : 1;
   const int nimg = MT > 1 ? MT : nslots;
   {  // slot s = problem qa + s
-    constexpr int kPw = (int)(sizeof(Gemv2wProblem) / 4);
-    const int* src = reinterpret_cast<const int*>(&pg.prob[qa]);
-    int* dst = reinterpret_cast<int*>(sprob);
+    constexpr int kPw = (int)(sizeof(Gemv2wProblem) / 8);
+    const long long* src = reinterpret_cast<const long long*>(&pg.prob[qa]);
+    long long* dst = reinterpret_cast<long long*>(sprob);
     for (int i = threadIdx.x; i < nslots * kPw; i += blockDim.x) dst[i] = src[i];
+  }
+  // the CTA's column space: slot s's tiles start at CTA tile stile[s] and CTA
+  // column scol[s]; every tile of a problem has that problem's column count
+  __shared__ int stile[kMaxSlotsW + 1], scol[kMaxSlotsW + 1];
+  if (threadIdx.x == 0) {
+    int c = 0;
+    for (int s = 0; s < nslots; ++s) {
+      const int ta = max(t0, stb[qa + s]), tb = min(t1, stb[qa + s + 1]);
+      stile[s] = ta - t0;
+      scol[s] = c;
+      c += (tb - ta) * sprob[s].cols;
+    }
+    stile[nslots] = t1 - t0;
+    scol[nslots] = c;
   }
   __syncthreads();
   const int gcols = p.gcols;
-  const int cg = (t1 - t0) * cols / gcols;  // granules in this CTA
+  const int cg = scol[nslots] / gcols;  // granules in this CTA
   auto bound = [&](int w) { return gcols * (cg * w / nw); };
   // the warp whose range holds column c (never an empty range)
   auto warp_of = [&](int c) {
     const int g = c / gcols;
     return min(nw - 1, ((g + 1) * nw + cg - 1) / cg - 1);
   };
+  // slot, CTA tile and column within the tile of CTA column c
+  auto locate = [&](int c, int& sl, int& r, int& cc) {
+    sl = 0;
+    while (sl + 1 < nslots && scol[sl + 1] <= c) ++sl;
+    const int ncol = sprob[sl].cols, d = c - scol[sl];
+    r = stile[sl] + d / ncol;
+    cc = d - (d / ncol) * ncol;
+  };
+  // first CTA column of CTA tile r of slot sl
+  auto tile_col = [&](int sl, int r) { return scol[sl] + (r - stile[sl]) * sprob[sl].cols; };
   const int ca = bound(warp), cb = bound(warp + 1);
-  const int q_ca = prob_of(t0 + ca / cols);  // problem of this warp's first column
+  int s_ca, r_ca, c_ca;
+  locate(ca, s_ca, r_ca, c_ca);
+  const int q_ca = qa + s_ca;  // problem of this warp's first column
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sp.bars) + warp * nst;
   uint8_t* ring = smem + sp.ring + (size_t)warp * nst * sp.stage_bytes;
@@ -269,11 +298,11 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
   const uint64_t pol = policy_evict_first();
 
   // ---- producer cursor (lane 0): next column of this warp's range to request
-  int pp = ca, rp = ca / cols, ccp = ca - (ca / cols) * cols, qp = q_ca, islot = 0, nissued = 0;
+  int pp = ca, rp = r_ca, ccp = c_ca, qp = q_ca, islot = 0, nissued = 0;
   auto issue_next = [&]() {
     if (pp >= cb) return;
-    const int ncols = min(sc, min(cols - ccp, cb - pp));
     const Gemv2wProblem& pq = sprob[qp - qa];
+    const int ncols = min(sc, min(pq.cols - ccp, cb - pp));
     const int T = t0 + rp - stb[qp];
     const int slot = islot;
     islot = islot + 1 == nst ? 0 : islot + 1;
@@ -283,19 +312,19 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
     int ga = 0;
     if constexpr (kTQ) {
       ga = ccp * kColK2 / p.group;
-      const int gb = min(p.groups, ((ccp + ncols) * kColK2 + p.group - 1) / p.group);
+      const int gb = min(pq.groups, ((ccp + ncols) * kColK2 + p.group - 1) / p.group);
       sb = (uint32_t)(gb - ga) * P * 64;
     }
     mbar_arrive_expect_tx(&bars[slot], tb + sb);
-    bulk_g2s(dst, pq.trit + ((size_t)T * cols + ccp) * kColB, tb, &bars[slot], pol);
+    bulk_g2s(dst, pq.trit + ((size_t)T * pq.cols + ccp) * kColB, tb, &bars[slot], pol);
     if constexpr (kTQ)
       bulk_g2s(dst + (size_t)sc * P * kPlaneColBytes,
-               reinterpret_cast<const uint8_t*>(pq.scale) + ((size_t)T * p.groups + ga) * P * 64, sb, &bars[slot],
+               reinterpret_cast<const uint8_t*>(pq.scale) + ((size_t)T * pq.groups + ga) * P * 64, sb, &bars[slot],
                pol);
     ++nissued;
     pp += ncols;
     ccp += ncols;
-    if (ccp == cols) {
+    if (ccp == pq.cols) {
       ccp = 0;
       ++rp;
       while (qp + 1 < p.nprob && t0 + rp >= stb[qp + 1]) ++qp;
@@ -312,22 +341,30 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
   // loads have returned: behind megabytes of outstanding bulk copies, a small
   // load waits for microseconds.
   pdl_wait();
+  // the widest image of this CTA's problems (images of narrower problems are
+  // staged to this width with zeros beyond their K)
+  int cmax = 0, gmax = 0;
+  for (int s = 0; s < nslots; ++s) {
+    cmax = max(cmax, sprob[s].cols);
+    gmax = max(gmax, sprob[s].groups);
+  }
   if constexpr (!kBf) {
     constexpr bool kQ8 = XM == kXBf16Q8;
     constexpr int kCk = kQ8 ? 8 : 16;  // activations per 16-byte chunk
-    const int nch = sp.kx / kCk;       // chunks per image
+    const int nch = cmax * kColK2 / kCk;  // chunks per image
     const int nflat = nimg * nch;
     const int nthr = blockDim.x;
     auto chunk_load = [&](int f) -> uint4 {
       const int s = f / nch, c = f - s * nch;
       if (MT > 1 && s >= mt) return make_uint4(0u, 0u, 0u, 0u);  // padding token
+      const int kq = sprob[MT > 1 ? 0 : s].k;
       const void* xp = MT > 1 ? static_cast<const void*>(static_cast<const int8_t*>(sprob[0].x) +
-                                                         (size_t)s * p.k * (kQ8 ? 2 : 1))
+                                                         (size_t)s * kq * (kQ8 ? 2 : 1))
                               : sprob[s].x;
       if constexpr (kQ8)
-        return load_bf16x8(static_cast<const uint16_t*>(xp), p.k, c * 8, p.x_vec);
+        return load_bf16x8(static_cast<const uint16_t*>(xp), kq, c * 8, p.x_vec);
       else
-        return load_s8x16(static_cast<const int8_t*>(xp), p.k, c * 16, p.x_vec);
+        return load_s8x16(static_cast<const int8_t*>(xp), kq, c * 16, p.x_vec);
     };
     uint4 xr[kXR];
 #pragma unroll
@@ -406,7 +443,7 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
     // sums of the image: per column (BitNet, then prefix sums) or per scale group (TQ)
     {
       const int span = kTQ ? p.group : kColK2;  // bytes summed per entry
-      const int nent = kTQ ? p.groups : cols;
+      const int nent = kTQ ? gmax : cmax;
       for (int e = threadIdx.x; e < nimg * nent; e += nthr) {
         const int s = e / nent, i = e - s * nent;
         uint8_t* sl = slot_ptr(s);
@@ -430,14 +467,15 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
           reinterpret_cast<float*>(sl + sp.sx_off)[threadIdx.x] =
               reinterpret_cast<const float*>(sprob[s].trit - kHeaderBytes + kCodebookOffset)[threadIdx.x];
       }
-      gemv_common::stage_x_bf16_chains(static_cast<const uint16_t*>(sprob[s].x), p.k, p.group, 0, sp.kx,
+      gemv_common::stage_x_bf16_chains(static_cast<const uint16_t*>(sprob[s].x), sprob[s].k, p.group, 0,
+                                       sprob[s].cols * (kB3 ? kColK3 : kColK2),
                                        reinterpret_cast<int8_t*>(sl), sl + sp.kx, sl + 2 * (size_t)sp.kx,
                                        reinterpret_cast<int4*>(sl + sp.sum_off));
     }
     __syncthreads();
   }
   if constexpr (!kTQ && !kB3) {  // single plane: column sums -> prefix sums
-    for (int s = warp; s < nimg; s += nw) prefix_columns(reinterpret_cast<int*>(slot_ptr(s) + sp.sum_off), cols);
+    for (int s = warp; s < nimg; s += nw) prefix_columns(reinterpret_cast<int*>(slot_ptr(s) + sp.sum_off), cmax);
     __syncthreads();
   }
 
@@ -520,13 +558,14 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
         v[t] = (long long)(pre[hi] - pre[lo] - acct[t][0]);
       }
     }
+    const int cols = pr.cols;
     if (lo == 0 && hi == cols) {
 #pragma unroll
       for (int t = 0; t < MT; ++t)
         if (t < mt) finish_t(pr, T, t, v[t]);
       return;
     }
-    const int base = r * cols;
+    const int base = tile_col(0, r);
     const int wlo = warp_of(base), whi = warp_of(base + cols - 1);
     int ncontrib = 0;
     for (int w = wlo; w <= whi; ++w) ncontrib += bound(w + 1) > bound(w);
@@ -563,12 +602,13 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
       const int* pre = reinterpret_cast<const int*>(sl + sp.sum_off);
       v = (long long)(pre[hi] - pre[lo] - fold_int(acc[0]));
     }
+    const int cols = pr.cols;
     if (lo == 0 && hi == cols) {
       finish(pr, T, v, vf, sl);
       return;
     }
     // a tile shared with other warps: partial row sums in warp order, added by the last to arrive
-    const int base = r * cols;
+    const int base = tile_col(q - qa, r);
     const int wlo = warp_of(base), whi = warp_of(base + cols - 1);
     int ncontrib = 0;
     for (int w = wlo; w <= whi; ++w) ncontrib += bound(w + 1) > bound(w);
@@ -597,13 +637,14 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
   };
 
   // ---- consumer: this warp's columns, stage by stage
-  int pc = ca, rc = ca / cols, ccc = ca - (ca / cols) * cols, qc = q_ca, cslot = 0;
+  int pc = ca, rc = r_ca, ccc = c_ca, qc = q_ca, cslot = 0;
+  int ccols = sprob[qc - qa].cols;  // columns of the current tile
   int seg_lo = ccc, ifail = -1, nconsumed = 0;
   uint32_t cphase = 0;
   reset();
   const uint32_t ring32 = smem_u32(ring) + lane * 16;
   while (pc < cb) {
-    const int ncols = min(sc, min(cols - ccc, cb - pc));
+    const int ncols = min(sc, min(ccols - ccc, cb - pc));
     const int slot = cslot;
     const uint32_t phase = cphase;
     if (++cslot == nst) {
@@ -839,7 +880,7 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
     ++nconsumed;
     pc += ncols;
     ccc += ncols;
-    if (ccc == cols || pc == cb) {
+    if (ccc == ccols || pc == cb) {
       if constexpr (MT > 1)
         segment_done_mt(rc, seg_lo, ccc);
       else
@@ -847,10 +888,11 @@ __global__ void __launch_bounds__(512, 1) gemv2w_kernel(const __grid_constant__ 
       reset();
       seg_lo = 0;
     }
-    if (ccc == cols) {
+    if (ccc == ccols) {
       ccc = 0;
       ++rc;
       while (qc + 1 < p.nprob && t0 + rc >= stb[qc + 1]) ++qc;
+      ccols = sprob[qc - qa].cols;
     }
   }
   if (ifail >= 0) {

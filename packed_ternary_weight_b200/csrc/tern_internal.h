@@ -101,6 +101,7 @@ struct Gemv2wProblem {
   void* y;                  // [n]
   int n, row_tiles;
   float tensor_scale;
+  int k, cols, groups;      // input width, its 64-k (80-k for d = 3) columns, scale groups
 };
 
 // Scalars first and the tiles' problem boundaries as one compact array, so
@@ -109,7 +110,7 @@ struct Gemv2wProblem {
 struct Gemv2wParams {
   int nprob, tiles_total;
   int grid;                 // CTAs (at most one per SM)
-  int tq, k, planes, group, groups, cols;
+  int tq, k, planes, group, groups, cols;  // k, groups, cols: the largest of the launch's problems
   int bt3;                  // balanced ternary d = 3 columns (80 k, 1632 bytes per tile column)
   int gcols;                // columns per granule of the warp ranges (a whole scale group)
   int out_bf16;
@@ -120,8 +121,27 @@ struct Gemv2wParams {
   int mt;                   // tokens of the (single) problem sharing the weight stream, or 1
   int early_w;              // set at launch: weights may be requested before the dependency wait
   int tile_begin[kMaxProblemsW + 1];  // first tile of each problem; [nprob] = tiles_total
+  int col_begin[kMaxProblemsW + 1];   // first column (tiles x columns) of each problem; [nprob] = total
   Gemv2wProblem prob[kMaxProblemsW];  // last member: the kernel copies only its own problems
 };
+
+// CTA c of G takes the tiles [gemv2w_cta_tile(c), gemv2w_cta_tile(c + 1)): the
+// first tile whose first column is at or after the c-th equal share of all
+// columns, so that CTAs get equal work when problems differ in K. Host and
+// device call the same function.
+TERN_HD inline int gemv2w_cta_tile(const int* tile_begin, const int* col_begin, int nprob, int c, int G) {
+  const long long ctot = col_begin[nprob];
+  const long long cg = ctot * c / G;
+  if (cg >= ctot) return tile_begin[nprob];
+  int lo = 0, hi = nprob - 1;  // the last problem whose first column is <= cg
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (col_begin[mid] <= cg) lo = mid; else hi = mid - 1;
+  }
+  const int ncol = (col_begin[lo + 1] - col_begin[lo]) / (tile_begin[lo + 1] - tile_begin[lo]);
+  const int d = (int)(cg - col_begin[lo]);
+  return tile_begin[lo] + (d + ncol - 1) / ncol;
+}
 
 // Batched GEMM on the tensor cores (tcgen05 kind::i8), m >= 16 tokens. The
 // fp16 group scale s of every (plane, row, group) is an integer u = |s| / 2^-24

@@ -183,3 +183,48 @@ def test_bt3_ragged_mix(tern):
     runs, _ = run_grouped(tern, layers, tern.ACT_BF16, reps=2)
     for a, b in zip(runs[0], runs[1]):
         assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+# ------------------------------------------------- problems of different K
+def test_bitnet_layer_set_one_launch(tern):
+    # the BitNet-2B layer set's shapes in one launch: q,k,v,o,gate,up (K = 2560)
+    # next to down (K = 6912); CTAs balance columns, images of both widths
+    shapes = [(2560, 2560), (640, 2560), (640, 2560), (2560, 2560), (6912, 2560), (6912, 2560), (2560, 6912)]
+    layers = [synth.bitnet_layer(n, k, 6100 + i) for i, (n, k) in enumerate(shapes * 4)]
+    layers.sort(key=lambda L: L.k)
+    check_int8_group(tern, layers, tern.ACT_BF16_Q8, nrows=512, flags=tern.F_PDL)
+    check_int8_group(tern, layers, tern.ACT_INT8, nrows=512)
+
+
+def test_mixed_k_interleaved_ragged(tern):
+    # K changes from problem to problem, ragged K (scalar loads), CTAs span
+    # problems of different widths
+    spec = [(9000, 1000), (70, 6912), (20000, 256), (33, 2560), (5000, 6912), (12000, 64), (3000, 4000)]
+    layers = [synth.bitnet_layer(n, k, 6200 + i) for i, (n, k) in enumerate(spec)]
+    check_int8_group(tern, layers, tern.ACT_INT8, nrows=1024)
+    check_int8_group(tern, layers, tern.ACT_BF16_Q8, nrows=1024)
+
+
+def test_mixed_k_tq_int8_and_bf16(tern):
+    spec = [(14336, 4096), (4096, 14336), (1024, 4096), (4096, 14336), (14336, 4096)]
+    layers = [synth.tq_layer(n, k, 3, 256, seed=6300 + i) for i, (n, k) in enumerate(spec)]
+    check_int8_group(tern, layers, tern.ACT_INT8, nrows=256)
+    (ys,), xbits = run_grouped(tern, layers, tern.ACT_BF16)
+    for i, (lay, y, x) in enumerate(zip(layers, ys, xbits)):
+        rows = sample_rows(lay.n, 128, i)
+        w = oracle.dequantize("tq", lay.trits[:, rows], lay.group, scales=lay.scales[:, rows])
+        check_bf16(y[rows], oracle.gemv_bf16(w, x)[0])
+
+
+def test_mixed_k_bt3(tern):
+    spec = [(9000, 4096), (4096, 14336), (30, 1040), (6000, 4096)]
+    layers = [synth.bt3_layer(n, k, seed=6400 + i) for i, (n, k) in enumerate(spec)]
+    (ys,), xbits = run_grouped(tern, layers, tern.ACT_BF16)
+    bt3_check(layers, ys, xbits, 256)
+
+
+def test_mixed_k_small_launch_runs_per_k(tern):
+    # too few tiles for the one-CTA-per-SM kernel: one row-group launch per run of equal K
+    spec = [(300, 1024), (200, 1024), (100, 2048), (64, 1024)]
+    layers = [synth.bitnet_layer(n, k, 6500 + i) for i, (n, k) in enumerate(spec)]
+    check_int8_group(tern, layers, tern.ACT_INT8, nrows=300)
