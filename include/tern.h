@@ -167,8 +167,10 @@ tern_status tern_gemv(const tern_desc* desc, const void* d_packed, tern_act act,
  * is given, and from m = 5 when the activations of a CUDA-core pass would
  * crowd shared memory (long K). Otherwise, with 2..15 tokens, the weights are
  * read once per pass of up to eight tokens on the CUDA cores; those kernels
- * cover BitNet, TQ{1..4}P with g = 256, TQ2P with g = 32 and TQ3P with g = 64
- * (TERN_EUNSUPPORTED for other plane and group combinations).
+ * cover BitNet, TQ{1..4}P with g = 256, TQ2P with g = 32 and TQ3P with g = 64;
+ * other plane and group combinations take the tensor path with a workspace
+ * (TERN_EUNSUPPORTED without one). One token: every TQ{1..4}P with
+ * g = 32, 64, 128, 256.
  */
 tern_status tern_gemm_batched(const tern_desc* desc, const void* d_packed, int32_t m, tern_act act,
                               const void* d_x, const float* d_xscale, tern_out out, void* d_y,

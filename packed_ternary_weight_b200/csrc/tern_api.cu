@@ -327,10 +327,14 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
   // CUDA-core pass's activation images leave room for fewer than 16 warps
   // (long K)
   bool use_tc = m >= 16 || (m >= 9 && d_ws);
-  if (!use_tc && m >= 5 && d_ws && xmode != kXBf16 && L.fmt != TERN_FMT_BT3) {
-    Gemv2wParams w{};
-    const int rt = L.row_tiles;
-    use_tc = plan_gemv2w(L, &rt, 1, xmode, sms, w, std::min(m, kMaxTokensW)) && w.nw < 16;
+  if (!use_tc && m >= 2 && d_ws && xmode != kXBf16 && L.fmt != TERN_FMT_BT3) {
+    if (!gemv2w_mt_has_kernel(L.planes, L.fmt == TERN_FMT_TQ, L.group)) {
+      use_tc = true;  // no CUDA-core kernel for several tokens of this plane count and group size
+    } else if (m >= 5) {
+      Gemv2wParams w{};
+      const int rt = L.row_tiles;
+      use_tc = plan_gemv2w(L, &rt, 1, xmode, sms, w, std::min(m, kMaxTokensW)) && w.nw < 16;
+    }
   }
   if (use_tc) {
     const int mb = std::min(m, kTcMaxTokens);

@@ -767,17 +767,27 @@ static int launch_one(const Gemv2Params& p, bool pdl, void* stream) {
 }
 
 // Instantiated combinations; anything else reports "unsupported" (-1).
-// Planes x group: TQ with 1-4 planes at g = 256 and the fine-group variants
-// of the workloads (2 planes at g = 32, 3 planes at g = 64); BitNet one plane.
-#define TERN_TQ_CASES(XM, MT)                                                    \
-  switch (p.planes * 100 + wg) {                                                \
-    case 116: return launch_one<XM, 1, 16, MT>(p, pdl, stream);                 \
-    case 216: return launch_one<XM, 2, 16, MT>(p, pdl, stream);                 \
-    case 316: return launch_one<XM, 3, 16, MT>(p, pdl, stream);                 \
-    case 416: return launch_one<XM, 4, 16, MT>(p, pdl, stream);                 \
-    case 202: return launch_one<XM, 2, 2, MT>(p, pdl, stream);                  \
-    case 304: return launch_one<XM, 3, 4, MT>(p, pdl, stream);                  \
-    default: return -1;                                                         \
+// Planes x group: TQ with 1-4 planes at g = 32, 64, 128 or 256 (sasori
+// README, "K and g"); BitNet one plane.
+#define TERN_TQ_CASES(XM, MT) \
+  switch (p.planes * 100 + wg) { \
+    case 102: return launch_one<XM, 1, 2, MT>(p, pdl, stream); \
+    case 104: return launch_one<XM, 1, 4, MT>(p, pdl, stream); \
+    case 108: return launch_one<XM, 1, 8, MT>(p, pdl, stream); \
+    case 116: return launch_one<XM, 1, 16, MT>(p, pdl, stream); \
+    case 202: return launch_one<XM, 2, 2, MT>(p, pdl, stream); \
+    case 204: return launch_one<XM, 2, 4, MT>(p, pdl, stream); \
+    case 208: return launch_one<XM, 2, 8, MT>(p, pdl, stream); \
+    case 216: return launch_one<XM, 2, 16, MT>(p, pdl, stream); \
+    case 302: return launch_one<XM, 3, 2, MT>(p, pdl, stream); \
+    case 304: return launch_one<XM, 3, 4, MT>(p, pdl, stream); \
+    case 308: return launch_one<XM, 3, 8, MT>(p, pdl, stream); \
+    case 316: return launch_one<XM, 3, 16, MT>(p, pdl, stream); \
+    case 402: return launch_one<XM, 4, 2, MT>(p, pdl, stream); \
+    case 404: return launch_one<XM, 4, 4, MT>(p, pdl, stream); \
+    case 408: return launch_one<XM, 4, 8, MT>(p, pdl, stream); \
+    case 416: return launch_one<XM, 4, 16, MT>(p, pdl, stream); \
+    default: return -1; \
   }
 
 int launch_gemv2(const Gemv2Params& p, int xmode, bool pdl, void* stream) {

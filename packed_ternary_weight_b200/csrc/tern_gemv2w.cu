@@ -8,15 +8,26 @@ int read_clear_dev_error_gemv2w(void* stream, unsigned* out) { return read_clear
 
 size_t gemv2w_smem_bytes(const Gemv2wParams& p, int xmode) { return plan2w(p, xmode).total; }
 
-#define TERN_W_TQ_CASES(XM)                                           \
-  switch (p.planes * 100 + wg) {                                      \
-    case 116: return launch_w<XM, 1, 16, 1>(p, pdl, stream);             \
-    case 216: return launch_w<XM, 2, 16, 1>(p, pdl, stream);             \
-    case 316: return launch_w<XM, 3, 16, 1>(p, pdl, stream);             \
-    case 416: return launch_w<XM, 4, 16, 1>(p, pdl, stream);             \
-    case 202: return launch_w<XM, 2, 2, 1>(p, pdl, stream);              \
-    case 304: return launch_w<XM, 3, 4, 1>(p, pdl, stream);              \
-    default: return -1;                                               \
+// TQ with 1-4 planes at g = 32, 64, 128 or 256 (sasori README, "K and g").
+#define TERN_W_TQ_CASES(XM) \
+  switch (p.planes * 100 + wg) { \
+    case 102: return launch_w<XM, 1, 2, 1>(p, pdl, stream); \
+    case 104: return launch_w<XM, 1, 4, 1>(p, pdl, stream); \
+    case 108: return launch_w<XM, 1, 8, 1>(p, pdl, stream); \
+    case 116: return launch_w<XM, 1, 16, 1>(p, pdl, stream); \
+    case 202: return launch_w<XM, 2, 2, 1>(p, pdl, stream); \
+    case 204: return launch_w<XM, 2, 4, 1>(p, pdl, stream); \
+    case 208: return launch_w<XM, 2, 8, 1>(p, pdl, stream); \
+    case 216: return launch_w<XM, 2, 16, 1>(p, pdl, stream); \
+    case 302: return launch_w<XM, 3, 2, 1>(p, pdl, stream); \
+    case 304: return launch_w<XM, 3, 4, 1>(p, pdl, stream); \
+    case 308: return launch_w<XM, 3, 8, 1>(p, pdl, stream); \
+    case 316: return launch_w<XM, 3, 16, 1>(p, pdl, stream); \
+    case 402: return launch_w<XM, 4, 2, 1>(p, pdl, stream); \
+    case 404: return launch_w<XM, 4, 4, 1>(p, pdl, stream); \
+    case 408: return launch_w<XM, 4, 8, 1>(p, pdl, stream); \
+    case 416: return launch_w<XM, 4, 16, 1>(p, pdl, stream); \
+    default: return -1; \
   }
 
 int launch_gemv2w(const Gemv2wParams& p, int xmode, bool pdl, void* stream) {

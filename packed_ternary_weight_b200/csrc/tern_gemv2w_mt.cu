@@ -26,6 +26,14 @@ int launch_mt_fmt(const Gemv2wParams& p, bool pdl, void* stream) {
 
 }  // namespace
 
+bool gemv2w_mt_has_kernel(int planes, int tq, int group) {
+  if (!tq) return planes == 1;
+  switch (planes * 100 + group / 16) {
+    case 116: case 216: case 316: case 416: case 202: case 304: return true;
+    default: return false;
+  }
+}
+
 int launch_gemv2w_mt(const Gemv2wParams& p, int xmode, bool pdl, void* stream) {
   if (p.bt3 || p.nprob != 1 || p.mt < 2 || p.mt > kMaxTokensW) return -1;
   const int mtp = gemv2w_mt_pad(p.mt);  // the kernel's token count (zero images beyond p.mt)

@@ -234,6 +234,7 @@ int read_clear_dev_error_gemm_tc(void* stream, unsigned* out);
 int launch_gemv2(const Gemv2Params& p, int xmode, bool pdl, void* stream);  // -1: no kernel
 int launch_gemv2w(const Gemv2wParams& p, int xmode, bool pdl, void* stream);  // -1: no kernel
 int launch_gemv2w_mt(const Gemv2wParams& p, int xmode, bool pdl, void* stream);  // p.mt > 1
+bool gemv2w_mt_has_kernel(int planes, int tq, int group);  // the plane / group combinations of launch_gemv2w_mt
 size_t gemv2w_smem_bytes(const Gemv2wParams& p, int xmode);
 int read_clear_dev_error_gemv2w(void* stream, unsigned* out);
 int read_clear_dev_error_gemv2w_mt(void* stream, unsigned* out);

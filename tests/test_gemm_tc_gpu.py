@@ -163,3 +163,10 @@ def test_deterministic_tc(tern):
     y1 = run(tern, lay, x, tern.ACT_INT8, repeat=False)
     y2 = run(tern, lay, x, tern.ACT_INT8, repeat=False)
     assert np.array_equal(y1.view(np.uint32), y2.view(np.uint32))
+
+
+@pytest.mark.parametrize("planes,group,m", [(2, 64, 4), (1, 128, 2), (4, 32, 7)])
+def test_few_tokens_without_cuda_core_kernel(tern, planes, group, m):
+    # plane counts and group sizes the several-token CUDA-core kernel is not built for: with a
+    # workspace they run on the tensor path, padded to 16 tokens
+    check(tern, synth.tq_layer(300, 1024, planes, group, seed=6700 + planes * 10 + group), m)

@@ -228,3 +228,15 @@ def test_mixed_k_small_launch_runs_per_k(tern):
     spec = [(300, 1024), (200, 1024), (100, 2048), (64, 1024)]
     layers = [synth.bitnet_layer(n, k, 6500 + i) for i, (n, k) in enumerate(spec)]
     check_int8_group(tern, layers, tern.ACT_INT8, nrows=300)
+
+
+@pytest.mark.parametrize("planes,group", [(1, 32), (1, 64), (2, 64), (2, 128), (3, 128), (4, 32), (4, 64)])
+def test_tq_plane_group_variants_grouped(tern, planes, group):
+    # the one-CTA-per-SM kernel for plane counts and group sizes beyond the pages' main configs
+    layers = [synth.tq_layer(5000, 1024, planes, group, seed=6600 + 10 * planes + group + i) for i in range(4)]
+    check_int8_group(tern, layers, tern.ACT_INT8, nrows=256)
+    (ys,), xbits = run_grouped(tern, layers, tern.ACT_BF16)
+    for i, (lay, y, x) in enumerate(zip(layers, ys, xbits)):
+        rows = sample_rows(lay.n, 128, i)
+        w = oracle.dequantize("tq", lay.trits[:, rows], lay.group, scales=lay.scales[:, rows])
+        check_bf16(y[rows], oracle.gemv_bf16(w, x)[0])

@@ -197,11 +197,20 @@ def test_tq3p_llama_shapes_bf16(tern, shape):
     tq_bf16_check(tern, lay, rows=rows)
 
 
-@pytest.mark.parametrize("planes,group", [(1, 256), (2, 256), (4, 256), (2, 32), (3, 64)])
+TQ_VARIANTS = [(p, g) for p in (1, 2, 3, 4) for g in (32, 64, 128, 256)]
+
+
+@pytest.mark.parametrize("planes,group", TQ_VARIANTS)
 def test_tq_bf16_variants(tern, planes, group):
+    # sasori's K = 1..4 planes at every group size it names (README, "K and g")
     lay = synth.tq_layer(200, 1024, planes, group, seed=planes * 100 + group)
     tq_bf16_check(tern, lay)
     tq_bf16_check(tern, lay, use_ws=False)
+
+
+@pytest.mark.parametrize("planes,group", TQ_VARIANTS)
+def test_tq_int8_variants(tern, planes, group):
+    tq_int8_check(tern, synth.tq_layer(200, 1024, planes, group, seed=planes * 100 + group + 1), 1)
 
 
 def test_tq_bf16_wide_dynamic_range(tern):
