@@ -199,7 +199,7 @@ bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, in
   return false;
 }
 
-// Plan of the tensor-core batched GEMM (m >= 16 int8 tokens, 2-bit formats)
+// Plan of the tensor-core batched GEMM (int8 tokens padded to 16, 2-bit formats)
 // for one launch of up to kTcMaxTokens tokens. The digit count D of the scales
 // is read by the kernel from the packed header, so the token passes and the
 // activation slot are sized here for every D the kernel may meet.

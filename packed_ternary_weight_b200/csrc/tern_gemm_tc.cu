@@ -1,6 +1,6 @@
 // Batched (prefill) packed ternary GEMM on the 5th-generation tensor cores:
 // Y[m][n] = sum_p sum_groups s[p][n][grp] * sum_{k in grp} t[p][n][k] * xq[m][k]
-// for m >= 16 int8 tokens, bit-identical to the exact integer rule of the
+// for int8 tokens (padded to a multiple of 16), bit-identical to the exact integer rule of the
 // int8 path (every fp16 scale is an integer multiple of 2^-24, so the sum is an
 // exact integer count of 2^-24, rounded once to fp32, then times the token's
 // activation scale). Formats: sasori-style additive TQ{K}P planes with fp16

@@ -143,7 +143,9 @@ TERN_HD inline int gemv2w_cta_tile(const int* tile_begin, const int* col_begin, 
   return tile_begin[lo] + (d + ncol - 1) / ncol;
 }
 
-// Batched GEMM on the tensor cores (tcgen05 kind::i8), m >= 16 tokens. The
+// Batched GEMM on the tensor cores (tcgen05 kind::i8): tokens padded to a
+// multiple of 16 (the host routes here from 16 tokens, or from 9 when the
+// caller gives a workspace). The
 // fp16 group scale s of every (plane, row, group) is an integer u = |s| / 2^-24
 // written in D' digits of b bits (b = 7, 6, 5 for one, two, three or four
 // planes); the A operand of digit d holds sum_p sign(s_p) * t_p * u_{p,d}
