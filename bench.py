@@ -134,6 +134,23 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------ rank plumbing
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank calls this, in the same order."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_gbs(step_bytes: float, ms_step: float, world: int) -> float:
+    """Whole-job throughput of N replicas: every rank's bytes over the slowest rank's time."""
+    return world * step_bytes / (ms_step * 1e-3) / 1e9
+
+
 # --------------------------------------------------------------- our impl
 STAGES = (("q_proj", "k_proj", "v_proj"), ("o_proj",), ("gate_proj", "up_proj"), ("down_proj",))
 
@@ -277,11 +294,8 @@ def run_ours(args, rank, world):
                 graph.replay()
             e1.record(stream)
             torch.cuda.synchronize()
-            ms = e0.elapsed_time(e1)
+            ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
             if world > 1:
-                t = torch.tensor([ms], device=dev)
-                dist.all_reduce(t, op=dist.ReduceOp.MAX)
-                ms = float(t.item())
                 dist.barrier()
         return ms
 
@@ -341,13 +355,10 @@ def run_ours(args, rank, world):
         e1.record(stream)
         torch.cuda.synchronize()
         ms_e2e = e0.elapsed_time(e1) / reps
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(ms_e2e, world, dev)
     assert tern.device_error(stream) == tern.OK
 
-    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    value = replica_gbs(step_bytes, ms_step, world)
     achieved = step_bytes / (ms_step * 1e-3) / 1e9     # every launch of the step is the GEMV kernel
     out = {
         "metric": METRIC,
@@ -384,7 +395,7 @@ def run_ours(args, rank, world):
                                   "one (programmatic dependent launch: weights prefetched before the wait)",
                          "ms_per_step": round(ms_chain_step, 4),
                          "gbs": round(step_bytes / (ms_chain_step * 1e-3) / 1e9, 1)},
-        "e2e": {"value": round(world * step_bytes / (ms_e2e * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "e2e": {"value": round(replica_gbs(step_bytes, ms_e2e, world), 1), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * len(step_launches),
         "parity_first_gemv_bit_exact": parity,
