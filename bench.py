@@ -395,6 +395,11 @@ def run_ours(args, rank, world):
                                   "one (programmatic dependent launch: weights prefetched before the wait)",
                          "ms_per_step": round(ms_chain_step, 4),
                          "gbs": round(step_bytes / (ms_chain_step * 1e-3) / 1e9, 1)},
+        "tokens_per_s_equiv": {"independent": round(world * 1e3 / ms_step, 1),
+                               "decode_chain": round(world * 1e3 / ms_chain_step, 1),
+                               "basis": "a step's GEMVs are the projection layers one decoded token at batch 1 "
+                                        "streams (attention, norms and the output head are not on this path); "
+                                        "tokens per second = steps per second, summed over replicas"},
         "e2e": {"value": round(replica_gbs(step_bytes, ms_e2e, world), 1), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * len(step_launches),
