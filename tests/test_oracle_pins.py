@@ -330,3 +330,45 @@ def test_bt3_reduces_to_one_plane():
     w = oracle.dequantize("bt3", t, 16, idx=idx, codebook=cb)
     sc = cb[idx].astype(np.float64)
     assert np.array_equal(w, np.repeat(sc, 16, axis=1) * t[0])
+
+
+# ------------------------------------------------------------ bf16 rounding
+def _rn_bf16(fr: Fraction) -> Fraction:
+    """Nearest bf16 value of an exact rational (8 significant bits, ties to even, fp32 exponent range)."""
+    if fr == 0:
+        return Fraction(0)
+    sign = -1 if fr < 0 else 1
+    a = abs(fr)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    e = max(e, -126)
+    quantum = Fraction(2) ** (e - 7)
+    q = a / quantum
+    fl = q.numerator // q.denominator
+    rem = q - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return sign * fl * quantum
+
+
+def test_round_bf16_vs_exact_rationals_and_ties():
+    g = np.random.default_rng(71)
+    v = (g.standard_normal(400) * 10.0 ** g.uniform(-30, 30, 400)).astype(np.float32)
+    # exact ties between two bf16 neighbours: 1 + 2^-8 (to even: 1), 1 + 3 * 2^-8 (to even: 1 + 2^-6)
+    ties = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 2.0 ** -126 * (1 + 2 ** -8)], np.float32)
+    v = np.concatenate([v, ties, np.float32([0.0, -0.0, 1.0, 3.0e38])])
+    got = oracle.round_bf16(v)
+    for a, b in zip(v, got):
+        assert Fraction(float(b)) == _rn_bf16(Fraction(float(a))), a
+    assert got[400] == 1.0 and got[401] == 1 + 2 ** -6 and got[402] == -1.0
+
+
+def test_round_bf16_matches_torch_cast():
+    torch = pytest.importorskip("torch")
+    g = np.random.default_rng(72)
+    v = (g.standard_normal(5000) * 10.0 ** g.uniform(-35, 35, 5000)).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.round_bf16(v), ref)
