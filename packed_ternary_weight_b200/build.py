@@ -32,8 +32,6 @@ def _compile(src: str, ptxas_verbose: bool) -> str:
     cmd = [NVCC, *ARCH, *COMMON, "-c", src, "-o", obj]
     if ptxas_verbose and src.endswith(".cu"):
         cmd += ["-Xptxas", "-v"]
-    if src.endswith(".cpp"):
-        cmd += ["-x", "cu"] if False else []
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
