@@ -231,3 +231,18 @@ def test_workspace_size_host_only():
     d = tern.make_desc("bitnet", 640, 2560, 1, 2560, 0.02)
     assert tern.workspace_size(d, 1) >= 0
     assert tern.workspace_size(tern.make_desc("tq", 1024, 4096, 2, 32), 16) > 0
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    # the binding copied where no libtern.so sits beside it: importing it must
+    # raise (there is no CPU fallback to drop to)
+    import importlib.util
+    import shutil
+    src = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                       "packed_ternary_weight_b200", "tern.py")
+    dst = tmp_path / "tern_nolib.py"
+    shutil.copy(src, dst)
+    spec = importlib.util.spec_from_file_location("tern_nolib", dst)
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError, match="libtern.so not built"):
+        spec.loader.exec_module(mod)
