@@ -561,9 +561,36 @@ def run_ceiling(args):
             "best": max(r["gbs"] for r in rows)}
 
 
+def code_hash(path: str) -> str:
+    """First 16 hex digits of the SHA-256 of a C++/CUDA source with its comments removed and its
+    whitespace collapsed: edits to comments alone keep the hash, any change to the code changes it."""
+    src = open(path, encoding="utf-8").read()
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":                                    # string or character literal, kept whole
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    code = " ".join("".join(out).split())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
+
+
 def committed_traffic():
     """DRAM bytes (read + written) per launch of the step from a committed ncu summary, if the summary
-    was taken on the current kernel source (else None)."""
+    was taken on the current kernel code (else None)."""
     p = os.path.join(ROOT, "profiles", "gemv2w_bitnet2b_step_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -574,8 +601,7 @@ def committed_traffic():
                 key, val = line.split(":", 1)
                 vals[key.strip()] = val.strip()
     src = os.path.join(ROOT, "packed_ternary_weight_b200", "csrc", "tern_gemv2w_kernel.cuh")
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if vals.get("kernel_source_sha256_16") != h:
+    if vals.get("kernel_code_sha256_16") != code_hash(src):
         return None
     try:
         return float(vals["dram_bytes_per_launch"])

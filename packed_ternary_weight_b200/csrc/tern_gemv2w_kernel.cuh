@@ -7,11 +7,13 @@
 // TQ{K}P planes with fp16 group scales).
 //
 // Work split. The row tiles (32 rows) of all problems of the launch form one
-// list; CTA c takes the contiguous range [T*c/G, T*(c+1)/G) of it, so every SM
-// gets the same number of tiles to within one. Inside the CTA the columns of
-// that range (tiles x columns, in memory order; problems may differ in K, so
-// a tile has its own problem's column count) are split into equal contiguous
-// ranges, one per warp, in units of whole scale groups. A warp
+// list; CTA c takes a contiguous range of it that starts at the first tile
+// whose first column is at or after the c-th equal share of all columns
+// (gemv2w_cta_tile), so that every SM gets the same number of columns to
+// within one tile when problems differ in K. Inside the CTA the columns of
+// that range (tiles x columns, in memory order; a tile has its own problem's
+// column count) are split into equal contiguous ranges, one per warp, in units
+// of whole scale groups. A warp
 // therefore streams one contiguous stretch of each problem's packed bytes and
 // the warps of a CTA finish together to within one column. A tile that lies
 // inside one warp's range is finished by that warp; a tile cut by one or more

@@ -1,0 +1,37 @@
+"""The key that ties the committed DRAM-traffic summary to the kernel it was
+captured on: comment edits keep it, code edits change it (CPU only)."""
+import bench
+
+
+def _hash(tmp_path, text):
+    p = tmp_path / "k.cuh"
+    p.write_text(text)
+    return bench.code_hash(str(p))
+
+
+BASE = '''// a kernel
+__device__ int f(int x) {  /* body */
+  asm volatile("mov.u32 %0, %1; // not a comment" : "=r"(x) : "r"(x));
+  return x + 1;   // increment
+}
+'''
+
+
+def test_comment_edits_keep_the_key(tmp_path):
+    a = _hash(tmp_path, BASE)
+    b = _hash(tmp_path, BASE.replace("// a kernel", "// the kernel, reworded\n// over two lines")
+              .replace("/* body */", "/* a\n   longer body comment */").replace("// increment", ""))
+    assert a == b
+
+
+def test_code_edits_change_the_key(tmp_path):
+    a = _hash(tmp_path, BASE)
+    assert _hash(tmp_path, BASE.replace("x + 1", "x + 2")) != a
+    # text inside a string literal is code, even when it looks like a comment
+    assert _hash(tmp_path, BASE.replace("// not a comment", "// changed")) != a
+    assert _hash(tmp_path, BASE.replace("return x", "return  x")) == a       # whitespace only
+
+
+def test_committed_summary_parses():
+    v = bench.committed_traffic()
+    assert v is None or v > 0
