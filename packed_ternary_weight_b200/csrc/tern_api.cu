@@ -119,9 +119,10 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
   return pl;
 }
 
-// Plan of the single-token kernel with one CTA per SM (gemv2w): equal tile
-// ranges per CTA, about 6 KB stages, as many warps and stages in flight as
-// shared memory allows next to the resident activation images. Applies when
+// Plan of the single-token kernel with one CTA per SM (gemv2w): tile ranges
+// of equal column counts per CTA (gemv2w_cta_tile), about 6 KB stages, as
+// many warps and stages in flight as shared memory allows next to the
+// resident activation images. Applies when
 // the launch has at least four tiles per SM (smaller launches are spread
 // over the SMs by K splits in the row-group kernel).
 // With mt > 1 tokens (one problem, integer activations) a launch of half a
