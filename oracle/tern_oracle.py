@@ -11,8 +11,9 @@ What it computes, with the passage each step follows:
   layout, W = s_w * t with one per-tensor scale (QORA-LLM-2B, "Ternary GEMV
   (No Multiplication)"); for balanced ternary of depth 3,
   W = cb[idx] * (9 t2 + 3 t1 + t0), 27 levels, group 16, 27-entry log-spaced
-  codebook (Entrit Llama-3.1-8B-trit-uniform-d3 card, "Quantization details").
-  All exact in fp64.
+  codebook (Entrit Llama-3.1-8B-trit-uniform-d3 card, "Quantization details");
+  depth d in general (the card's d = 3; 2 and 4 by the same positional rule):
+  W = cb[idx] * sum_j 3^j t_j, 3^d levels. All exact in fp64.
 * ``gemv_bf16`` -- y = W x in fp64 for bf16 activations (dequantise then
   matmul: the fake-quant reference the sasori kernel is said to reproduce,
   sasori README, "g (group-size)").
@@ -109,8 +110,11 @@ def dequantize(fmt: str, trits: np.ndarray, group: int = 0, tensor_scale: float 
             w += np.repeat(s[p], group, axis=1) * t[p]
         return w
     if fmt == "bt3":
+        # depth d = number of trit planes: level = sum_j 3^j t_j (d = 3: -13 .. 13)
         cb = np.asarray(codebook, dtype=np.float32).astype(np.float64)
-        level = 9 * t[2] + 3 * t[1] + t[0]                 # -13 .. 13
+        level = np.zeros((n, k), dtype=np.int64)
+        for j in range(t.shape[0]):
+            level += 3 ** j * t[j]
         sc = cb[np.asarray(idx, dtype=np.int64)]           # [N][K/16]
         return np.repeat(sc, 16, axis=1) * level
     raise ValueError(fmt)
@@ -179,14 +183,15 @@ def bits_per_weight(fmt: str, planes: int = 1, group: int = 256) -> float:
     """Bits per weight of the formats' logical content.
 
     TQ{K}P: K planes of 2-bit trits plus one fp16 scale per group of g per plane
-    (sasori README, "K and g" table): K * (2 + 16 / g).
+    (sasori README, "K and g" table): K * (2 + 16 / g). Balanced ternary: the
+    information content at depth d = ``planes`` (see ``bt3_information_bpw``).
     """
     if fmt == "tq":
         return planes * (2.0 + 16.0 / group)
     if fmt == "bitnet":
         return 2.0
     if fmt == "bt3":
-        return bt3_information_bpw()
+        return bt3_information_bpw(depth=planes)
     raise ValueError(fmt)
 
 

@@ -372,3 +372,60 @@ def test_round_bf16_matches_torch_cast():
     v = (g.standard_normal(5000) * 10.0 ** g.uniform(-35, 35, 5000)).astype(np.float32)
     ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
     assert np.array_equal(oracle.round_bf16(v), ref)
+
+
+# ------------------------------------------- balanced ternary of depth d
+def _all_tuples(d):
+    """Every trit tuple of depth d as planes [d][1][3^d] (t_j of tuple i is base-3 digit j of i, minus 1)."""
+    i = np.arange(3 ** d)
+    return np.stack([((i // 3 ** j) % 3 - 1) for j in range(d)])[:, None, :].astype(np.int8)
+
+
+@pytest.mark.parametrize("d", [2, 3, 4])
+def test_bt_levels_are_a_bijection_onto_the_balanced_range(d):
+    # 3^d tuples -> 3^d distinct integer levels -(3^d - 1)/2 .. (3^d - 1)/2 (balanced ternary)
+    t = _all_tuples(d)
+    k = -(-3 ** d // 16) * 16
+    t = np.concatenate([t, np.zeros((d, 1, k - 3 ** d), np.int8)], axis=2)
+    w = oracle.dequantize("bt3", t, 16, idx=np.zeros((1, k // 16), np.uint8), codebook=np.ones(27, np.float32))
+    half = (3 ** d - 1) // 2
+    assert sorted(w[0, :3 ** d].astype(int).tolist()) == list(range(-half, half + 1))
+
+
+@pytest.mark.parametrize("d", [2, 4])
+def test_bt_depth_brute_force_loops(d):
+    g = np.random.default_rng(80 + d)
+    n, k = 3, 48
+    t = g.integers(-1, 2, size=(d, n, k)).astype(np.int8)
+    idx = g.integers(0, 27, size=(n, k // 16)).astype(np.uint8)
+    cb = synth.codebook27()
+    w = oracle.dequantize("bt3", t, 16, idx=idx, codebook=cb)
+    for r in range(n):
+        for c in range(k):
+            lvl = 0
+            for j in range(d):            # Horner from the most significant trit
+                lvl = 3 * lvl + int(t[d - 1 - j, r, c])
+            assert Fraction(w[r, c]) == Fraction(float(cb[idx[r, c // 16]])) * lvl
+
+
+def test_bt_depths_nest():
+    # a zero top trit reduces depth d + 1 to depth d
+    g = np.random.default_rng(90)
+    n, k = 4, 32
+    t = synth.draw_trits(g, (4, n, k))
+    idx = g.integers(0, 27, size=(n, k // 16)).astype(np.uint8)
+    cb = synth.codebook27()
+    for d in (2, 3):
+        top = t[:d + 1].copy()
+        top[d] = 0
+        assert np.array_equal(oracle.dequantize("bt3", top, 16, idx=idx, codebook=cb),
+                              oracle.dequantize("bt3", t[:d], 16, idx=idx, codebook=cb))
+
+
+def test_bt_bpw_steps_by_one_trit_from_the_printed_d3():
+    printed = load("bpw_pages.json")["bt3"]
+    b3 = oracle.bits_per_weight("bt3", 3)
+    assert round(b3, printed["digits"]) == pytest.approx(printed["printed"])
+    # each level of depth adds one trit (log2 3 bits) per weight; the codebook index is unchanged
+    assert oracle.bits_per_weight("bt3", 4) - b3 == pytest.approx(math.log2(3))
+    assert b3 - oracle.bits_per_weight("bt3", 2) == pytest.approx(math.log2(3))
