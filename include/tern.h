@@ -14,11 +14,14 @@
  *                    plane per group of g weights along the input dimension
  *                    (sasori README, "K and g - the quality dials" and
  *                    "How it works");
- *   TERN_FMT_BT3     balanced ternary of depth 3 (27 levels): weight =
- *                    cb[idx] * (9 t2 + 3 t1 + t0), trits base-3 packed five
- *                    per byte, group 16, 27-entry log-spaced scale codebook
- *                    with the index stored as three trits (Entrit
- *                    Llama-3.1-8B-trit-uniform-d3 card, "Quantization details").
+ *   TERN_FMT_BT3     balanced ternary of depth d (3^d levels): weight =
+ *                    cb[idx] * sum_j 3^j t_j (d = 3: 9 t2 + 3 t1 + t0, 27
+ *                    levels), trits base-3 packed five per byte, group 16,
+ *                    27-entry log-spaced scale codebook with the index stored
+ *                    as three trits (Entrit Llama-3.1-8B-trit-uniform-d3
+ *                    card, "Quantization details", d = 3; depths 2 and 4 by
+ *                    the same rule are packed, and the GEMV calls refuse them
+ *                    with TERN_EUNSUPPORTED).
  *
  * Conventions for every call:
  *   - All pointers named d_* are device pointers; the others are host
@@ -85,7 +88,8 @@ typedef struct tern_desc {
   int32_t fmt;          /* tern_format */
   int32_t n;            /* output rows N >= 1 */
   int32_t k;            /* input columns K >= 1 */
-  int32_t planes;       /* BITNET: 1; TQ: 1..4; BT3: 3 (the depth) */
+  int32_t planes;       /* BITNET: 1; TQ: 1..4; BT3: the depth d, 2..4 (GEMV
+                           kernels: 3) */
   int32_t group;        /* BITNET: ignored (whole row); TQ: g, a multiple of 16
                            in {16,32,64,128,256} dividing K; BT3: 16 */
   float tensor_scale;   /* BITNET: the per-tensor scale s_w; else ignored */
@@ -101,7 +105,7 @@ tern_status tern_packed_size(const tern_desc* desc, size_t* bytes);
 /*
  * Pack logical weights into the library's layout (host only, no device work).
  *   trits       int8 [planes][N][K], values -1, 0, +1 (TERN_EFORMAT otherwise).
- *               BT3: plane p holds t_p, the trit of weight 3^p.
+ *               BT3: plane p holds t_p, the trit of weight 3^p (p < d).
  *   scales_fp16 TQ: fp16 bit patterns [planes][N][K/group], finite; else NULL.
  *   scale_idx   BT3: uint8 [N][K/16], values 0..26 (codebook index); else NULL.
  *   codebook    BT3: float [27], finite; stored in the header; else NULL.

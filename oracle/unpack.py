@@ -8,7 +8,8 @@ benchmark's CPU baseline can start from the same bytes the GPU reads.
 Format (all little-endian):
 
 * 256-byte header: u32 magic 0x4E524554, u32 version 2, u32 fmt (1 BitNet,
-  2 TQ, 3 balanced ternary d=3), u32 N, u32 K, u32 planes, u32 group,
+  2 TQ, 3 balanced ternary), u32 N, u32 K, u32 planes (balanced ternary: the
+  depth d), u32 group,
   f32 tensor scale, u32 row tiles ceil(N/32), u32 columns, u64 trit offset,
   u64 trit bytes, u64 scale offset, u64 scale bytes; at byte 72 u32 "scale
   digits": TQ, the number of base-128 digits of the largest |s| / 2^-24 over
@@ -22,17 +23,20 @@ Format (all little-endian):
   row n = 32T + r. Padding rows and columns hold code 00.
 * TQ scales: fp16 scale of (T, group G, plane p, row r) at
   scale_offset + ((T*groups + G)*P + p)*64 + 2*r.
-* Balanced ternary d = 3: a column is 80 consecutive k of a 32-row tile, 1632
-  bytes at trit_offset + (T*cols + c)*1632. Its first 1536 bytes hold, per row
-  r, 16 byte triples: byte b (0..2) of triple i at b*512 + 16*r + i. Every byte
-  holds five base-3 digits u = t + 1 (first digit least significant); the 15
-  digits of triple i, byte 0 first, are the trits t0, t1, t2 (weights 1, 3, 9)
-  of k = 80c + i, then of k = 80c + 16 + i, ..., then of k = 80c + 64 + i
-  (weight j of the triple, j = 0..4, is k = 80c + 16j + i). The last 96 bytes hold the
-  scale indices of the column's five groups of 16 as one more triple per row:
-  byte b (0..2) of row r at 1536 + 32*b + r, five base-3 digits each; digit
-  3j + q of the triple (byte 0 first) is base-3 digit q of the index of group
-  5c + j. Padding trits are 0 (digit 1), padding indices 0.
+* Balanced ternary of depth d (2, 3 or 4; the Entrit card's d = 3): a column
+  is 80 consecutive k of a 32-row tile, 512*d + 96 bytes at
+  trit_offset + (T*cols + c)*(512*d + 96). Its first 512*d bytes hold, per
+  row r, 16 byte tuples of d bytes: byte b (0..d-1) of tuple i at
+  b*512 + 16*r + i. Every byte holds five base-3 digits u = t + 1 (first
+  digit least significant); the 5d digits of tuple i, byte 0 first, are the
+  trits t0 .. t(d-1) (weights 1, 3, 9, 27) of k = 80c + i, then of
+  k = 80c + 16 + i, ..., then of k = 80c + 64 + i (weight j of the tuple,
+  j = 0..4, is k = 80c + 16j + i; its trit p is digit d*j + p). The last 96
+  bytes hold the scale indices of the column's five groups of 16 as one
+  triple per row: byte b (0..2) of row r at 512*d + 32*b + r, five base-3
+  digits each; digit 3j + q of the triple (byte 0 first) is base-3 digit q
+  of the index of group 5c + j. Padding trits are 0 (digit 1), padding
+  indices 0.
 """
 from __future__ import annotations
 
@@ -103,17 +107,17 @@ def _base3_digits(byte: np.ndarray) -> np.ndarray:
 
 
 def _unpack_bt3(buf: np.ndarray, h: dict):
-    n, k, T, C = h["n"], h["k"], h["row_tiles"], h["cols"]
+    n, k, T, C, d = h["n"], h["k"], h["row_tiles"], h["cols"], h["planes"]
     raw = np.asarray(buf, dtype=np.uint8)[h["trit_offset"]:h["trit_offset"] + h["trit_bytes"]]
-    col = raw.reshape(T, C, 1632)
-    tri = col[:, :, :1536].reshape(T, C, 3, 32, 16)               # [T][c][b][r][i]
-    dig = _base3_digits(tri)                                      # [T][c][b][r][i][q]
-    # digit s = 5b + q of the triple; trit p of weight j is digit 3j + p
-    dig = dig.transpose(0, 1, 3, 4, 2, 5).reshape(T, C, 32, 16, 5, 3)  # [T][c][r][i][j][p]
+    col = raw.reshape(T, C, 512 * d + 96)
+    tup = col[:, :, :512 * d].reshape(T, C, d, 32, 16)            # [T][c][b][r][i]
+    dig = _base3_digits(tup)                                      # [T][c][b][r][i][q]
+    # digit s = 5b + q of the tuple; trit p of weight j is digit d*j + p
+    dig = dig.transpose(0, 1, 3, 4, 2, 5).reshape(T, C, 32, 16, 5, d)  # [T][c][r][i][j][p]
     t = (dig - 1).astype(np.int8)
     # k = 80c + 16j + i
-    t = t.transpose(5, 0, 2, 1, 4, 3).reshape(3, T * 32, C * 80)
-    ib = col[:, :, 1536:].reshape(T, C, 3, 32)                   # [T][c][b][r]
+    t = t.transpose(5, 0, 2, 1, 4, 3).reshape(d, T * 32, C * 80)
+    ib = col[:, :, 512 * d:].reshape(T, C, 3, 32)                 # [T][c][b][r]
     idig = _base3_digits(ib)                                      # [T][c][b][r][q]
     idig = idig.transpose(0, 1, 3, 2, 4).reshape(T, C, 32, 5, 3)  # [T][c][r][j][digit]
     idx = idig[..., 0] + 3 * idig[..., 1] + 9 * idig[..., 2]      # [T][c][r][j]

@@ -287,7 +287,8 @@ tern_status check_one(const tern_desc* desc, const void* d_packed, tern_act act,
 // What the kernels support for this layout and activation mode.
 tern_status supported_2bit(const Layout& L, int xmode) {
   const bool tq = L.fmt == TERN_FMT_TQ;
-  if (L.fmt == TERN_FMT_BT3) return xmode == kXBf16 ? TERN_OK : TERN_EUNSUPPORTED;
+  // balanced ternary: the kernels take depth 3 with bf16 activations (depths 2 and 4 are packed only)
+  if (L.fmt == TERN_FMT_BT3) return xmode == kXBf16 && L.planes == 3 ? TERN_OK : TERN_EUNSUPPORTED;
   if (xmode == kXBf16 && !tq) return TERN_EUNSUPPORTED;
   if (tq && L.k % kColK2 != 0) return TERN_EUNSUPPORTED;
   if (!tq && (long long)L.k * 127 >= (1ll << 24)) return TERN_EUNSUPPORTED;  // exact int32 -> fp32

@@ -27,7 +27,9 @@ constexpr int kColK2 = 64;          // k per 16-byte chunk, 2-bit planes
 constexpr int kColK3 = 80;          // k per 16-byte chunk, base-3 planes
 constexpr int kChunkBytes = 16;
 constexpr int kPlaneColBytes = kTileRows * kChunkBytes;   // 512
-constexpr int kBt3ColBytes = 3 * kPlaneColBytes + 3 * kTileRows;  // 1632
+// balanced ternary of depth d: d base-3 bytes per 5 weights of a row, then the group-index triple
+constexpr int bt_col_bytes(int d) { return d * kPlaneColBytes + 3 * kTileRows; }
+constexpr int kBt3ColBytes = bt_col_bytes(3);  // 1632: d = 3, the depth the kernels take
 constexpr int kBt3Groups = 5;       // groups of 16 per base-3 column
 
 struct Layout {

@@ -4,7 +4,7 @@
 // Header (version 2): magic, version, format, N, K, planes, group, tensor
 // scale, row tiles, columns, stream offsets and sizes, at byte 72 the number
 // of base-128 digits of the largest TQ scale in units of 2^-24 (1 for BitNet,
-// 0 for d = 3), and the d = 3 codebook at byte 128.
+// 0 for balanced ternary), and the balanced-ternary codebook at byte 128.
 //
 // 2-bit planes (BitNet b1.58 layout of the QORA-LLM-2B page, "Ternary GEMV";
 // sasori TQ{K}P planes): each weight is a 2-bit code 00 -> 0, 01 -> +1,
@@ -17,18 +17,18 @@
 // TQ scales (fp16, one per plane per group of g along K) are ordered
 // [row tile][group][plane][row].
 //
-// Balanced ternary d = 3 (Entrit card, "Quantization details"): digits
-// u = t + 1 are packed five per byte in base 3 (first digit least
-// significant). A column covers 80 k of a 32-row tile. Per row it holds 16
-// byte triples: triple i carries the 15 trits of the five weights
-// k = 80c + 16j + i (j = 0..4, one weight of each of the column's five groups
-// of 16), weight by weight (t0, t1, t2 of weight j are trits 3j, 3j+1, 3j+2 of
-// the triple, trits 5b..5b+4 in byte b); byte b of triple i sits at
-// b * 512 + 16 r + i. Then one more triple per row (bytes at 1536 + 32 b + r)
-// holding the five groups' codebook indices in the same order (digit q of
-// index j is trit 3j + q). Keeping the three trits of a weight together
-// lets the decoder read a weight's level U = u0 + 3 u1 + 9 u2 with a few
-// divisions by 3, 9 and 27 instead of extracting every digit.
+// Balanced ternary of depth d (Entrit card, "Quantization details": d = 3;
+// d = 2 and 4 by the same rule): digits u = t + 1 are packed five per byte in
+// base 3 (first digit least significant). A column covers 80 k of a 32-row
+// tile. Per row it holds 16 tuples of d bytes: tuple i carries the 5d trits
+// of the five weights k = 80c + 16j + i (j = 0..4, one weight of each of the
+// column's five groups of 16), weight by weight (t0 .. t(d-1) of weight j are
+// trits dj .. dj+d-1 of the tuple, trits 5b..5b+4 in byte b); byte b of tuple
+// i sits at b * 512 + 16 r + i. Then one triple per row (bytes at
+// 512 d + 32 b + r) holding the five groups' codebook indices in the same
+// order (digit q of index j is trit 3j + q). Keeping the trits of a weight
+// together lets the decoder read a weight's level U = u0 + 3 u1 + 9 u2 (d = 3)
+// with a few divisions by 3, 9 and 27 instead of extracting every digit.
 #include <cmath>
 #include <cstring>
 #include <vector>
@@ -70,12 +70,12 @@ tern_status layout_of(const tern_desc* d, Layout* L) {
       l.scale_bytes = (size_t)l.row_tiles * l.groups * l.planes * kTileRows * 2;
       break;
     case TERN_FMT_BT3:
-      if (d->planes != 3 || d->group != 16 || d->k % 16 != 0) return TERN_EINVAL;
-      l.planes = 3;
+      if (d->planes < 2 || d->planes > 4 || d->group != 16 || d->k % 16 != 0) return TERN_EINVAL;
+      l.planes = d->planes;
       l.group = 16;
       l.groups = d->k / 16;
       l.cols = (d->k + kColK3 - 1) / kColK3;
-      l.trit_bytes = (size_t)l.row_tiles * l.cols * kBt3ColBytes;
+      l.trit_bytes = (size_t)l.row_tiles * l.cols * bt_col_bytes(l.planes);
       l.scale_bytes = 0;
       break;
     default:
@@ -176,9 +176,9 @@ static tern_status pack_tq_scales(const Layout& L, const uint16_t* s, uint8_t* o
   return TERN_OK;
 }
 
-static tern_status pack_bt3(const Layout& L, const int8_t* trits, const uint8_t* idx, uint8_t* out) {
-  const int N = L.n, K = L.k, G = L.groups;
-  for (size_t i = 0; i < (size_t)3 * N * K; ++i)
+static tern_status pack_bt(const Layout& L, const int8_t* trits, const uint8_t* idx, uint8_t* out) {
+  const int N = L.n, K = L.k, G = L.groups, D = L.planes, colb = bt_col_bytes(L.planes);
+  for (size_t i = 0; i < (size_t)D * N * K; ++i)
     if (trits[i] < -1 || trits[i] > 1) return TERN_EFORMAT;
   for (size_t i = 0; i < (size_t)N * G; ++i)
     if (idx[i] > 26) return TERN_EFORMAT;
@@ -186,17 +186,17 @@ static tern_status pack_bt3(const Layout& L, const int8_t* trits, const uint8_t*
 #pragma omp parallel for schedule(static)
   for (int T = 0; T < L.row_tiles; ++T) {
     for (int c = 0; c < L.cols; ++c) {
-      uint8_t* col = base + ((size_t)T * L.cols + c) * kBt3ColBytes;
+      uint8_t* col = base + ((size_t)T * L.cols + c) * colb;
       for (int r = 0; r < kTileRows; ++r) {
         const int n = T * kTileRows + r;
         for (int i = 0; i < 16; ++i) {
-          unsigned dig[15];  // the triple's trits, weight-major
+          unsigned dig[20];  // the tuple's trits, weight-major
           for (int j = 0; j < 5; ++j) {
             const int k = c * kColK3 + 16 * j + i;
-            for (int p = 0; p < 3; ++p)
-              dig[3 * j + p] = (n < N && k < K) ? (unsigned)(trits[((size_t)p * N + n) * K + k] + 1) : 1u;
+            for (int p = 0; p < D; ++p)
+              dig[D * j + p] = (n < N && k < K) ? (unsigned)(trits[((size_t)p * N + n) * K + k] + 1) : 1u;
           }
-          for (int b = 0; b < 3; ++b) {
+          for (int b = 0; b < D; ++b) {
             unsigned v = 0, pw = 1;
             for (int q = 0; q < 5; ++q, pw *= 3) v += dig[5 * b + q] * pw;
             col[b * kPlaneColBytes + r * kChunkBytes + i] = (uint8_t)v;
@@ -218,7 +218,7 @@ static tern_status pack_bt3(const Layout& L, const int8_t* trits, const uint8_t*
         for (int b = 0; b < 3; ++b) {
           unsigned v = 0, pw = 1;
           for (int q = 0; q < 5; ++q, pw *= 3) v += dig[5 * b + q] * pw;
-          col[3 * kPlaneColBytes + b * kTileRows + r] = (uint8_t)v;
+          col[D * kPlaneColBytes + b * kTileRows + r] = (uint8_t)v;
         }
       }
     }
@@ -257,7 +257,7 @@ extern "C" tern_status tern_pack(const tern_desc* desc, const int8_t* trits, con
   uint8_t* o = static_cast<uint8_t*>(out);
   std::memset(o, 0, L.total);
   write_header(o, L, desc, codebook);
-  if (L.fmt == TERN_FMT_BT3) return pack_bt3(L, trits, scale_idx, o);
+  if (L.fmt == TERN_FMT_BT3) return pack_bt(L, trits, scale_idx, o);
   st = pack_2bit(L, trits, o);
   if (st != TERN_OK) return st;
   if (L.fmt == TERN_FMT_TQ) st = pack_tq_scales(L, scales_fp16, o);

@@ -104,7 +104,7 @@ class Layer:
     fmt: str                 # "bitnet" | "tq" | "bt3"
     n: int
     k: int
-    planes: int              # P for bitnet/tq; 3 (depth) for bt3
+    planes: int              # P for bitnet/tq; the depth d for bt3
     group: int               # g along K; K for bitnet; 16 for bt3
     trits: np.ndarray        # int8 [P][N][K]
     tensor_scale: float = 0.0            # bitnet
@@ -130,12 +130,12 @@ def tq_layer(n: int, k: int, planes: int, group: int, seed: int, name: str = "")
     return Layer("tq", n, k, planes, group, t, scales=s, seed=seed, name=name)
 
 
-def bt3_layer(n: int, k: int, seed: int, name: str = "") -> Layer:
+def bt3_layer(n: int, k: int, seed: int, name: str = "", depth: int = 3) -> Layer:
     assert k % 16 == 0
     g = rng(seed)
-    t = draw_trits(g, (3, n, k))
+    t = draw_trits(g, (depth, n, k))
     idx = g.integers(0, 27, size=(n, k // 16), dtype=np.uint8)
-    return Layer("bt3", n, k, 3, 16, t, idx=idx, codebook=codebook27(), seed=seed, name=name)
+    return Layer("bt3", n, k, depth, 16, t, idx=idx, codebook=codebook27(), seed=seed, name=name)
 
 
 # ---------------------------------------------------------------- workloads

@@ -246,3 +246,66 @@ def test_binding_fails_loudly_without_library(tmp_path):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError, match="libtern.so not built"):
         spec.loader.exec_module(mod)
+
+
+# ------------------------------------------ balanced ternary of depth 2 and 4
+@pytest.mark.parametrize("depth", [2, 4])
+@pytest.mark.parametrize("n,k", [(1, 16), (33, 160), (70, 400), (5, 2576)])
+def test_roundtrip_bt_depths(depth, n, k):
+    roundtrip(synth.bt3_layer(n, k, seed=n + k + depth, depth=depth))
+
+
+def test_bt_depth2_bytes_by_hand():
+    # one row, K = 16: t1[3] = -1 (digit 0), everything else 0 (digit 1). Tuple 3
+    # holds the digits of k = 3 (weight 0: t0, t1), then of the padding weights
+    # k = 19, 35, ... (digit 1): byte 0 = 1 + 0*3 + 1*9 + 1*27 + 1*81 = 118, byte 1
+    # = 121. The index 5 = 2 + 1*3: triple byte 0 = 2 + 1*3 + 0*9 = 5 at 2 * 512.
+    t = np.zeros((2, 1, 16), np.int8)
+    t[1, 0, 3] = -1
+    d = tern.make_desc("bt3", 1, 16, 2, 16)
+    buf = tern.pack(d, t, scale_idx=np.array([[5]], np.uint8), codebook=synth.codebook27())
+    assert len(buf) == 256 + 2 * 512 + 96
+    col = buf[256:]
+    assert col[3] == 118 and col[512 + 3] == 121 and col[0] == 121 and col[512] == 121
+    assert col[1024] == 5 and col[1024 + 32] == 0 and col[1024 + 64] == 0
+    u = oracle.unpack(buf)
+    assert np.array_equal(u["trits"], t) and u["idx"].tolist() == [[5]]
+
+
+def test_bt_depth4_bytes_by_hand():
+    # one row, K = 16: t3[5] = +1 (digit 2). Tuple 5, byte 0 holds t0..t3 of k = 5
+    # (1, 1, 1, 2) and t0 of the padding weight k = 21 (1): 1 + 3 + 9 + 2*27 + 81 =
+    # 148; its bytes 1..3 are 121. A weight's four trits straddle bytes from the
+    # second weight on: byte 1 = t1..t3 of k = 21 and t0, t1 of k = 37.
+    t = np.zeros((4, 1, 16), np.int8)
+    t[3, 0, 5] = 1
+    d = tern.make_desc("bt3", 1, 16, 4, 16)
+    buf = tern.pack(d, t, scale_idx=np.array([[26]], np.uint8), codebook=synth.codebook27())
+    assert len(buf) == 256 + 4 * 512 + 96
+    col = buf[256:]
+    assert col[5] == 148 and all(col[b * 512 + 5] == 121 for b in (1, 2, 3))
+    assert col[2048] == 26        # 26 = 2 + 2*3 + 2*9: digits 2, 2, 2 of the first index
+    u = oracle.unpack(buf)
+    assert np.array_equal(u["trits"], t) and u["idx"].tolist() == [[26]]
+
+
+def test_bt_depth_sizes_and_bits():
+    for depth in (2, 3, 4):
+        d = tern.make_desc("bt3", 4096, 4096, depth, 16)
+        assert tern.packed_size(d) == 256 + 128 * 52 * (512 * depth + 96)
+        # (16 d + 3) base-3 bytes per 80 weights of a row: (16 d + 3) / 10 bits per weight
+        d = tern.make_desc("bt3", 32, 4000, depth, 16)
+        assert (tern.packed_size(d) - 256) * 8 / (32 * 4000) == pytest.approx((16 * depth + 3) / 10)
+    for depth in (1, 5):
+        expect(tern.EINVAL, lambda: tern.packed_size(tern.make_desc("bt3", 8, 32, depth, 16)))
+
+
+def test_bt_other_depths_have_no_kernel():
+    # packed, but the GEMV entry points refuse them on the host, before any device work
+    torch = pytest.importorskip("torch")
+    lay = synth.bt3_layer(64, 160, seed=9, depth=2)
+    d, buf = tern.pack_layer(lay)
+    packed = torch.from_numpy(buf).clone()          # torch's allocation: 64-byte aligned
+    x = torch.zeros(160, dtype=torch.int16)
+    y = torch.zeros(64, dtype=torch.float32)
+    expect(tern.EUNSUPPORTED, lambda: tern.gemv(d, packed, tern.ACT_BF16, x, None, tern.OUT_F32, y, stream=0))
