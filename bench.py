@@ -412,6 +412,23 @@ def run_ours(args, rank, world):
     return out
 
 
+def model_token_rate(rows, layers: int):
+    """Tokens/s-equivalent of a decode step that runs every shape of `rows` once per layer at batch 1
+    (projections only): from the per-shape chain times (each GEMV waiting for the previous one) and
+    from the per-shape independent throughputs (all bytes streamed at each shape's rate). None where a
+    row lacks the figure."""
+    one = [r for r in rows if r.get("m", 1) == 1]
+    if not one:
+        return None
+    out = {"layers": layers, "shapes_per_layer": len(one)}
+    if all("chain_us_per_gemv" in r for r in one):
+        out["decode_chain"] = round(1e6 / (layers * sum(r["chain_us_per_gemv"] for r in one)), 1)
+    if all("independent_gbs" in r for r in one):
+        s_per_layer = sum(r["bytes_per_gemv"] / (r["independent_gbs"] * 1e9) for r in one)
+        out["independent"] = round(1.0 / (layers * s_per_layer), 1)
+    return out
+
+
 def run_config(args):
     """Per-shape tables for the other workloads (one JSON line, rank 0, one GPU).
 
@@ -526,7 +543,10 @@ def run_config(args):
         del packs
         torch.cuda.empty_cache()
     assert tern.device_error(stream) == tern.OK
-    return {"metric": METRIC, "config": {"workload": args.config}, "unit": "GB/s", "peak": peak, "per_shape": rows}
+    out = {"metric": METRIC, "config": {"workload": args.config}, "unit": "GB/s", "peak": peak, "per_shape": rows}
+    if args.config in ("tq3p", "bt3"):   # the seven projections of one Llama-3.1-8B layer
+        out["tokens_per_s_equiv"] = model_token_rate(rows, synth.LLAMA_8B_LAYERS)
+    return out
 
 
 def run_ceiling(args):

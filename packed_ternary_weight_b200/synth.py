@@ -54,6 +54,7 @@ LLAMA_8B_SHAPES = (
     ("up_proj", 14336, 4096),
     ("down_proj", 4096, 14336),
 )
+LLAMA_8B_LAYERS = 32
 
 
 def rng(seed: int) -> np.random.Generator:

@@ -35,3 +35,15 @@ def test_code_edits_change_the_key(tmp_path):
 def test_committed_summary_parses():
     v = bench.committed_traffic()
     assert v is None or v > 0
+
+
+def test_model_token_rate():
+    # two shapes per layer, 2 layers: chain 10 + 30 us per layer -> 80 us per token
+    rows = [dict(m=1, bytes_per_gemv=1e6, chain_us_per_gemv=10.0, independent_gbs=1000.0),
+            dict(m=1, bytes_per_gemv=3e6, chain_us_per_gemv=30.0, independent_gbs=3000.0),
+            dict(m=4, bytes_per_gemv=9e9, chain_us_per_gemv=1.0)]          # batched rows are not part of it
+    r = bench.model_token_rate(rows, 2)
+    assert r["decode_chain"] == 12500.0                # 1e6 / 80
+    assert r["independent"] == 250000.0                # 2 layers x (1 us + 1 us) per token
+    assert r["shapes_per_layer"] == 2
+    assert "independent" not in bench.model_token_rate([dict(m=1, bytes_per_gemv=1, chain_us_per_gemv=1.0)], 1)
