@@ -134,6 +134,21 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def clock_verdict(clk):
+    """Why a timed region's clock record rejects its number, or None: hardware or thermal slowdown
+    active, or the SM clock held well below its maximum with no reason given (a leftover clock lock).
+    sw_power_cap alone is the normal state of a 1 kW part under load and is kept."""
+    if not clk or not clk.get("samples"):
+        return None
+    bad = [r for r in clk.get("reasons", []) if r in ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")]
+    if bad:
+        return "throttled: " + ", ".join(bad)
+    sm, mx = clk.get("sm_mhz"), clk.get("sm_max_mhz")
+    if sm and mx and sm < 0.75 * mx and not clk.get("reasons"):
+        return "SM clock %.0f of %.0f MHz with no reason" % (sm, mx)
+    return None
+
+
 # ------------------------------------------------------------ rank plumbing
 def max_over_ranks(ms: float, world: int, device) -> float:
     """The slowest rank's time: every rank calls this, in the same order."""
@@ -303,15 +318,25 @@ def run_ours(args, rank, world):
         for _ in range(args.warmup):
             g_step.replay()
         torch.cuda.synchronize()
-    clocks = ClockSampler(dev.index, not args.no_clocks and rank == 0)
-    t_end = time.time() + (1.0 if not args.no_clocks else 0.0)   # soak so the clock samples see this load
-    with torch.cuda.stream(stream):
-        while time.time() < t_end:
-            for _ in range(20):
-                g_step.replay()
-            torch.cuda.synchronize()
-    ms_total = timed(g_steps, args.steps // spb)
-    clk = clocks.stop()
+
+    def measure():
+        clocks = ClockSampler(dev.index, not args.no_clocks and rank == 0)
+        t_end = time.time() + (1.0 if not args.no_clocks else 0.0)   # soak so the clock samples see this load
+        with torch.cuda.stream(stream):
+            while time.time() < t_end:
+                for _ in range(20):
+                    g_step.replay()
+                torch.cuda.synchronize()
+        ms = timed(g_steps, args.steps // spb)
+        return ms, clocks.stop()
+
+    ms_total, clk = measure()
+    # a record that rejects the number: measure once more (every rank takes the same decision)
+    why = clock_verdict(clk)
+    if max_over_ranks(1.0 if why else 0.0, world, dev) > 0:
+        ms_total, clk = measure()
+        if clk is not None:
+            clk["remeasured_after"] = why
     ms_step = ms_total / args.steps
 
     peak, peak_kind = measured_peaks()

@@ -47,3 +47,15 @@ def test_model_token_rate():
     assert r["independent"] == 250000.0                # 2 layers x (1 us + 1 us) per token
     assert r["shapes_per_layer"] == 2
     assert "independent" not in bench.model_token_rate([dict(m=1, bytes_per_gemv=1, chain_us_per_gemv=1.0)], 1)
+
+
+def test_clock_verdict():
+    ok = dict(sm_mhz=1800.0, sm_max_mhz=1965.0, reasons=["sw_power_cap"], samples=10)
+    assert bench.clock_verdict(ok) is None                                  # the power cap is kept
+    assert bench.clock_verdict(None) is None and bench.clock_verdict(dict(samples=0)) is None
+    hot = dict(ok, reasons=["hw_thermal_slowdown", "sw_power_cap"])
+    assert bench.clock_verdict(hot) == "throttled: hw_thermal_slowdown"
+    locked = dict(sm_mhz=1200.0, sm_max_mhz=1965.0, reasons=[], samples=10)
+    assert "no reason" in bench.clock_verdict(locked)
+    capped_low = dict(locked, reasons=["sw_power_cap"])                   # low, but with a reason
+    assert bench.clock_verdict(capped_low) is None
