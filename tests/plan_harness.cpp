@@ -1,6 +1,7 @@
-// C entry points over the launch-planning helpers that the host and the
-// kernels share (tern_internal.h), built with the host compiler by
-// tests/test_plan_cpu.py so that their invariants are checked without a GPU.
+// C entry points over helpers that the host and the kernels share (launch
+// planning in tern_internal.h, balanced-ternary level decoding in
+// tern_bt_levels.h), built with the host compiler by tests/test_plan_cpu.py so
+// that they are checked without a GPU.
 #include "packed_ternary_weight_b200/csrc/tern_internal.h"
 
 extern "C" {
@@ -37,6 +38,31 @@ int h_const(int which) {
     case 7: return tern::kPlaneColBytes;
     case 8: return tern::kMaxTokensW;
     default: return -1;
+  }
+}
+
+}  // extern "C"
+
+// Balanced-ternary level decoders of depth 2 and 4 (tern_bt_levels.h).
+#include "packed_ternary_weight_b200/csrc/tern_bt_levels.h"
+
+extern "C" {
+
+// n packed argument words per byte position; out[5 i + j] = level j of word i
+void h_pair_levels(const uint32_t* b0, const uint32_t* b1, int n, uint32_t* out) {
+  for (int i = 0; i < n; ++i) {
+    uint32_t U[5];
+    tern::pair_levels(b0[i], b1[i], U);
+    for (int j = 0; j < 5; ++j) out[5 * i + j] = U[j];
+  }
+}
+
+void h_quad_levels(const uint32_t* b0, const uint32_t* b1, const uint32_t* b2, const uint32_t* b3, int n,
+                   uint32_t* out) {
+  for (int i = 0; i < n; ++i) {
+    uint32_t U[5];
+    tern::quad_levels(b0[i], b1[i], b2[i], b3[i], U);
+    for (int j = 0; j < 5; ++j) out[5 * i + j] = U[j];
   }
 }
 

@@ -1,7 +1,8 @@
-"""Host logic of the launch plans, on CPU: the helpers that the host planner and
-the kernels both call (the column-balanced CTA split of the one-CTA-per-SM GEMV,
-the token-pass and shared-memory plans of the tensor-core GEMM) are built with
-the host compiler and checked against brute force and against the limits they
+"""Host logic on CPU: the helpers that the host and the kernels both call (the
+column-balanced CTA split of the one-CTA-per-SM GEMV, the token-pass and
+shared-memory plans of the tensor-core GEMM, the level decoders of balanced
+ternary at depth 2 and 4) are built with the host compiler and checked against
+brute force, exhaustive enumeration, the packer's own bytes and the limits they
 must respect (shared memory, tensor-memory columns, alignment)."""
 import ctypes
 import os
@@ -169,3 +170,94 @@ def test_tensor_layout_fits_every_route(h):
             if tq:                                                      # the stage's scale blocks
                 assert sg == (64 * C // group if 64 * C >= group else 1)
                 assert sc >= 4 * sg * planes * 64
+
+
+# ------------------------------------- balanced-ternary levels, depth 2 and 4
+def _u32(a):
+    return np.ascontiguousarray(a, dtype=np.uint32)
+
+
+def _levels_ref(tuple_bytes, d):
+    """Levels U_j = sum_p 3^p u_{dj+p} from the 5d base-3 digits of a tuple of d bytes (byte 0 first)."""
+    digs = []
+    for b in tuple_bytes:
+        v = int(b)
+        for _ in range(5):
+            digs.append(v % 3)
+            v //= 3
+    return [sum(3 ** p * digs[d * j + p] for p in range(d)) for j in range(5)]
+
+
+def _decode(h, d, cols):
+    """cols: [d][n] packed words (two tuples per word, one per 16-bit lane)."""
+    n = cols.shape[1]
+    out = np.zeros(5 * n, np.uint32)
+    P = ctypes.POINTER(ctypes.c_uint32)
+    keep = [_u32(c) for c in cols]                      # the buffers stay alive during the call
+    args = [k.ctypes.data_as(P) for k in keep]
+    if d == 2:
+        h.h_pair_levels(*args, n, out.ctypes.data_as(P))
+    else:
+        h.h_quad_levels(*args, n, out.ctypes.data_as(P))
+    return out.reshape(n, 5)
+
+
+def _check_lanes(h, d, lo, hi):
+    """lo, hi: [n][d] bytes of the tuples in the low and high lanes."""
+    cols = (hi.astype(np.uint32) << 16) | lo.astype(np.uint32)
+    got = _decode(h, d, cols.T)
+    for lane, tb in ((0, lo), (16, hi)):
+        g = (got >> lane) & 0xFFFF
+        ref = np.array([_levels_ref(t, d) for t in tb])
+        assert np.array_equal(g, ref), (d, lane)
+
+
+def test_pair_levels_exhaustive(h):
+    # every tuple of two base-3 bytes (243^2), against a different tuple in the other lane
+    b = np.arange(243)
+    lo = np.stack(np.meshgrid(b, b, indexing="ij"), -1).reshape(-1, 2)
+    _check_lanes(h, 2, lo, lo[::-1].copy())
+
+
+def test_quad_levels_every_byte_pair(h):
+    # each level reads at most two neighbouring bytes: every value pair of bytes (i, i + 1),
+    # the other bytes random, both lanes
+    g = np.random.default_rng(3)
+    b = np.arange(243)
+    pairs = np.stack(np.meshgrid(b, b, indexing="ij"), -1).reshape(-1, 2)
+    for i in range(3):
+        lo = g.integers(0, 243, size=(len(pairs), 4))
+        lo[:, i:i + 2] = pairs
+        hi = g.integers(0, 243, size=(len(pairs), 4))
+        hi[:, (i + 1) % 3:(i + 1) % 3 + 2] = pairs[::-1]
+        _check_lanes(h, 4, lo, hi)
+
+
+@pytest.mark.parametrize("d", [2, 4])
+def test_levels_from_packed_layers(h, d):
+    # the decoders on the packer's own bytes give the oracle's levels: tuple i of row r in a
+    # column holds k = 80c + 16j + i (j = 0..4)
+    from packed_ternary_weight_b200 import synth, tern
+    import oracle
+    lay = synth.bt3_layer(64, 160, seed=40 + d, depth=d)
+    _, buf = tern.pack_layer(lay)
+    hdr = oracle.parse_header(buf)
+    col = np.asarray(buf[hdr["trit_offset"]:], np.uint8)
+    colb = 512 * d + 96
+    level = sum(3 ** p * lay.trits[p].astype(np.int64) for p in range(d)) + (3 ** d - 1) // 2   # U of every weight
+    for T in range(hdr["row_tiles"]):
+        for c in range(hdr["cols"]):
+            base = (T * hdr["cols"] + c) * colb
+            tb = np.stack([col[base + b * 512: base + b * 512 + 512].reshape(32, 16) for b in range(d)], -1)
+            tb = tb.reshape(-1, d)                                 # [(r, i)][b]
+            half = len(tb) // 2
+            cols = ((tb[half:].astype(np.uint32) << 16) | tb[:half]).T
+            got = _decode(h, d, cols)
+            U = np.concatenate([got & 0xFFFF, got >> 16])          # [(r, i)][j]
+            r = np.arange(32).repeat(16)
+            i = np.tile(np.arange(16), 32)
+            for j in range(5):
+                k = 80 * c + 16 * j + i
+                n = 32 * T + r
+                m = (k < lay.k) & (n < lay.n)
+                assert np.array_equal(U[m, j], level[n[m], k[m]]), (T, c, j)
