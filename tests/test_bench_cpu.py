@@ -1,5 +1,7 @@
-"""The key that ties the committed DRAM-traffic summary to the kernel it was
-captured on: comment edits keep it, code edits change it (CPU only)."""
+"""bench.py's host logic on CPU: the key that ties the committed DRAM-traffic
+summary to the kernel it was captured on (comment edits keep it, code edits
+change it), the token-rate arithmetic, the clock verdict, and the reference
+arm's JSON line."""
 import bench
 
 
@@ -59,3 +61,17 @@ def test_clock_verdict():
     assert "no reason" in bench.clock_verdict(locked)
     capped_low = dict(locked, reasons=["sw_power_cap"])                   # low, but with a reason
     assert bench.clock_verdict(capped_low) is None
+
+
+def test_reference_arm_line():
+    # the reference arm is the oracle on host cores: its JSON line carries the contract's keys
+    import argparse
+    args = argparse.Namespace(steps=1, warmup=0)
+    out = bench.run_reference(args, 0, 1)
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in out, key
+    assert out["impl"] == "reference" and out["value"] > 0 and out["unit"] == "GB/s"
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] == 1
+    assert out["e2e"]["value"] == out["value"] and out["e2e"]["h2d_bytes_per_step"] == 0
+    assert bench.run_reference(args, 1, 2) is None            # other ranks do no work
