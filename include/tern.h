@@ -139,6 +139,8 @@ tern_status tern_workspace_size(const tern_desc* desc, int32_t m, size_t* bytes)
  * single-GEMV workload's "per-token absmax"; the pages give no rounding rule):
  *   a = max |x|, inv = fl32(127 / a), xq = clamp(rint(fl32(x * inv)), -127, 127)
  *   (round half to even), sx = fl32(a / 127); an all-zero token gives xq = 0, sx = 0.
+ *   A token whose a is below 127 / FLT_MAX (about 3.7e-37) has inv = +inf: its
+ *   non-zero values give +-127 and its zeros 0. Activations must be finite.
  *   d_x_bf16 [m][k] bf16 bits; d_xq int8 [m][k]; d_xscale float [m].
  */
 tern_status tern_quantize_act(const uint16_t* d_x_bf16, int32_t m, int32_t k, int8_t* d_xq,

@@ -75,7 +75,10 @@ def quantize_act(x_bits: np.ndarray):
       inv = fl32(127 / a)
       xq  = clamp(rint_half_even(fl32(x_i * inv)), -127, 127)
       sx  = fl32(a / 127)
-    and xq = 0, sx = 0 for an all-zero token.
+    and xq = 0, sx = 0 for an all-zero token. When a is so small that 127 / a
+    overflows fp32 (a < 127 / FLT_MAX, about 3.7e-37), inv is +inf: non-zero x
+    give +-inf, clamped to +-127, and x = 0 gives 0 (the product 0 * inf is
+    taken as 0; the pages say nothing about this case).
     """
     x = (np.asarray(x_bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
     x = np.atleast_2d(x)
@@ -86,8 +89,10 @@ def quantize_act(x_bits: np.ndarray):
         a = np.float32(np.max(np.abs(x[r]))) if x.shape[1] else np.float32(0)
         if a == 0:
             continue
-        inv = np.float32(np.float32(127.0) / a)
-        v = (x[r] * inv).astype(np.float32)          # one fp32 multiply each
+        with np.errstate(over="ignore", invalid="ignore"):
+            inv = np.float32(np.float32(127.0) / a)
+            v = (x[r] * inv).astype(np.float32)      # one fp32 multiply each
+        v = np.where(x[r] == 0, np.float32(0), v)     # 0 * inf (inv overflowed) counts as 0
         q = np.clip(np.rint(v), -127, 127)            # numpy rint: half to even
         xq[r] = q.astype(np.int8)
         sx[r] = np.float32(a / np.float32(127.0))

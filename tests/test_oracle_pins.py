@@ -429,3 +429,15 @@ def test_bt_bpw_steps_by_one_trit_from_the_printed_d3():
     # each level of depth adds one trit (log2 3 bits) per weight; the codebook index is unchanged
     assert oracle.bits_per_weight("bt3", 4) - b3 == pytest.approx(math.log2(3))
     assert b3 - oracle.bits_per_weight("bt3", 2) == pytest.approx(math.log2(3))
+
+
+def test_quantize_act_tiny_token():
+    # absmax below 127 / FLT_MAX: 127 / a overflows to +inf, so every non-zero value
+    # saturates to +-127, zeros stay 0, and sx = fl32(a / 127) is exact rational rounding
+    a = np.float32(2.0 ** -126)                       # smallest normal, also a bf16 value
+    x = bf16_bits([[a, 0.0, -a / 4, a / 2 ** 6]])    # the last two are bf16 subnormals
+    xq, sx = oracle.quantize_act(x)
+    assert xq[0].tolist() == [127, 0, -127, 127]
+    assert Fraction(float(sx[0])) == rn_f32(Fraction(float(a)) / 127)
+    with np.errstate(over="ignore"):
+        assert np.isinf(np.float32(127.0) / a)        # the case this pins: inv overflows
