@@ -151,7 +151,9 @@ tern_status tern_quantize_act(const uint16_t* d_x_bf16, int32_t m, int32_t k, in
  *   d_packed  the bytes produced by tern_pack, copied to the device,
  *             16-byte aligned.
  *   act       TERN_ACT_INT8: d_x int8 [K], d_xscale float [1];
- *             TERN_ACT_BF16: d_x bf16 [K], d_xscale NULL.
+ *             TERN_ACT_BF16: d_x bf16 [K], d_xscale NULL;
+ *             TERN_ACT_BF16_Q8: d_x bf16 [K], quantised inside the GEMV
+ *             (d_xscale ignored). BT3 takes TERN_ACT_BF16 only.
  *   out       TERN_OUT_F32 (float [N]) or TERN_OUT_BF16 (bf16 bits [N]).
  *   d_ws      workspace of ws_bytes (see tern_workspace_size); may be NULL when
  *             tern_workspace_size reports 0, otherwise TERN_ENOSPACE.
@@ -164,6 +166,7 @@ tern_status tern_gemv(const tern_desc* desc, const void* d_packed, tern_act act,
  * Y = X W^T for m tokens (m >= 1), the weights read once for all tokens.
  *   d_x [m][K] (int8 or bf16 bits), d_xscale float [m] for TERN_ACT_INT8,
  *   d_y [m][N]. For TERN_ACT_INT8 the result is bit-identical to the oracle.
+ *   TERN_ACT_BF16 (and so BT3) takes m = 1 only (TERN_EUNSUPPORTED otherwise).
  * For m >= 16 with the 2-bit formats and int8 (or in-kernel quantised bf16)
  * activations the product runs on the tensor cores (tcgen05 int8 MMA, up to
  * 256 tokens per launch); the fp16 group scales are split into small integer
@@ -203,7 +206,7 @@ tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, const void*
 /*
  * tern_gemv without a caller-provided workspace, for callers that cannot
  * allocate device memory (code running where cudaMalloc is not permitted, or
- * inside a framework that owns every device allocation). The paper has no
+ * inside a framework that owns every device allocation). The pages have no
  * counterpart; this is a deployment convenience of this library.
  *   Arguments as tern_gemv (one token), minus d_ws / ws_bytes.
  *   Scratch: a fixed 1 MiB array in device memory owned by the library; every
@@ -237,7 +240,9 @@ tern_status tern_stream_read(const void* d_src, size_t bytes, int32_t mode, int3
 /*
  * Read and clear the device error word (synchronises `stream`).
  * Returns TERN_OK if no kernel reported a failure, TERN_ETIMEOUT if a bounded
- * wait expired, TERN_ECUDA if the read failed.
+ * wait expired, TERN_EFORMAT if a kernel met packed data it cannot use (the
+ * tensor path: a header scale-digit count outside 1..6), TERN_ECUDA if the
+ * read failed.
  */
 tern_status tern_device_error(void* stream);
 
