@@ -33,6 +33,19 @@ def test_all_declared_symbols_exported():
         assert ctypes.cast(getattr(tern.lib, n), ctypes.c_void_p).value
 
 
+def test_binding_declares_every_argument():
+    # every entry point of the header has ctypes argument types in the binding, one per C
+    # parameter (an undeclared size_t or pointer would be passed as a 32-bit int)
+    txt = open(os.path.join(ROOT, "include", "tern.h")).read()
+    for name in header_functions():
+        params = re.search(r"^\s*(?:tern_status|const char\*)\s+" + name + r"\s*\(([^)]*)\)\s*;", txt,
+                           re.S | re.M).group(1)
+        n = 0 if params.strip() in ("", "void") else params.count(",") + 1
+        fn = getattr(tern.lib, name)
+        assert fn.argtypes is not None, name
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+
+
 def test_status_strings():
     for c in range(8):
         assert tern.status_string(c)
