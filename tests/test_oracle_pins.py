@@ -441,3 +441,13 @@ def test_quantize_act_tiny_token():
     assert Fraction(float(sx[0])) == rn_f32(Fraction(float(a)) / 127)
     with np.errstate(over="ignore"):
         assert np.isinf(np.float32(127.0) / a)        # the case this pins: inv overflows
+
+
+def test_bitnet_workload_shapes_follow_the_page():
+    # the BitNet b1.58-2B layer set's seven projections, as the page's architecture fixes them
+    a = load("architecture_pages.json")["bitnet_2b"]
+    h, q, kv, ffn = a["hidden"], a["q_heads"] * a["head_dim"], a["kv_heads"] * a["head_dim"], a["ffn"]
+    want = {"q_proj": (q, h), "k_proj": (kv, h), "v_proj": (kv, h), "o_proj": (h, q),
+            "gate_proj": (ffn, h), "up_proj": (ffn, h), "down_proj": (h, ffn)}
+    assert {name: (n, k) for name, n, k in synth.BITNET_2B_SHAPES} == want
+    assert synth.BITNET_2B_LAYERS == a["layers"]
