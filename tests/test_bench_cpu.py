@@ -75,3 +75,29 @@ def test_reference_arm_line():
     assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] == 1
     assert out["e2e"]["value"] == out["value"] and out["e2e"]["h2d_bytes_per_step"] == 0
     assert bench.run_reference(args, 1, 2) is None            # other ranks do no work
+
+
+def test_parity_samples_plumbing():
+    # the bench's spot check finds each sampled GEMV's rows at its own offset of the step's outputs
+    import numpy as np
+
+    import oracle
+    from packed_ternary_weight_b200 import synth
+    n_layers = 30
+    by, off = {}, 0
+    for li in range(n_layers):
+        for nm, n, k in synth.BITNET_2B_SHAPES:
+            by[(li, nm)] = dict(n=n, k=k, yoff=off)
+            off += n
+    y = np.full(off, np.nan, np.float32)
+    names = [nm for nm, _, _ in synth.BITNET_2B_SHAPES]
+    for li, nm in bench.parity_checks(n_layers):
+        L = by[(li, nm)]
+        lay = synth.bitnet_layer(L["n"], L["k"], synth.bitnet_layer_set_seed(li, names.index(nm)), 0.02)
+        q, s = oracle.quantize_act(synth.draw_x_bf16(lay.seed, 1, lay.k))
+        y[L["yoff"]:L["yoff"] + L["n"]] = oracle.gemv_bitnet_int8(lay.trits, q, s, 0.02)[0]
+    assert bench.parity_samples(y, by, n_layers)
+    li, nm = bench.parity_checks(n_layers)[-1]
+    rows = np.sort(np.random.default_rng(li).choice(by[(li, nm)]["n"], 256, replace=False))
+    y[by[(li, nm)]["yoff"] + rows[7]] += 1.0                     # one wrong output in the last sample
+    assert not bench.parity_samples(y, by, n_layers)
