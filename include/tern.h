@@ -20,8 +20,8 @@
  *                    27-entry log-spaced scale codebook with the index stored
  *                    as three trits (Entrit Llama-3.1-8B-trit-uniform-d3
  *                    card, "Quantization details", d = 3; depths 2 and 4 by
- *                    the same rule are packed, and the GEMV calls refuse them
- *                    with TERN_EUNSUPPORTED).
+ *                    the same rule: the card's positional weights, one trit
+ *                    fewer or more per weight).
  *
  * Conventions for every call:
  *   - All pointers named d_* are device pointers; the others are host
@@ -88,8 +88,7 @@ typedef struct tern_desc {
   int32_t fmt;          /* tern_format */
   int32_t n;            /* output rows N >= 1 */
   int32_t k;            /* input columns K >= 1 */
-  int32_t planes;       /* BITNET: 1; TQ: 1..4; BT3: the depth d, 2..4 (GEMV
-                           kernels: 3) */
+  int32_t planes;       /* BITNET: 1; TQ: 1..4; BT3: the depth d, 2..4 */
   int32_t group;        /* BITNET: ignored (whole row); TQ: g, a multiple of 16
                            in {16,32,64,128,256} dividing K; BT3: 16 */
   float tensor_scale;   /* BITNET: the per-tensor scale s_w; else ignored */
@@ -99,11 +98,19 @@ typedef struct tern_desc {
 /* Human-readable name of a status code (static string). */
 const char* tern_status_string(tern_status s);
 
-/* Size in bytes of the packed buffer for `desc` (256-byte header + streams). */
+/* Size in bytes of the packed buffer for `desc` (256-byte header + streams).
+ * Follows the pages' bits-per-weight accounting: sasori README, "K and g -
+ * the quality dials" (K (2 + 16/g) bits per weight for TQ{K}P); Entrit card,
+ * "Quantization details" (about 5 bits per weight at d = 3, group 16); the
+ * physical size adds whole 32-row tiles and 64- or 80-weight columns. */
 tern_status tern_packed_size(const tern_desc* desc, size_t* bytes);
 
 /*
  * Pack logical weights into the library's layout (host only, no device work).
+ * The pages' "convert once, then run" step: sasori README, "Quickstart -
+ * quantize" (the quantiser writes a packed GGUF) and QORA-LLM-2B, "Converting
+ * from Safetensors" (bf16 weights to a 2-bit ternary binary); the byte layout
+ * is this library's own (the pages' formats are not given in full).
  *   trits       int8 [planes][N][K], values -1, 0, +1 (TERN_EFORMAT otherwise).
  *               BT3: plane p holds t_p, the trit of weight 3^p (p < d).
  *   scales_fp16 TQ: fp16 bit patterns [planes][N][K/group], finite; else NULL.
@@ -119,7 +126,9 @@ tern_status tern_pack(const tern_desc* desc, const int8_t* trits, const uint16_t
                       size_t* out_used);
 
 /*
- * Workspace needed by tern_gemv / tern_gemm_batched for `m` tokens.
+ * Workspace needed by tern_gemv / tern_gemm_batched for `m` tokens. No page
+ * defines it: it is this library's scratch for split reductions and the
+ * tensor-core path.
  *   m < 16: 0 for most layers (K-splits normally reduce inside a thread-block
  *     cluster; only a very long K needs more splits than a cluster holds).
  *   m >= 16 (2-bit formats, TERN_ACT_INT8 or TERN_ACT_BF16_Q8): the tensor-
@@ -148,6 +157,10 @@ tern_status tern_quantize_act(const uint16_t* d_x_bf16, int32_t m, int32_t k, in
 
 /*
  * y = W x for one token (M = 1); same as tern_gemm_batched with m = 1.
+ * The decode GEMV of the pages: QORA-LLM-2B, "Ternary GEMV (No
+ * Multiplication)" (add/sub of activations, one scalar multiply at the end);
+ * sasori README, "How it works" (per-group scaled trit planes, additions
+ * instead of weight multiplies); Entrit card, "Quantization details".
  *   d_packed  the bytes produced by tern_pack, copied to the device,
  *             16-byte aligned.
  *   act       TERN_ACT_INT8: d_x int8 [K], d_xscale float [1];
@@ -164,6 +177,9 @@ tern_status tern_gemv(const tern_desc* desc, const void* d_packed, tern_act act,
 
 /*
  * Y = X W^T for m tokens (m >= 1), the weights read once for all tokens.
+ * The same product as tern_gemv for a batch of tokens (sasori README, "g
+ * (group-size)": fine groups cost decode speed; the several-token and prefill
+ * forms are this library's, the pages run one token at a time).
  *   d_x [m][K] (int8 or bf16 bits), d_xscale float [m] for TERN_ACT_INT8,
  *   d_y [m][N]. For TERN_ACT_INT8 the result is bit-identical to the oracle.
  *   TERN_ACT_BF16 (and so BT3) takes m = 1 only (TERN_EUNSUPPORTED otherwise).
@@ -211,11 +227,15 @@ tern_status tern_gemv_grouped(int32_t count, const tern_desc* descs, const void*
  *   Arguments as tern_gemv (one token), minus d_ws / ws_bytes.
  *   Scratch: a fixed 1 MiB array in device memory owned by the library; every
  *   GPU that loads the library holds it until the process exits. A layer whose
- *   workspace (tern_workspace_size with m = 1) exceeds 1 MiB is rejected with
+ *   workspace (tern_workspace_size with m = 1: the largest over all
+ *   activation modes, whatever `act` is) exceeds 1 MiB is rejected with
  *   TERN_ENOSPACE before anything is enqueued.
  *   The first call on a device looks up the array's device address (once per
  *   device, with that device current); make that first call before any stream
- *   capture. Each call clears the part of the scratch it uses on `stream`
+ *   capture. The address is kept for the life of the process: after
+ *   cudaDeviceReset (or any teardown of the device's primary context) this
+ *   call must not be used again in that process. Each call clears the part of
+ *   the scratch it uses on `stream`
  *   (cudaMemsetAsync) and never allocates or frees memory.
  *   All calls on a device share the same scratch: calls that may overlap on
  *   the GPU (different streams without ordering between them) race.
@@ -245,6 +265,17 @@ tern_status tern_stream_read(const void* d_src, size_t bytes, int32_t mode, int3
  * read failed.
  */
 tern_status tern_device_error(void* stream);
+
+/*
+ * Failure-detection self-test (the pages have no counterpart). Enqueues one
+ * small kernel whose bounded wait cannot succeed: it waits on a shared-memory
+ * barrier that nothing arrives at, gives up after about limit_ns nanoseconds
+ * (the GEMV kernels use the same wait with a 1 s limit), records a timeout in
+ * the device error word and returns. A later tern_device_error() reports
+ * TERN_ETIMEOUT once; the CUDA context stays usable.
+ *   limit_ns  1,000 .. 1,000,000,000 (TERN_EINVAL otherwise).
+ */
+tern_status tern_selftest_wait(uint64_t limit_ns, void* stream);
 
 #ifdef __cplusplus
 }

@@ -52,7 +52,7 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
   const int units = (L.cols + gc - 1) / gc;
   const int P = L.planes;
   const int colk = bt3 ? kColK3 : kColK2;                      // k per column
-  const int colb = bt3 ? kBt3ColBytes : P * kPlaneColBytes;   // bytes per column of a row tile
+  const int colb = bt3 ? bt_col_bytes(P) : P * kPlaneColBytes;  // bytes per column of a row tile
   const int mt = gemv2_mt(xmode, m);
   int rt_total = 0;
   for (int i = 0; i < nprob; ++i) rt_total += row_tiles[i];
@@ -132,7 +132,7 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
 bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, int sms, Gemv2wParams& p,
                  int mt = 1, const int* prob_cols = nullptr) {
   const bool bt3 = L.fmt == TERN_FMT_BT3;
-  if (bt3 && xmode != kXBf16) return false;
+  if (bt3 && (xmode != kXBf16 || L.planes != 3)) return false;  // d = 2, 4: the row-group kernel
   if (nprob > kMaxProblemsW) return false;
   if (mt > 1 && (nprob != 1 || bt3 || xmode == kXBf16 || mt > kMaxTokensW)) return false;
   int begin[kMaxProblemsW + 1];
@@ -287,8 +287,8 @@ tern_status check_one(const tern_desc* desc, const void* d_packed, tern_act act,
 // What the kernels support for this layout and activation mode.
 tern_status supported_2bit(const Layout& L, int xmode) {
   const bool tq = L.fmt == TERN_FMT_TQ;
-  // balanced ternary: the kernels take depth 3 with bf16 activations (depths 2 and 4 are packed only)
-  if (L.fmt == TERN_FMT_BT3) return xmode == kXBf16 && L.planes == 3 ? TERN_OK : TERN_EUNSUPPORTED;
+  // balanced ternary: bf16 activations (depth 3 on both kernels, 2 and 4 on the row-group kernel)
+  if (L.fmt == TERN_FMT_BT3) return xmode == kXBf16 ? TERN_OK : TERN_EUNSUPPORTED;
   if (xmode == kXBf16 && !tq) return TERN_EUNSUPPORTED;
   if (tq && L.k % kColK2 != 0) return TERN_EUNSUPPORTED;
   if (!tq && (long long)L.k * 127 >= (1ll << 24)) return TERN_EUNSUPPORTED;  // exact int32 -> fp32
@@ -626,6 +626,7 @@ extern "C" tern_status tern_device_error(void* stream) {
   if (read_clear_dev_error_stream(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_gemv3(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_gemm_tc(stream, &v) != 0) return TERN_ECUDA;
+  if (read_clear_dev_error_selftest(stream, &v) != 0) return TERN_ECUDA;
   if (v & TERN_DEVERR_TIMEOUT) return TERN_ETIMEOUT;
   return v ? TERN_EFORMAT : TERN_OK;
 }

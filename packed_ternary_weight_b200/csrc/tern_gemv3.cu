@@ -31,6 +31,7 @@
 
 #include <type_traits>
 
+#include "tern_bt_levels.h"
 #include "tern_gemv_common.cuh"
 #include "tern_ptx.cuh"
 
@@ -52,7 +53,7 @@ __host__ __device__ inline Smem3 smem3_plan(const Gemv2Params& p) {
   Smem3 s{};
   const int kr = p.cols_per_split * kColK3;
   const int gr = kr / 16;
-  s.stage_bytes = (int)align_up((size_t)p.stage_cols * kBt3ColBytes, 128);
+  s.stage_bytes = (int)align_up((size_t)p.stage_cols * bt_col_bytes(p.planes), 128);
   size_t off = 0;
   s.bars = off;
   off = align_up(off + (size_t)p.wpc * p.nstage * 8, 128);
@@ -90,7 +91,12 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
 
 }  // namespace
 
+// D: the depth (2, 3 or 4); the tuple of a row holds D bytes, the level bias is (3^D - 1) / 2.
+template <int D>
 __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv2Params p) {
+  static_assert(D >= 2 && D <= 4, "depth 2..4");
+  constexpr int kColB = bt_col_bytes(D);
+  constexpr long long kBias = D == 2 ? 4 : (D == 3 ? 13 : 40);
   extern __shared__ __align__(128) uint8_t smem[];
   const Smem3 sp = smem3_plan(p);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -141,9 +147,9 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
     const int slot = islot;
     islot = islot + 1 == nst ? 0 : islot + 1;
     const int cs = c0 + is_ * sc, ce = min(c1, cs + sc);
-    const uint32_t tb = (uint32_t)(ce - cs) * kBt3ColBytes;
+    const uint32_t tb = (uint32_t)(ce - cs) * kColB;
     mbar_arrive_expect_tx(&bars[slot], tb);
-    bulk_g2s(ring + (size_t)slot * sp.stage_bytes, pq.trit + ((size_t)T * p.cols + cs) * kBt3ColBytes, tb,
+    bulk_g2s(ring + (size_t)slot * sp.stage_bytes, pq.trit + ((size_t)T * p.cols + cs) * kColB, tb,
              &bars[slot], pol);
     ++nissued;
     if (++is_ == spt) {
@@ -204,31 +210,42 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
         const int cs = c0 + s * sc;
         const int ncs = min(sc, c1 - cs);
         for (int cc = 0; cc < ncs; ++cc) {
-          const uint32_t col = st32 + (uint32_t)(cc * kBt3ColBytes);
+          const uint32_t col = st32 + (uint32_t)(cc * kColB);
           const uint32_t kx = (uint32_t)((cs + cc - c0) * kColK3);
           // scale indices of the column's five groups: one more triple, same
           // order as the trits
           uint32_t ix[5];
-          triple_levels(lds_u8(col + 3 * kPlaneColBytes + lane), lds_u8(col + 3 * kPlaneColBytes + 32 + lane),
-                        lds_u8(col + 3 * kPlaneColBytes + 64 + lane), ix);
+          triple_levels(lds_u8(col + D * kPlaneColBytes + lane), lds_u8(col + D * kPlaneColBytes + 32 + lane),
+                        lds_u8(col + D * kPlaneColBytes + 64 + lane), ix);
           // U = u0 + 3 u1 + 9 u2 in byte lanes, for the 4 words x 5 digit positions
           uint32_t U[4][5];
           const uint4 b0 = lds128<0>(col + lane * 16);
           const uint4 b1 = lds128<kPlaneColBytes>(col + lane * 16);
-          const uint4 b2 = lds128<2 * kPlaneColBytes>(col + lane * 16);
-          auto word_u = [&](auto wi_c, uint32_t w0, uint32_t w1, uint32_t w2) {
+          uint4 b2 = make_uint4(0u, 0u, 0u, 0u), b3 = make_uint4(0u, 0u, 0u, 0u);
+          if constexpr (D >= 3) b2 = lds128<2 * kPlaneColBytes>(col + lane * 16);
+          if constexpr (D >= 4) b3 = lds128<3 * kPlaneColBytes>(col + lane * 16);
+          // tuples 4w, 4w+2 in the 16-bit lanes of the even bytes, 4w+1, 4w+3 of the odd ones
+          auto levels = [&](uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t (&u)[5]) {
+            if constexpr (D == 2)
+              pair_levels(w0, w1, u);
+            else if constexpr (D == 3)
+              triple_levels(w0, w1, w2, u);
+            else
+              quad_levels(w0, w1, w2, w3, u);
+          };
+          auto word_u = [&](auto wi_c, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
             constexpr int w = decltype(wi_c)::value;
+            constexpr uint32_t kE = 0x00FF00FFu;
             uint32_t ue[5], uo[5];
-            triple_levels(w0 & 0x00FF00FFu, w1 & 0x00FF00FFu, w2 & 0x00FF00FFu, ue);  // triples 4w, 4w+2
-            triple_levels((w0 >> 8) & 0x00FF00FFu, (w1 >> 8) & 0x00FF00FFu, (w2 >> 8) & 0x00FF00FFu,
-                          uo);  // triples 4w+1, 4w+3
+            levels(w0 & kE, w1 & kE, w2 & kE, w3 & kE, ue);
+            levels((w0 >> 8) & kE, (w1 >> 8) & kE, (w2 >> 8) & kE, (w3 >> 8) & kE, uo);
 #pragma unroll
             for (int j = 0; j < 5; ++j) U[w][j] = ue[j] | (uo[j] << 8);
           };
-          word_u(std::integral_constant<int, 0>{}, b0.x, b1.x, b2.x);
-          word_u(std::integral_constant<int, 1>{}, b0.y, b1.y, b2.y);
-          word_u(std::integral_constant<int, 2>{}, b0.z, b1.z, b2.z);
-          word_u(std::integral_constant<int, 3>{}, b0.w, b1.w, b2.w);
+          word_u(std::integral_constant<int, 0>{}, b0.x, b1.x, b2.x, b3.x);
+          word_u(std::integral_constant<int, 1>{}, b0.y, b1.y, b2.y, b3.y);
+          word_u(std::integral_constant<int, 2>{}, b0.z, b1.z, b2.z, b3.z);
+          word_u(std::integral_constant<int, 3>{}, b0.w, b1.w, b2.w, b3.w);
 #pragma unroll
           for (int j = 0; j < 5; ++j) {
             const uint32_t xo = kx + 16u * j;
@@ -248,7 +265,7 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
             L = dp4a_uu(U[2][j], lv.z, L);
             L = dp4a_uu(U[3][j], lv.w, L);
             const int g = (int)(kx >> 4) + j;  // group within the split
-            const long long S = ((long long)H * 65536 + (long long)M * 256 + L) - 13ll * gsum[g];
+            const long long S = ((long long)H * 65536 + (long long)M * 256 + L) - kBias * gsum[g];
             yacc = fmaf(lds_f32(cb32 + 4u * ix[j]) * gmul[g], __ll2float_rn(S), yacc);
           }
         }
@@ -297,13 +314,14 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
 size_t gemv3_smem_bytes(const Gemv2Params& p) { return smem3_plan(p).total; }
 
 int launch_gemv3(const Gemv2Params& p, bool pdl, void* stream) {
-  if (p.m != 1 || (p.ks > 1 && !p.cluster)) return -1;
+  if (p.m != 1 || (p.ks > 1 && !p.cluster) || p.planes < 2 || p.planes > 4) return -1;
   const Smem3 sp = smem3_plan(p);
-  cudaError_t e = cudaFuncSetAttribute(gemv3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
+  auto kern = p.planes == 2 ? gemv3_kernel<2> : (p.planes == 3 ? gemv3_kernel<3> : gemv3_kernel<4>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
   if (e != cudaSuccess) return (int)e;
   const bool clus = p.cluster && p.ks > 1;
   if (clus && p.ks > 8) {
-    e = cudaFuncSetAttribute(gemv3_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return (int)e;
   }
   Gemv2Params q = p;
@@ -314,7 +332,7 @@ int launch_gemv3(const Gemv2Params& p, bool pdl, void* stream) {
     int dev = 0, sms = 0, occ = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gemv3_kernel, 32 * p.wpc, sp.total);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, 32 * p.wpc, sp.total);
     if (e != cudaSuccess) return (int)e;
     if (occ > 0 && gx > sms * occ) {
       gx = sms * occ;
@@ -342,7 +360,7 @@ int launch_gemv3(const Gemv2Params& p, bool pdl, void* stream) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return (int)cudaLaunchKernelEx(&cfg, gemv3_kernel, q);
+  return (int)cudaLaunchKernelEx(&cfg, kern, q);
 }
 
 }  // namespace tern

@@ -28,7 +28,7 @@ constexpr int kColK3 = 80;          // k per 16-byte chunk, base-3 planes
 constexpr int kChunkBytes = 16;
 constexpr int kPlaneColBytes = kTileRows * kChunkBytes;   // 512
 // balanced ternary of depth d: d base-3 bytes per 5 weights of a row, then the group-index triple
-constexpr int bt_col_bytes(int d) { return d * kPlaneColBytes + 3 * kTileRows; }
+TERN_HD constexpr int bt_col_bytes(int d) { return d * kPlaneColBytes + 3 * kTileRows; }
 constexpr int kBt3ColBytes = bt_col_bytes(3);  // 1632: d = 3, the depth the kernels take
 constexpr int kBt3Groups = 5;       // groups of 16 per base-3 column
 
@@ -247,6 +247,7 @@ int launch_quantize(const uint16_t* x, int m, int k, int8_t* xq, float* xs, void
 int read_clear_dev_error_gemv2(void* stream, unsigned* out);
 int read_clear_dev_error_stream(void* stream, unsigned* out);
 int read_clear_dev_error_gemv3(void* stream, unsigned* out);
+int read_clear_dev_error_selftest(void* stream, unsigned* out);
 int launch_gemv3(const Gemv2Params& p, bool pdl, void* stream);  // balanced ternary d = 3, bf16 x, m = 1
 size_t gemv3_smem_bytes(const Gemv2Params& p);
 int launch_stream_read(const void* src, size_t bytes, int mode, int chunk, int depth, int ctas_per_sm, int warps,

@@ -89,11 +89,12 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 
 // Wait for phase `parity` of `bar` to complete, giving up after about
-// kWaitLimitNs; on expiry the device error word records a timeout and false is
-// returned (the caller then stops using the stage).
+// limit_ns (kWaitLimitNs in every GEMV kernel); on expiry the device error
+// word records a timeout and false is returned (the caller then stops using
+// the stage).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_bounded_ns(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   // back off between tests so that waiting warps leave the issue slots to the
   // warps that have data; check the time limit only now and then
@@ -101,11 +102,15 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   for (uint32_t it = 1;; ++it) {
     __nanosleep(it < 4 ? 32u : 128u);
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u && global_timer_ns() - t0 > kWaitLimitNs) {
+    if ((it & 63u) == 0u && global_timer_ns() - t0 > limit_ns) {
       atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_bounded_ns(bar, parity, kWaitLimitNs);
 }
 
 // Programmatic dependent launch: wait until the preceding grid on the stream

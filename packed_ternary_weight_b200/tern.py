@@ -57,7 +57,8 @@ lib.tern_stream_read.argtypes = [_vp, _sz, ctypes.c_int32, ctypes.c_int32, ctype
                                  ctypes.c_int32, _vp, _vp]
 lib.tern_gemv_grouped.argtypes = [ctypes.c_int32, ctypes.POINTER(Desc), ctypes.POINTER(_vp), ctypes.c_int,
                                   ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.c_int, ctypes.POINTER(_vp), _vp]
-for _f in (lib.tern_packed_size, lib.tern_pack, lib.tern_workspace_size, lib.tern_quantize_act, lib.tern_gemv,
+lib.tern_selftest_wait.argtypes = [ctypes.c_uint64, _vp]
+for _f in (lib.tern_selftest_wait, lib.tern_packed_size, lib.tern_pack, lib.tern_workspace_size, lib.tern_quantize_act, lib.tern_gemv,
            lib.tern_gemm_batched, lib.tern_device_error, lib.tern_gemv_noalloc, lib.tern_gemv_grouped,
            lib.tern_stream_read):
     _f.restype = ctypes.c_int
@@ -184,3 +185,8 @@ def stream_read(src, mode: int, chunk: int, depth: int, ctas_per_sm: int, warps:
 
 def device_error(stream=None) -> int:
     return lib.tern_device_error(_stream(stream))
+
+
+def selftest_wait(limit_ns: int, stream=None):
+    """Enqueue the failure-detection self-test: a bounded wait that expires after limit_ns."""
+    _check(lib.tern_selftest_wait(limit_ns, _stream(stream)), "tern_selftest_wait")

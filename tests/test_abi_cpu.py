@@ -114,6 +114,33 @@ def test_bitnet_bytes_by_hand():
     assert oracle.unpack(buf)["trits"].tolist() == t.tolist()
 
 
+def test_tq_scale_bytes_by_hand():
+    # N = 33 (two 32-row tiles), K = 128, two planes, g = 64: two groups, two
+    # 64-k columns. Trit stream = 2 tiles * 2 columns * 2 planes * 512 B = 4096 B,
+    # so the scale stream starts at 256 + 4096 = 4352. The fp16 scale of (tile T,
+    # group G, plane p, row r) sits at 4352 + ((T*2 + G)*2 + p)*64 + 2r:
+    #   n = 5  (T 0, r 5),  G 0, p 0 -> 4352 + 10          1.0    = 0x3C00
+    #   n = 31 (T 0, r 31), G 1, p 0 -> 4352 + 128 + 62     2^-24 = 0x0001 (subnormal)
+    #   n = 32 (T 1, r 0),  G 1, p 1 -> 4352 + 7*64         0.375 = 0x3600
+    #   n = 32,             G 0, p 1 -> 4352 + 5*64        -2.0   = 0xC000
+    t = np.zeros((2, 33, 128), np.int8)
+    sc = np.zeros((2, 33, 2), np.float16)
+    sc[0, 5, 0], sc[0, 31, 1], sc[1, 32, 1], sc[1, 32, 0] = 1.0, 2.0 ** -24, 0.375, -2.0
+    d = tern.make_desc("tq", 33, 128, 2, 64)
+    buf = tern.pack(d, t, sc)
+    h = oracle.parse_header(buf)
+    assert h["scale_offset"] == 4352 and h["scale_bytes"] == 2 * 2 * 2 * 32 * 2
+    u16 = lambda off: int(buf[off]) | (int(buf[off + 1]) << 8)      # noqa: E731
+    expect_at = {4352 + 10: 0x3C00, 4352 + 128 + 62: 0x0001, 4352 + 7 * 64: 0x3600, 4352 + 5 * 64: 0xC000}
+    for off, v in expect_at.items():
+        assert u16(off) == v, (off, hex(u16(off)))
+    rest = np.array(buf[4352:], np.uint8).copy()
+    for off in expect_at:
+        rest[off - 4352:off - 4352 + 2] = 0
+    assert not rest.any()                           # every other scale (padding rows included) is zero
+    assert np.array_equal(oracle.unpack(buf)["scales"].view(np.uint16), sc.view(np.uint16))
+
+
 def test_bt3_bytes_by_hand():
     # one row, K = 16 (one group): t0[3] = +1 (digit 2), everything else 0
     # (digit 1). Triple i holds the trits of k = 16 j + i (j = 0..4), weight by
@@ -313,12 +340,20 @@ def test_bt_depth_sizes_and_bits():
         expect(tern.EINVAL, lambda: tern.packed_size(tern.make_desc("bt3", 8, 32, depth, 16)))
 
 
-def test_bt_other_depths_have_no_kernel():
-    # packed, but the GEMV entry points refuse them on the host, before any device work
+def test_bt_depths_take_bf16_only():
+    # every depth has a kernel for bf16 activations; int8 activations are refused
+    # on the host, before any device work
     torch = pytest.importorskip("torch")
-    lay = synth.bt3_layer(64, 160, seed=9, depth=2)
-    d, buf = tern.pack_layer(lay)
-    packed = torch.from_numpy(buf).clone()          # torch's allocation: 64-byte aligned
-    x = torch.zeros(160, dtype=torch.int16)
-    y = torch.zeros(64, dtype=torch.float32)
-    expect(tern.EUNSUPPORTED, lambda: tern.gemv(d, packed, tern.ACT_BF16, x, None, tern.OUT_F32, y, stream=0))
+    for depth in (2, 3, 4):
+        lay = synth.bt3_layer(64, 160, seed=9, depth=depth)
+        d, buf = tern.pack_layer(lay)
+        packed = torch.from_numpy(buf).clone()          # torch's allocation: 64-byte aligned
+        x = torch.zeros(160, dtype=torch.int8)
+        sx = torch.ones(1, dtype=torch.float32)
+        y = torch.zeros(64, dtype=torch.float32)
+        expect(tern.EUNSUPPORTED, lambda: tern.gemv(d, packed, tern.ACT_INT8, x, sx, tern.OUT_F32, y, stream=0))
+
+
+def test_selftest_limit_checked_on_host():
+    for bad in (0, 999, 2_000_000_000):
+        expect(tern.EINVAL, lambda: tern.selftest_wait(bad, stream=0))

@@ -64,17 +64,40 @@ def test_clock_verdict():
 
 
 def test_reference_arm_line():
-    # the reference arm is the oracle on host cores: its JSON line carries the contract's keys
+    # the reference arm is the oracle on host cores (spawned processes, oracle code only): its JSON
+    # line carries the contract's keys; two layers keep the test short
     import argparse
-    args = argparse.Namespace(steps=1, warmup=0)
+    import sys
+    args = argparse.Namespace(steps=1, warmup=0, layers=2)
     out = bench.run_reference(args, 0, 1)
     for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
                 "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
         assert key in out, key
     assert out["impl"] == "reference" and out["value"] > 0 and out["unit"] == "GB/s"
-    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] == 1
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["cores"] >= 1
+    assert out["config"]["same_config"] is True               # a whole pass of the (two-layer) set
     assert out["e2e"]["value"] == out["value"] and out["e2e"]["h2d_bytes_per_step"] == 0
     assert bench.run_reference(args, 1, 2) is None            # other ranks do no work
+    # the product library is not loaded on this leg (checked in a fresh interpreter)
+    code = ("import argparse, sys, bench; bench.run_reference(argparse.Namespace(steps=1, warmup=0, layers=1), 0, 1); "
+            "assert 'packed_ternary_weight_b200.tern' not in sys.modules")
+    import subprocess
+    r = subprocess.run([sys.executable, "-c", code], cwd=bench.ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+
+
+def test_oracle_pool_covers_the_layer_set():
+    # every GEMV of the layer set is in exactly one worker's share, and a full pass counts all bytes
+    items = bench.layer_set_items(2)
+    assert len(items) == 14
+    pool = bench.OraclePool(2, 3)
+    try:
+        shares = [it for sh in pool.shares for it in sh]
+        assert sorted(shares) == sorted(items)
+        b, dt = pool.run(1.0)
+        assert b == sum(bench.gemv_algo_bytes(n, k) for _, _, n, k in items) and dt > 0
+    finally:
+        pool.close()
 
 
 def test_parity_samples_plumbing():

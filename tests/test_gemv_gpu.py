@@ -95,6 +95,41 @@ def test_quantize_bit_exact(tern, m, k):
     assert np.array_equal(sx.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
 
 
+def test_quantize_tiny_and_subnormal_tokens(tern):
+    """Token 0: absmax 2^-126, below 127 / FLT_MAX, so 127 / absmax overflows to
+    +inf; its non-zero values (one of them a bf16 subnormal) quantise to +-127 and
+    its zeros to 0. Token 1: absmax 1 with bf16-subnormal values beside it, which
+    quantise to 0. Checked against the oracle for the quantiser and for the GEMV
+    that quantises inside the kernel."""
+    a = np.float32(2.0 ** -126)
+    sub = np.float32(2.0 ** -130)                   # bf16 subnormal
+    t0 = [a, 0.0, -a / 4, sub, -sub, 0.0, a, -a] + [0.0] * 8
+    t1 = [1.0, sub, -sub, 2.0 ** -127, 0.5, -0.25, 0.0, -1.0] + [0.0] * 8
+    x = synth.f32_to_bf16_bits(np.array([t0, t1], np.float32))
+    xq = torch.empty((2, 16), dtype=torch.int8, device="cuda")
+    sx = torch.empty((2,), dtype=torch.float32, device="cuda")
+    tern.quantize_act(x_dev(x), xq, sx)
+    q_ref, s_ref = oracle.quantize_act(x)
+    assert q_ref[0, :8].tolist() == [127, 0, -127, 127, -127, 0, 127, -127]
+    assert q_ref[1, 1:4].tolist() == [0, 0, 0]
+    assert np.array_equal(xq.cpu().numpy(), q_ref)
+    assert np.array_equal(sx.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    lay = synth.bitnet_layer(64, 16, seed=5)
+    d, buf = tern.pack_layer(lay)
+    y = torch.empty((2, lay.n), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(16, tern.workspace_size(d, 2)), dtype=torch.uint8, device="cuda")
+    tern.gemm_batched(d, dev(buf), 2, tern.ACT_BF16_Q8, x_dev(x), None, tern.OUT_F32, y, ws)
+    torch.cuda.synchronize()
+    assert tern.device_error() == tern.OK
+    y_ref = oracle.gemv_bitnet_int8(lay.trits, q_ref, s_ref, lay.tensor_scale)
+    assert np.array_equal(y.cpu().numpy().view(np.uint32), y_ref.view(np.uint32))
+    for i in range(2):                              # one token at a time: the single-token kernels
+        y1 = torch.empty((1, lay.n), dtype=torch.float32, device="cuda")
+        tern.gemv(d, dev(buf), tern.ACT_BF16_Q8, x_dev(x[i:i + 1]), None, tern.OUT_F32, y1, ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(y1.cpu().numpy()[0].view(np.uint32), y_ref[i].view(np.uint32))
+
+
 # ---------------------------------------------------------- BitNet int8 path
 def bitnet_check(tern, layer, m=1, **kw):
     x = synth.draw_x_bf16(layer.seed, m, layer.k)
