@@ -267,6 +267,76 @@ tern_status tern_stream_read(const void* d_src, size_t bytes, int32_t mode, int3
 tern_status tern_device_error(void* stream);
 
 /*
+ * Decode step of a BitNet b1.58 transformer at batch 1 (QORA-LLM-2B page,
+ * "Architecture" and "SubLN Pattern (4 norms per layer)"). Per layer:
+ *   x = RMSNorm(h) -> q, k, v (ternary linears) -> RoPE (rotate_half) on q, k
+ *   -> k, v appended to the bf16 cache at `pos` -> GQA attention over
+ *   positions 0..pos -> RMSNorm -> o_proj -> h += o -> RMSNorm -> gate, up ->
+ *   RMSNorm(relu(gate)^2 * up) -> down_proj -> h += d.
+ * Every ternary linear quantises its input per token to int8 (the rule of
+ * tern_quantize_act on fp32 values) and is exact as in tern_gemv. RMSNorm:
+ * y_i = fl(fl(x_i * r) * g_i), r = 1/sqrt(mean(x^2) + eps) rounded once to
+ * fp32. RoPE products and sums rounded in fp32; relu^2 * up and the residual
+ * adds in fp32; attention (scores scaled by 1/sqrt(128), softmax, weighted
+ * values) in fp32.
+ */
+typedef struct tern_decode_model {
+  int32_t layers;        /* 1..64 */
+  int32_t hidden;        /* D, a multiple of 64 */
+  int32_t inter;         /* F (FFN width), a multiple of 64 */
+  int32_t heads;         /* H query heads of 128; H * 128 a multiple of 64 */
+  int32_t kv_heads;      /* KVH, H / KVH in 1..4, KVH <= 16 */
+  int32_t head_dim;      /* 128 */
+  int32_t max_pos;       /* cache capacity in positions */
+  float eps;             /* RMSNorm epsilon */
+  /* host array [layers * 7] of device pointers to tern_pack'ed BitNet buffers
+     (16-byte aligned), per layer in the order q [H*128][D], k [KVH*128][D],
+     v [KVH*128][D], o [D][H*128], gate [F][D], up [F][D], down [D][F] */
+  const void* const* packed;
+  const float* d_gains;  /* fp32 [layers][2D + H*128 + F]: input_layernorm (D),
+                            attn_sub_norm (H*128), post_attention_layernorm (D),
+                            ffn_sub_norm (F) */
+  uint16_t* d_kcache;    /* bf16 [layers][KVH][max_pos][128] keys (after RoPE) */
+  uint16_t* d_vcache;    /* bf16 [layers][KVH][max_pos][128] values */
+  const float* d_rope;   /* fp32 [max_pos][64][2] cos, sin (tern_decode_rope_table) */
+} tern_decode_model;
+
+/* cos and sin of p * theta^(-2i/head_dim), p < max_pos, i < head_dim/2, each
+ * computed in double precision and rounded to fp32, into the host buffer out
+ * [max_pos][head_dim/2][2] (RoPE, "rotate_half, theta=500,000" on the
+ * QORA-LLM-2B page). */
+tern_status tern_decode_rope_table(int32_t max_pos, int32_t head_dim, double theta, float* out);
+
+/* Workspace of tern_decode_step (256-byte aligned, zero-filled before its
+ * first use; a completed step leaves it ready for the next). No page defines
+ * it: barrier counters, the GEMVs' partial row sums, the attention's partial
+ * softmax states and output. */
+tern_status tern_decode_workspace_size(const tern_decode_model* model, size_t* bytes);
+
+/*
+ * Run stages first..last (inclusive) of the decode step of the token at
+ * position `pos` (0 <= pos < max_pos). Stage index = 5 * layer + s with
+ * s = 0 q/k/v, 1 attention, 2 o_proj, 3 gate/up, 4 down_proj; a run may
+ * start at s = 0, 2 or 3 (TERN_EINVAL otherwise). The whole step is
+ * first = 0, last = 5 * layers - 1.
+ *   d_h_in   fp32 [D]: the residual stream where the run starts.
+ *   d_h_out  fp32 [D]: the residual stream after the run's last residual add.
+ *   d_attn_in  fp32 [H*128]: the attention output when the run starts at an
+ *              o_proj stage, else ignored (may be NULL).
+ *   d_trace  optional fp32 [layers][2*H*128 + 2*KVH*128]: per layer q after
+ *            RoPE [H*128], k after RoPE [KVH*128], v [KVH*128], attention
+ *            output [H*128] (written for the layers whose stages run).
+ * The cache positions 0..pos-1 must hold the earlier tokens' keys and values;
+ * the step writes position pos of every layer it runs attention for. One
+ * cooperative launch with one CTA per SM; all waits are bounded (1 s), and a
+ * step that gave up reports TERN_ETIMEOUT through tern_device_error, after
+ * which the workspace must be zero-filled again.
+ */
+tern_status tern_decode_step(const tern_decode_model* model, int32_t pos, const float* d_h_in, float* d_h_out,
+                             int32_t first, int32_t last, const float* d_attn_in, float* d_trace, void* d_ws,
+                             size_t ws_bytes, void* stream);
+
+/*
  * Failure-detection self-test (the pages have no counterpart). Enqueues one
  * small kernel whose bounded wait cannot succeed: it waits on a shared-memory
  * barrier that nothing arrives at, gives up after about limit_ns nanoseconds

@@ -6,3 +6,4 @@ never imports it and shares no code with it.
 """
 from .tern_oracle import *  # noqa: F401,F403
 from .unpack import *  # noqa: F401,F403
+from . import decode  # noqa: F401,E402  (the BitNet decode layer composition)

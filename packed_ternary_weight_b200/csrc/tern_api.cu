@@ -627,6 +627,7 @@ extern "C" tern_status tern_device_error(void* stream) {
   if (read_clear_dev_error_gemv3(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_gemm_tc(stream, &v) != 0) return TERN_ECUDA;
   if (read_clear_dev_error_selftest(stream, &v) != 0) return TERN_ECUDA;
+  if (read_clear_dev_error_decode(stream, &v) != 0) return TERN_ECUDA;
   if (v & TERN_DEVERR_TIMEOUT) return TERN_ETIMEOUT;
   return v ? TERN_EFORMAT : TERN_OK;
 }

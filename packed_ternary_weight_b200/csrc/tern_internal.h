@@ -253,6 +253,52 @@ size_t gemv3_smem_bytes(const Gemv2Params& p);
 int launch_stream_read(const void* src, size_t bytes, int mode, int chunk, int depth, int ctas_per_sm, int warps,
                        unsigned* sink, void* stream);
 
+// ------------------------------------------------ persistent decode step
+constexpr int kDecMaxLayers = 64;
+constexpr int kDecHeadDim = 128;
+constexpr int kDecMaxVec = 14336;        // largest hidden / FFN / attention width
+constexpr int kDecMaxKvHeads = 16;
+constexpr int kDecMaxRep = 4;            // query heads per KV head
+constexpr int kDecMaxSplits = 4;         // column ranges per row tile
+constexpr int kDecMaxPartsPerCta = 8;
+constexpr int kDecMaxSlots = 64;         // 4 KB weight slots of the ring
+constexpr size_t kDecSmemBytes = 227 * 1024;
+
+// One GEMV stage of a decode layer (the same shapes in every layer): the
+// projections' row tiles, each cut into `splits` column ranges ("parts").
+struct DecStage {
+  int nprob;           // projections in the stage (q, k, v: 3; gate, up: 2; else 1)
+  int proj[3];         // their indices among q, k, v, o, gate, up, down
+  int tile0[4];        // first stage tile of each projection; tile0[nprob] = tiles
+  int cols;            // 64-k columns (K / 64)
+  int splits, parts;   // parts = tiles * splits
+};
+
+struct DecParams {
+  const uint8_t* packed[kDecMaxLayers][7];   // BitNet packed buffers (device)
+  const float* gains;       // [layers][gain_stride]: input D | attn_sub H*128 | post D | ffn_sub F
+  uint16_t* kc;             // bf16 [layers][KVH][max_pos][128]
+  uint16_t* vc;
+  const float* rope;        // [max_pos][64][2] cos, sin
+  const float* h_in;        // [D]
+  float* h_out;             // [D]
+  const float* attn_in;     // [H*128] when the run starts at an o_proj stage
+  float* trace;             // optional [layers][trace_stride]
+  uint8_t* ws;
+  size_t off_ctl, off_part[4], off_att, off_attn, ws_bytes;
+  int layers, D, F, H, KVH, max_pos, pos, first, last;
+  int gain_stride, trace_stride;
+  int vmax;                 // max(D, F, H*128): the image width
+  int grid, ns;             // CTAs; attention position ranges per KV head
+  float eps;
+  DecStage st[4];           // qkv, o, gate/up, down
+};
+
+int launch_decode(const DecParams& p, void* stream);  // -1: does not fit one CTA per SM
+size_t decode_smem_bytes(const DecParams& p);
+int decode_ring_slots(const DecParams& p);
+int read_clear_dev_error_decode(void* stream, unsigned* out);
+
 // Shared-memory bytes a 2-bit GEMV CTA needs for these parameters.
 size_t gemv2_smem_bytes(const Gemv2Params& p, int xmode);
 int gemv2_mt(int xmode, int m);   // tokens per pass of the kernel instantiated for m

@@ -177,3 +177,50 @@ def tq2p_prefill_layers():
     """TQ2P (2 planes, g = 32) prefill layers; seed 400 + shape index."""
     for si, (name, n, k) in enumerate(PREFILL_SHAPES):
         yield tq_layer(n, k, 2, 32, seed=400 + si, name=name)
+
+
+# ------------------------------------------------------------ decode step
+# Synthetic BitNet b1.58 decoder (no trained weights): per layer the seven
+# projections of the layer set's recipe (seeds 1000 + 7 layer + projection
+# by default), RMSNorm gains bf16(1 + 0.1 z), a KV cache prefix of bf16
+# N(0,1) keys and values, and the residual stream of the token as bf16 N(0,1)
+# values (standing in for an embedding row).
+@dataclass
+class DecodeModel:
+    D: int
+    F: int
+    H: int
+    KVH: int
+    layers: list            # per layer: seven Layer objects (q, k, v, o, gate, up, down)
+    gains: list             # per layer: four fp32 vectors (input D, attn_sub H*128, post D, ffn_sub F)
+    kcache: np.ndarray      # bf16 bits [L][KVH][max_pos][128]
+    vcache: np.ndarray
+    h0: np.ndarray          # fp32 [D]
+    pos: int
+    max_pos: int
+
+
+def decode_model(D: int = 2560, F: int = 6912, H: int = 20, KVH: int = 5, n_layers: int = 1, pos: int = 1023,
+                 max_pos: int = 1024, seed: int = 1000, head_dim: int = 128) -> DecodeModel:
+    """Seeded synthetic decoder inputs. Layer li, projection pi uses seed + 7 li + pi (with the
+    default seed and BitNet-2B shapes these are the layer set's layers)."""
+    shapes = [(H * head_dim, D), (KVH * head_dim, D), (KVH * head_dim, D), (D, H * head_dim), (F, D), (F, D),
+              (D, F)]
+    names = [nm for nm, _, _ in BITNET_2B_SHAPES]
+    layers, gains = [], []
+    for li in range(n_layers):
+        layers.append([bitnet_layer(n, k, seed + 7 * li + pi, 0.02, name=f"L{li}.{names[pi]}")
+                       for pi, (n, k) in enumerate(shapes)])
+        g = rng(seed + 500_000 + li)
+        gains.append([bf16_bits_to_f32(f32_to_bf16_bits((1.0 + 0.1 * g.standard_normal(n)).astype(np.float32)))
+                      for n in (D, H * head_dim, D, F)])
+    g = rng(seed + 600_000)
+    kc = f32_to_bf16_bits(g.standard_normal((n_layers, KVH, max_pos, head_dim), dtype=np.float32))
+    vc = f32_to_bf16_bits(g.standard_normal((n_layers, KVH, max_pos, head_dim), dtype=np.float32))
+    h0 = bf16_bits_to_f32(f32_to_bf16_bits(g.standard_normal(D, dtype=np.float32)))
+    return DecodeModel(D, F, H, KVH, layers, gains, kc, vc, h0, pos, max_pos)
+
+
+def decode_attn_input(seed: int, n: int) -> np.ndarray:
+    """A stand-in attention output (fp32 N(0,1)) for runs that start at o_proj."""
+    return rng(seed + 700_000).standard_normal(n, dtype=np.float32)

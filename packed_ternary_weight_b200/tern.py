@@ -58,6 +58,21 @@ lib.tern_stream_read.argtypes = [_vp, _sz, ctypes.c_int32, ctypes.c_int32, ctype
 lib.tern_gemv_grouped.argtypes = [ctypes.c_int32, ctypes.POINTER(Desc), ctypes.POINTER(_vp), ctypes.c_int,
                                   ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.c_int, ctypes.POINTER(_vp), _vp]
 lib.tern_selftest_wait.argtypes = [ctypes.c_uint64, _vp]
+
+
+class DecodeModelC(ctypes.Structure):
+    _fields_ = [("layers", ctypes.c_int32), ("hidden", ctypes.c_int32), ("inter", ctypes.c_int32),
+                ("heads", ctypes.c_int32), ("kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("max_pos", ctypes.c_int32), ("eps", ctypes.c_float), ("packed", ctypes.POINTER(_vp)),
+                ("d_gains", _vp), ("d_kcache", _vp), ("d_vcache", _vp), ("d_rope", _vp)]
+
+
+lib.tern_decode_rope_table.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_double, _vp]
+lib.tern_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeModelC), ctypes.POINTER(_sz)]
+lib.tern_decode_step.argtypes = [ctypes.POINTER(DecodeModelC), ctypes.c_int32, _vp, _vp, ctypes.c_int32,
+                                 ctypes.c_int32, _vp, _vp, _vp, _sz, _vp]
+for _f in (lib.tern_decode_rope_table, lib.tern_decode_workspace_size, lib.tern_decode_step):
+    _f.restype = ctypes.c_int
 for _f in (lib.tern_selftest_wait, lib.tern_packed_size, lib.tern_pack, lib.tern_workspace_size, lib.tern_quantize_act, lib.tern_gemv,
            lib.tern_gemm_batched, lib.tern_device_error, lib.tern_gemv_noalloc, lib.tern_gemv_grouped,
            lib.tern_stream_read):
@@ -190,3 +205,37 @@ def device_error(stream=None) -> int:
 def selftest_wait(limit_ns: int, stream=None):
     """Enqueue the failure-detection self-test: a bounded wait that expires after limit_ns."""
     _check(lib.tern_selftest_wait(limit_ns, _stream(stream)), "tern_selftest_wait")
+
+
+def decode_rope_table(max_pos: int, head_dim: int = 128, theta: float = 500000.0) -> np.ndarray:
+    """cos/sin table [max_pos][head_dim/2][2] (fp32) computed by the library."""
+    out = np.empty((max_pos, head_dim // 2, 2), dtype=np.float32)
+    _check(lib.tern_decode_rope_table(max_pos, head_dim, theta, _ptr(out)), "tern_decode_rope_table")
+    return out
+
+
+class DecodeModel:
+    """Marshalled tern_decode_model: device buffers are caller-owned tensors; the host array of
+    packed-buffer pointers lives as long as this object."""
+
+    def __init__(self, packed, gains, kcache, vcache, rope, hidden: int, inter: int, heads: int, kv_heads: int,
+                 max_pos: int, eps: float = 1e-5, head_dim: int = 128):
+        n = len(packed)
+        assert n % 7 == 0
+        self._keep = (packed, gains, kcache, vcache, rope)
+        self._ptrs = (_vp * n)(*[p.data_ptr() for p in packed])
+        self.c = DecodeModelC(n // 7, hidden, inter, heads, kv_heads, head_dim, max_pos, eps,
+                              ctypes.cast(self._ptrs, ctypes.POINTER(_vp)), gains.data_ptr(), kcache.data_ptr(),
+                              vcache.data_ptr(), rope.data_ptr())
+
+    def workspace_size(self) -> int:
+        out = _sz()
+        _check(lib.tern_decode_workspace_size(ctypes.byref(self.c), ctypes.byref(out)), "tern_decode_workspace_size")
+        return out.value
+
+    def step(self, pos: int, h_in, h_out, ws, first: int = 0, last: int | None = None, attn_in=None, trace=None,
+             stream=None):
+        last = 5 * self.c.layers - 1 if last is None else last
+        _check(lib.tern_decode_step(ctypes.byref(self.c), pos, _ptr(h_in), _ptr(h_out), first, last, _ptr(attn_in),
+                                    _ptr(trace), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+               "tern_decode_step")
