@@ -58,7 +58,7 @@ def parse():
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other workloads' per-shape rows in the default line")
     ap.add_argument("--profile", default=None,
-                    help="run only one case eagerly for a profiler: step | <shape>_indep | <shape>_chain "
+                    help="run only one case eagerly for a profiler: step | decode | <shape>_indep | <shape>_chain "
                          "(headline workload); with --config tq3p|bt3|tq2p|single: <shape>:<m> (the copies "
                          "launched one after another) or <shape>:1:indep (one grouped launch)")
     ap.add_argument("--reps", type=int, default=3)
@@ -270,6 +270,10 @@ def run_ours(args, rank, world):
     gbytes = lambda L: L["wbytes"] + 2 * L["k"] + 4 * L["n"]    # noqa: E731
     step_bytes = sum(gbytes(L) for L in layers)
 
+    if args.profile == "decode":
+        run_decode(tern, torch, stream, {(L["layer"], L["name"]): L["packed"] for L in layers}, args.layers,
+                   reps=args.reps, clocks=False)
+        return None
     if args.profile:
         cases = {"step": step, "chain_step": chain_step}
         for nm, _, _ in synth.BITNET_2B_SHAPES:
@@ -395,6 +399,10 @@ def run_ours(args, rank, world):
                               independent_pool="%d copies (%.0f MB) in %d launch(es), 4 rounds per graph" % (
                                   copies, bp / 1e6, len(launches))))
 
+    # the whole decode step of a token (every layer, attention included), one launch per token
+    decode = run_decode(tern, torch, stream, {(L["layer"], L["name"]): L["packed"] for L in layers}, args.layers,
+                        reps=max(3, min(args.steps, 100)), clocks=not args.no_clocks and rank == 0)
+
     # end to end through the public API: pinned H2D of the step's activations,
     # the captured step, D2H of the step's outputs
     h2d = x_all_host.numel() * 2
@@ -458,10 +466,12 @@ def run_ours(args, rank, world):
                          "ms_per_step": round(ms_chain_step, 4),
                          "gbs": round(step_bytes / (ms_chain_step * 1e-3) / 1e9, 1)},
         "tokens_per_s_equiv": {"independent": round(world * 1e3 / ms_step, 1),
+                               "decode_step": decode["tokens_per_s"],
                                "decode_chain": round(world * 1e3 / ms_chain_step, 1),
                                "basis": "a step's GEMVs are the projection layers one decoded token at batch 1 "
                                         "streams (attention, norms and the output head are not on this path); "
                                         "tokens per second = steps per second, summed over replicas"},
+        "decode_step": decode,
         "e2e": {"value": round(replica_gbs(step_bytes, ms_e2e, world), 1), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * len(step_launches),
@@ -495,6 +505,64 @@ def model_token_rate(rows, layers: int):
     if all("independent_gbs" in r for r in one):
         s_per_layer = sum(r["bytes_per_gemv"] / (r["independent_gbs"] * 1e9) for r in one)
         out["independent"] = round(1.0 / (layers * s_per_layer), 1)
+    return out
+
+
+DECODE_POS = 1023
+DECODE_WORKLOAD = ("BitNet b1.58-2B decode step at batch 1: 30 layers (RMSNorm, q/k/v, RoPE theta 500000, GQA 20/5 x "
+                   "128 over a bf16 KV cache, attn_sub_norm, o_proj, residual, RMSNorm, gate/up, relu^2 * up, "
+                   "ffn_sub_norm, down_proj, residual), token at position %d (%d cached positions), the layer set's "
+                   "packed weights, synthetic gains, cache and residual stream" % (DECODE_POS, DECODE_POS))
+
+
+def run_decode(tern, torch, stream, packed_by, n_layers: int, reps: int, pos: int = DECODE_POS, clocks=True):
+    """The whole decode step of one token (one cooperative launch per token), timed with events over
+    back-to-back launches. packed_by: (layer, projection name) -> packed device buffer."""
+    m = synth.decode_model(n_layers=n_layers, pos=pos, max_pos=pos + 1)
+    names = [nm for nm, _, _ in synth.BITNET_2B_SHAPES]
+    packed = [packed_by[(li, nm)] for li in range(n_layers) for nm in names]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    gains = torch.from_numpy(np.concatenate([np.concatenate(g) for g in m.gains]).astype(np.float32)).to(dev)
+    kc = torch.from_numpy(m.kcache.view(np.int16)).to(dev)
+    vc = torch.from_numpy(m.vcache.view(np.int16)).to(dev)
+    rope = torch.from_numpy(tern.decode_rope_table(m.max_pos)).to(dev)
+    model = tern.DecodeModel(packed, gains, kc, vc, rope, m.D, m.F, m.H, m.KVH, m.max_pos)
+    ws = torch.zeros(model.workspace_size(), dtype=torch.uint8, device=dev)
+    h_in = torch.from_numpy(m.h0).to(dev)
+    h_out = torch.empty_like(h_in)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            model.step(pos, h_in, h_out, ws, stream=stream)
+        torch.cuda.synchronize()
+        assert tern.device_error(stream) == tern.OK
+        clk = ClockSampler(dev.index, clocks)
+        t_end = time.time() + (0.5 if clocks else 0.0)
+        while time.time() < t_end:
+            for _ in range(20):
+                model.step(pos, h_in, h_out, ws, stream=stream)
+            torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            model.step(pos, h_in, h_out, ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ck = clk.stop()
+    assert tern.device_error(stream) == tern.OK
+    ms = e0.elapsed_time(e1) / reps
+    wbytes = sum(int(p.numel()) - 256 for p in packed)
+    kv_read = 2 * n_layers * m.KVH * pos * 128 * 2
+    other = gains.numel() * 4 + 2 * n_layers * m.KVH * 128 * 2 + rope.shape[1] * 8
+    total = wbytes + kv_read + other
+    peak, _ = measured_peaks()
+    out = {"workload": DECODE_WORKLOAD, "launches_per_token": 1, "ms_per_token": round(ms, 4),
+           "tokens_per_s": round(1e3 / ms, 1), "bytes_per_token": total,
+           "bytes_basis": "packed ternary weights %.1f MB + cached keys and values read %.1f MB + gains, RoPE row "
+                          "and the new cache entries %.2f MB" % (wbytes / 1e6, kv_read / 1e6, other / 1e6),
+           "gbs": round(total / (ms * 1e-3) / 1e9, 1), "frac": round(total / (ms * 1e-3) / 1e9 / peak, 4),
+           "timing": "%d back-to-back launches (one per token), CUDA events" % reps}
+    if ck is not None:
+        out["clocks"] = ck
     return out
 
 

@@ -261,7 +261,7 @@ constexpr int kDecMaxKvHeads = 16;
 constexpr int kDecMaxRep = 4;            // query heads per KV head
 constexpr int kDecMaxSplits = 4;         // column ranges per row tile
 constexpr int kDecMaxPartsPerCta = 8;
-constexpr int kDecMaxSlots = 64;         // 4 KB weight slots of the ring
+constexpr int kDecMaxSlots = 32;         // 8 KB weight slots of the ring
 constexpr size_t kDecSmemBytes = 227 * 1024;
 
 // One GEMV stage of a decode layer (the same shapes in every layer): the
