@@ -267,6 +267,35 @@ tern_status tern_stream_read(const void* d_src, size_t bytes, int32_t mode, int3
 tern_status tern_device_error(void* stream);
 
 /*
+ * Dense -> ternary fit of a weight matrix on the GPU, producing the inputs of
+ * tern_pack (the pages' "quantize" step: sasori README, "How it works & paper"
+ * -- each matrix fit on its own into K per-group-scaled trit planes, weight
+ * only, no calibration -- and "K and g"). Greedy residual planes: per row and
+ * group of g, and plane p, gamma = mean |R_p|; t = sign(R_p) where |R_p| >
+ * gamma / 2, else 0; s = fp16_rn(mean of |R_p| over the non-zero trits) (0 if
+ * none); R_{p+1} = R_p - s t; R_0 = W. fp64 arithmetic, group sums in index
+ * order.
+ *   d_w       fp32 [n][k], device.
+ *   d_trits   int8 [planes][n][k] out; d_scales fp16 bits [planes][n][k/group] out.
+ *   planes 1..4; group a power of two in 16..256 dividing k.
+ */
+tern_status tern_fit_tq(const float* d_w, int32_t n, int32_t k, int32_t planes, int32_t group, int8_t* d_trits,
+                        uint16_t* d_scales, void* stream);
+
+/*
+ * Dense -> balanced ternary fit of depth d (Entrit card, "Quantization
+ * details": uniform PTQ, depth 3, group 16, 27-entry log-spaced codebook):
+ * per row and group of 16, for each codebook entry c the levels L =
+ * clamp(rint(w / c), -(3^d-1)/2, (3^d-1)/2); the entry with the least sum of
+ * squared errors (lowest index on a tie); trits = balanced-ternary digits of L
+ * (L = sum_j 3^j t_j). fp64 arithmetic, sums in index order.
+ *   d_w        fp32 [n][k], k a multiple of 16; d_codebook fp32 [27], device.
+ *   d_trits    int8 [depth][n][k] out; d_idx uint8 [n][k/16] out. depth 2..4.
+ */
+tern_status tern_fit_bt(const float* d_w, int32_t n, int32_t k, int32_t depth, const float* d_codebook,
+                        int8_t* d_trits, uint8_t* d_idx, void* stream);
+
+/*
  * Decode step of a BitNet b1.58 transformer at batch 1 (QORA-LLM-2B page,
  * "Architecture" and "SubLN Pattern (4 norms per layer)"). Per layer:
  *   x = RMSNorm(h) -> q, k, v (ternary linears) -> RoPE (rotate_half) on q, k

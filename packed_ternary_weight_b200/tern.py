@@ -58,6 +58,8 @@ lib.tern_stream_read.argtypes = [_vp, _sz, ctypes.c_int32, ctypes.c_int32, ctype
 lib.tern_gemv_grouped.argtypes = [ctypes.c_int32, ctypes.POINTER(Desc), ctypes.POINTER(_vp), ctypes.c_int,
                                   ctypes.POINTER(_vp), ctypes.POINTER(_vp), ctypes.c_int, ctypes.POINTER(_vp), _vp]
 lib.tern_selftest_wait.argtypes = [ctypes.c_uint64, _vp]
+lib.tern_fit_tq.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp]
+lib.tern_fit_bt.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp, _vp]
 
 
 class DecodeModelC(ctypes.Structure):
@@ -73,7 +75,7 @@ lib.tern_decode_step.argtypes = [ctypes.POINTER(DecodeModelC), ctypes.c_int32, _
                                  ctypes.c_int32, _vp, _vp, _vp, _sz, _vp]
 for _f in (lib.tern_decode_rope_table, lib.tern_decode_workspace_size, lib.tern_decode_step):
     _f.restype = ctypes.c_int
-for _f in (lib.tern_selftest_wait, lib.tern_packed_size, lib.tern_pack, lib.tern_workspace_size, lib.tern_quantize_act, lib.tern_gemv,
+for _f in (lib.tern_selftest_wait, lib.tern_fit_tq, lib.tern_fit_bt, lib.tern_packed_size, lib.tern_pack, lib.tern_workspace_size, lib.tern_quantize_act, lib.tern_gemv,
            lib.tern_gemm_batched, lib.tern_device_error, lib.tern_gemv_noalloc, lib.tern_gemv_grouped,
            lib.tern_stream_read):
     _f.restype = ctypes.c_int
@@ -239,3 +241,16 @@ class DecodeModel:
         _check(lib.tern_decode_step(ctypes.byref(self.c), pos, _ptr(h_in), _ptr(h_out), first, last, _ptr(attn_in),
                                     _ptr(trace), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
                "tern_decode_step")
+
+
+def fit_tq(w, planes: int, group: int, trits, scales, stream=None):
+    """Fit fp32 device weights [n][k] into TQ planes: trits int8 [planes][n][k], scales fp16 [planes][n][k/group]."""
+    n, k = w.shape
+    _check(lib.tern_fit_tq(_ptr(w), n, k, planes, group, _ptr(trits), _ptr(scales), _stream(stream)), "tern_fit_tq")
+
+
+def fit_bt(w, depth: int, codebook, trits, idx, stream=None):
+    """Fit fp32 device weights [n][k] into balanced ternary: trits int8 [depth][n][k], idx uint8 [n][k/16]."""
+    n, k = w.shape
+    _check(lib.tern_fit_bt(_ptr(w), n, k, depth, _ptr(codebook), _ptr(trits), _ptr(idx), _stream(stream)),
+           "tern_fit_bt")
