@@ -53,13 +53,14 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
   const int P = L.planes;
   const int colk = bt3 ? kColK3 : kColK2;                      // k per column
   const int colb = bt3 ? bt_col_bytes(P) : P * kPlaneColBytes;  // bytes per column of a row tile
-  const int mt = gemv2_mt(xmode, m);
+  const int mt = bt3 ? gemv3_mt(m) : gemv2_mt(xmode, m);
   int rt_total = 0;
   for (int i = 0; i < nprob; ++i) rt_total += row_tiles[i];
   pl.wpc = 4;
   const int sc_target = std::max(gc, (4096 / colb) / gc * gc);
   const int ks_par = std::min(units, std::max(1, (12 * sms + rt_total - 1) / rt_total));
-  const int bpk = xmode == kXInt8 ? mt : xmode == kXBf16Q8 ? 3 * mt : 3;  // staged bytes per k
+  // staged bytes per k (bf16: the 24-bit image; balanced ternary: one per token)
+  const int bpk = xmode == kXInt8 ? mt : xmode == kXBf16Q8 ? 3 * mt : (bt3 ? 3 * mt : 3);
   int ks_x = 1;
   while (ks_x < units && (size_t)((units + ks_x - 1) / ks_x) * gc * colk * bpk > 96 * 1024) ++ks_x;
   int ks = std::max(ks_par, ks_x);
@@ -319,7 +320,6 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
   const int xmode = xmode_of(act);
   tern_status st = supported_2bit(L, xmode);
   if (st != TERN_OK) return st;
-  if (xmode == kXBf16 && m != 1) return TERN_EUNSUPPORTED;
   const int sms = device_sms();
   const uint8_t* base = static_cast<const uint8_t*>(d_packed);
   const bool pdl = (desc->flags & TERN_F_PDL) != 0;
@@ -440,7 +440,9 @@ tern_status run_single(const tern_desc* desc, const Layout& L, const void* d_pac
       }
     }
   }
-  const int mt_max = gemv2_mt(xmode, m);
+  // the row-group kernels: passes of up to 8 tokens (balanced ternary), 4 or
+  // 16 (integer activations) or one (bf16 activations over 2-bit planes)
+  const int mt_max = L.fmt == TERN_FMT_BT3 ? 8 : gemv2_mt(xmode, m);
   for (int t0 = 0; t0 < m; t0 += mt_max) {
     const int mc = std::min(mt_max, m - t0);
     const int rt = L.row_tiles;

@@ -53,26 +53,27 @@ __host__ __device__ inline Smem3 smem3_plan(const Gemv2Params& p) {
   Smem3 s{};
   const int kr = p.cols_per_split * kColK3;
   const int gr = kr / 16;
+  const size_t mt = (size_t)gemv3_mt(p.m);  // activation images: one per token, padded to 1, 2, 4 or 8
   s.stage_bytes = (int)align_up((size_t)p.stage_cols * bt_col_bytes(p.planes), 128);
   size_t off = 0;
   s.bars = off;
   off = align_up(off + (size_t)p.wpc * p.nstage * 8, 128);
   s.ring = off;
   off += (size_t)p.wpc * p.nstage * s.stage_bytes;
-  s.xa = off;
-  off = align_up(off + (size_t)kr, 128);
+  s.xa = off;  // [mt][kr] each
+  off = align_up(off + mt * kr, 128);
   s.xb = off;
-  off = align_up(off + (size_t)kr, 128);
+  off = align_up(off + mt * kr, 128);
   s.xc = off;
-  off = align_up(off + (size_t)kr, 128);
-  s.gsum = off;
-  off = align_up(off + (size_t)gr * 8, 16);
+  off = align_up(off + mt * kr, 128);
+  s.gsum = off;  // [mt][gr]
+  off = align_up(off + mt * gr * 8, 16);
   s.gmult = off;
-  off = align_up(off + (size_t)gr * 4, 16);
+  off = align_up(off + mt * gr * 4, 16);
   s.cb = off;
   off = align_up(off + 27 * 4, 16);
   s.red = off;
-  off = align_up(off + ((p.cluster && p.ks > 1) ? (size_t)p.ks * p.wpc * 32 * 4 : 0), 16);
+  off = align_up(off + ((p.cluster && p.ks > 1) ? (size_t)p.ks * mt * p.wpc * 32 * 4 : 0), 16);
   s.total = off;
   return s;
 }
@@ -92,7 +93,9 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
 }  // namespace
 
 // D: the depth (2, 3 or 4); the tuple of a row holds D bytes, the level bias is (3^D - 1) / 2.
-template <int D>
+// MT: tokens per launch (1, 2, 4 or 8; p.m of them are real): each column's
+// levels are decoded once and dotted with every token's activation image.
+template <int D, int MT>
 __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv2Params p) {
   static_assert(D >= 2 && D <= 4, "depth 2..4");
   constexpr int kColB = bt_col_bytes(D);
@@ -108,6 +111,9 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
   const int sc = p.stage_cols, nst = p.nstage;
   const int spt = (ncols + sc - 1) / sc;
   const int k0 = c0 * kColK3, kr = ncols * kColK3;
+  const int kr_img = p.cols_per_split * kColK3;  // per-token stride of the images
+  const int gr_img = kr_img / 16;
+  const int m = MT == 1 ? 1 : p.m;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + sp.bars) + warp * nst;
   uint8_t* ring = smem + sp.ring + (size_t)warp * nst * sp.stage_bytes;
 
@@ -173,7 +179,7 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
   int cur_prob = -1, nconsumed = 0, ifail = -1, pi = prob_of(gbeg);
   int cslot = 0;
   uint32_t cphase = 0;
-  float yacc = 0.f;
+  float yacc[MT];
   for (int gi = gbeg; gi < gend; ++gi) {
     while (pi + 1 < p.nprob && gi >= p.prob[pi + 1].cta_begin) ++pi;
     const Gemv2Problem& pr = p.prob[pi];
@@ -184,16 +190,19 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
       if (threadIdx.x < 27)
         reinterpret_cast<float*>(smem + sp.cb)[threadIdx.x] =
             reinterpret_cast<const float*>(pr.trit - kHeaderBytes + kCodebookOffset)[threadIdx.x];
-      gemv_common::stage_x_bf16_image(static_cast<const uint16_t*>(pr.x), p.k, 16, k0, kr,
-                                      reinterpret_cast<int8_t*>(smem + sp.xa), smem + sp.xb, smem + sp.xc,
-                                      reinterpret_cast<long long*>(smem + sp.gsum),
-                                      reinterpret_cast<float*>(smem + sp.gmult));
+      for (int t = 0; t < m; ++t)
+        gemv_common::stage_x_bf16_image(static_cast<const uint16_t*>(pr.x) + (size_t)t * p.k, p.k, 16, k0, kr,
+                                        reinterpret_cast<int8_t*>(smem + sp.xa) + (size_t)t * kr_img,
+                                        smem + sp.xb + (size_t)t * kr_img, smem + sp.xc + (size_t)t * kr_img,
+                                        reinterpret_cast<long long*>(smem + sp.gsum) + (size_t)t * gr_img,
+                                        reinterpret_cast<float*>(smem + sp.gmult) + (size_t)t * gr_img);
       __syncthreads();
       cur_prob = pi;
     }
     const int T = tile_of(gi, pi);
     const bool active = T < pr.row_tiles;
-    yacc = 0.f;
+#pragma unroll
+    for (int t = 0; t < MT; ++t) yacc[t] = 0.f;
     if (active && ifail < 0) {
       for (int s = 0; s < spt; ++s, ++nconsumed) {
         const int slot = cslot;
@@ -248,25 +257,31 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
           word_u(std::integral_constant<int, 3>{}, b0.w, b1.w, b2.w, b3.w);
 #pragma unroll
           for (int j = 0; j < 5; ++j) {
-            const uint32_t xo = kx + 16u * j;
-            const uint4 hv = lds128<0>(x32 + xo), mv = lds128<0>(xm32 + xo), lv = lds128<0>(xl32 + xo);
-            int H = 0;
-            unsigned M = 0, L = 0;
-            H = dp4a_us(U[0][j], (int)hv.x, H);
-            H = dp4a_us(U[1][j], (int)hv.y, H);
-            H = dp4a_us(U[2][j], (int)hv.z, H);
-            H = dp4a_us(U[3][j], (int)hv.w, H);
-            M = dp4a_uu(U[0][j], mv.x, M);
-            M = dp4a_uu(U[1][j], mv.y, M);
-            M = dp4a_uu(U[2][j], mv.z, M);
-            M = dp4a_uu(U[3][j], mv.w, M);
-            L = dp4a_uu(U[0][j], lv.x, L);
-            L = dp4a_uu(U[1][j], lv.y, L);
-            L = dp4a_uu(U[2][j], lv.z, L);
-            L = dp4a_uu(U[3][j], lv.w, L);
             const int g = (int)(kx >> 4) + j;  // group within the split
-            const long long S = ((long long)H * 65536 + (long long)M * 256 + L) - kBias * gsum[g];
-            yacc = fmaf(lds_f32(cb32 + 4u * ix[j]) * gmul[g], __ll2float_rn(S), yacc);
+            const float cbv = lds_f32(cb32 + 4u * ix[j]);
+#pragma unroll
+            for (int t = 0; t < MT; ++t) {
+              if (MT > 1 && t >= m) break;
+              const uint32_t xo = kx + 16u * j + (uint32_t)(t * kr_img);
+              const uint4 hv = lds128<0>(x32 + xo), mv = lds128<0>(xm32 + xo), lv = lds128<0>(xl32 + xo);
+              int H = 0;
+              unsigned M = 0, L = 0;
+              H = dp4a_us(U[0][j], (int)hv.x, H);
+              H = dp4a_us(U[1][j], (int)hv.y, H);
+              H = dp4a_us(U[2][j], (int)hv.z, H);
+              H = dp4a_us(U[3][j], (int)hv.w, H);
+              M = dp4a_uu(U[0][j], mv.x, M);
+              M = dp4a_uu(U[1][j], mv.y, M);
+              M = dp4a_uu(U[2][j], mv.z, M);
+              M = dp4a_uu(U[3][j], mv.w, M);
+              L = dp4a_uu(U[0][j], lv.x, L);
+              L = dp4a_uu(U[1][j], lv.y, L);
+              L = dp4a_uu(U[2][j], lv.z, L);
+              L = dp4a_uu(U[3][j], lv.w, L);
+              const int gt = g + t * gr_img;
+              const long long S = ((long long)H * 65536 + (long long)M * 256 + L) - kBias * gsum[gt];
+              yacc[t] = fmaf(cbv * gmul[gt], __ll2float_rn(S), yacc[t]);
+            }
           }
         }
         fence_proxy_async_smem();
@@ -276,15 +291,19 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
     }
 
     const int row = T * kTileRows + lane;
-    auto write_out = [&](float v) {
+    auto write_out = [&](int t, float v) {
       if (row >= pr.n) return;
+      const size_t o = (size_t)t * pr.n + row;
       if (p.out_bf16)
-        reinterpret_cast<__nv_bfloat16*>(pr.y)[row] = __float2bfloat16_rn(v);
+        reinterpret_cast<__nv_bfloat16*>(pr.y)[o] = __float2bfloat16_rn(v);
       else
-        reinterpret_cast<float*>(pr.y)[row] = v;
+        reinterpret_cast<float*>(pr.y)[o] = v;
     };
     if (p.ks == 1) {
-      if (active) write_out(yacc);
+      if (active)
+#pragma unroll
+        for (int t = 0; t < MT; ++t)
+          if (t < m) write_out(t, yacc[t]);
       continue;
     }
     if (active && ifail >= 0) {
@@ -294,15 +313,23 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
     // K is split: the splits of this row group form the cluster; reduce in rank 0
     const int rows_cta = p.wpc * kTileRows;
     if (active) {
-      const size_t idx = (size_t)split * rows_cta + warp * kTileRows + lane;
-      st_cluster_u32(map_cluster_rank(smem_u32(smem + sp.red + idx * 4), 0), __float_as_uint(yacc));
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        if (t >= m) break;
+        const size_t idx = ((size_t)split * MT + t) * rows_cta + warp * kTileRows + lane;
+        st_cluster_u32(map_cluster_rank(smem_u32(smem + sp.red + idx * 4), 0), __float_as_uint(yacc[t]));
+      }
     }
     cluster_sync();
     if (split == 0 && active) {
-      float sf = 0.f;
-      for (int s = 0; s < p.ks; ++s)
-        sf += reinterpret_cast<const float*>(smem + sp.red)[(size_t)s * rows_cta + warp * kTileRows + lane];
-      write_out(sf);
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        if (t >= m) break;
+        float sf = 0.f;
+        for (int s = 0; s < p.ks; ++s)
+          sf += reinterpret_cast<const float*>(smem + sp.red)[((size_t)s * MT + t) * rows_cta + warp * kTileRows + lane];
+        write_out(t, sf);
+      }
     }
     return;
   }
@@ -314,9 +341,17 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
 size_t gemv3_smem_bytes(const Gemv2Params& p) { return smem3_plan(p).total; }
 
 int launch_gemv3(const Gemv2Params& p, bool pdl, void* stream) {
-  if (p.m != 1 || (p.ks > 1 && !p.cluster) || p.planes < 2 || p.planes > 4) return -1;
+  if (p.m < 1 || p.m > 8 || (p.ks > 1 && !p.cluster) || p.planes < 2 || p.planes > 4) return -1;
   const Smem3 sp = smem3_plan(p);
-  auto kern = p.planes == 2 ? gemv3_kernel<2> : (p.planes == 3 ? gemv3_kernel<3> : gemv3_kernel<4>);
+  auto pick = [](int d, auto mt_c) {
+    constexpr int T = decltype(mt_c)::value;
+    return d == 2 ? gemv3_kernel<2, T> : (d == 3 ? gemv3_kernel<3, T> : gemv3_kernel<4, T>);
+  };
+  const int mt = gemv3_mt(p.m);
+  auto kern = mt == 1   ? pick(p.planes, std::integral_constant<int, 1>{})
+              : mt == 2 ? pick(p.planes, std::integral_constant<int, 2>{})
+              : mt == 4 ? pick(p.planes, std::integral_constant<int, 4>{})
+                        : pick(p.planes, std::integral_constant<int, 8>{});
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp.total);
   if (e != cudaSuccess) return (int)e;
   const bool clus = p.cluster && p.ks > 1;

@@ -248,7 +248,9 @@ int read_clear_dev_error_gemv2(void* stream, unsigned* out);
 int read_clear_dev_error_stream(void* stream, unsigned* out);
 int read_clear_dev_error_gemv3(void* stream, unsigned* out);
 int read_clear_dev_error_selftest(void* stream, unsigned* out);
-int launch_gemv3(const Gemv2Params& p, bool pdl, void* stream);  // balanced ternary d = 3, bf16 x, m = 1
+int launch_gemv3(const Gemv2Params& p, bool pdl, void* stream);  // balanced ternary, bf16 x, m = 1..8
+// tokens per launch of the balanced-ternary kernel: m padded to 1, 2, 4 or 8
+TERN_HD inline int gemv3_mt(int m) { return m <= 1 ? 1 : (m <= 2 ? 2 : (m <= 4 ? 4 : 8)); }
 size_t gemv3_smem_bytes(const Gemv2Params& p);
 int launch_stream_read(const void* src, size_t bytes, int mode, int chunk, int depth, int ctas_per_sm, int warps,
                        unsigned* sink, void* stream);
