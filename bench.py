@@ -620,7 +620,14 @@ def run_config(args, name=None):
         pk = torch.from_numpy(buf).cuda()
         packs = [pk] + [pk.clone() for _ in range(copies - 1)]
         del lay.trits
-        tokens = synth.PREFILL_TOKENS if name == "tq2p" else (1,)
+        if name == "tq2p":
+            tokens = synth.PREFILL_TOKENS
+        elif name == "bt3" and lay.name in ("q_proj", "gate_proj"):
+            tokens = (1, 2, 4, 8)        # weights read once for the tokens of a pass
+        elif name == "tq3p" and lay.name == "gate_proj":
+            tokens = (1, 2)              # bf16 over 2-bit planes: one pass per token
+        else:
+            tokens = (1,)
         for m in tokens:
             x = synth.draw_x_bf16(lay.seed, m, lay.k)
             xd = torch.from_numpy(x.view(np.int16)).cuda()
@@ -721,6 +728,36 @@ def run_config(args, name=None):
     return out
 
 
+def run_fit(args):
+    """Dense -> ternary fits on the GPU of a Llama-3.1-8B gate_proj-shaped fp32 matrix (14336 x 4096,
+    N(0, 0.02^2)): TQ3P at g = 256 and balanced ternary d = 3, time per matrix (CUDA events)."""
+    import torch
+
+    from packed_ternary_weight_b200 import tern
+    n, k = 14336, 4096
+    g = torch.Generator(device="cuda").manual_seed(5)
+    w = torch.randn((n, k), device="cuda", generator=g) * 0.02
+    out = {"shape": "%dx%d fp32" % (n, k)}
+    t3 = torch.empty((3, n, k), dtype=torch.int8, device="cuda")
+    s3 = torch.empty((3, n, k // 256), dtype=torch.int16, device="cuda")
+    ix = torch.empty((n, k // 16), dtype=torch.uint8, device="cuda")
+    cb = torch.from_numpy(synth.codebook27()).cuda()
+    for nm, fn in (("tq3p_g256", lambda: tern.fit_tq(w, 3, 256, t3, s3)),
+                   ("bt_d3", lambda: tern.fit_bt(w, 3, cb, t3, ix))):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(3):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / 3
+        out[nm] = {"ms_per_matrix": round(ms, 3), "gweights_per_s": round(n * k / (ms * 1e-3) / 1e9, 2)}
+    assert tern.device_error() == tern.OK
+    return out
+
+
 def run_all_configs(args):
     """The other workloads' per-shape rows, for the default bench line, with the SM clock sampled
     while they run."""
@@ -730,6 +767,7 @@ def run_all_configs(args):
     for v in out.values():
         v.pop("metric", None)
         v.pop("peak", None)
+    out["fit"] = run_fit(args)
     out["seconds"] = round(time.time() - t0, 1)
     clk = clocks.stop()
     if clk is not None:
