@@ -403,30 +403,64 @@ def run_ours(args, rank, world):
     decode = run_decode(tern, torch, stream, {(L["layer"], L["name"]): L["packed"] for L in layers}, args.layers,
                         reps=max(3, min(args.steps, 100)), clocks=not args.no_clocks and rank == 0)
 
-    # end to end through the public API: pinned H2D of the step's activations,
-    # the captured step, D2H of the step's outputs
+    # end to end through the public API, pipelined as a server runs it: every
+    # step copies its bf16 activations in from pinned host memory and its fp32
+    # outputs back out; step i's input copy (copy stream) overlaps step i-1's
+    # compute, and step i-1's output copy (another copy stream) overlaps step
+    # i's; two device buffer sets alternate, each reused only after the copies
+    # that read or fill it have finished
     h2d = x_all_host.numel() * 2
     d2h = y_all_host.numel() * 4
+    x_b = [x_all, torch.empty_like(x_all)]
+    y_b = [y_all, torch.empty_like(y_all)]
+    x_h = [x_all_host, x_all_host.clone().pin_memory()]
+    y_h = [y_all_host, torch.empty_like(y_all_host).pin_memory()]
+
+    def step_on(xbuf, ybuf):
+        Ls = sorted(layers, key=lambda L: L["k"])
+        return tern.Grouped([L["desc"] for L in Ls], [L["packed"] for L in Ls], tern.ACT_BF16_Q8,
+                            [xbuf[L["xoff"]:L["xoff"] + L["k"]] for L in Ls], None, tern.OUT_F32,
+                            [ybuf[L["yoff"]:L["yoff"] + L["n"]] for L in Ls])
+
     with torch.cuda.stream(stream):
-        def e2e_step():
-            x_all.copy_(x_all_host, non_blocking=True)
-            g_step.replay()
-            y_all_host.copy_(y_all, non_blocking=True)
-        for _ in range(3):
-            e2e_step()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        ms_e2e = e0.elapsed_time(e1) / reps
-    ms_e2e = max_over_ranks(ms_e2e, world, dev)
+        g_b = [g_step, capture(lambda g=step_on(x_b[1], y_b[1]): g.launch(stream))]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = {k: [torch.cuda.Event(), torch.cuda.Event()] for k in ("in", "done", "out")}
+
+    def e2e_pipeline(n):
+        for i in range(n):
+            b = i & 1
+            if i >= 2:
+                s_in.wait_event(ev["done"][b])          # step i-2 has read x_b[b]
+            with torch.cuda.stream(s_in):
+                x_b[b].copy_(x_h[b], non_blocking=True)
+                ev["in"][b].record(s_in)
+            stream.wait_event(ev["in"][b])
+            if i >= 2:
+                stream.wait_event(ev["out"][b])         # step i-2's outputs have left y_b[b]
+            with torch.cuda.stream(stream):
+                g_b[b].replay()
+                ev["done"][b].record(stream)
+            s_out.wait_event(ev["done"][b])
+            with torch.cuda.stream(s_out):
+                y_h[b].copy_(y_b[b], non_blocking=True)
+                ev["out"][b].record(s_out)
+
+    e2e_pipeline(3)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(s_in)
+    e2e_pipeline(reps)
+    s_out.wait_event(ev["out"][(reps - 1) & 1])
+    e1.record(s_out)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / reps, world, dev)
     assert tern.device_error(stream) == tern.OK
+    # the last step's outputs reached the host intact
+    e2e_ok = bool(torch.equal(y_h[(reps - 1) & 1], y_all.cpu())) if rank == 0 else None
 
     value = replica_gbs(step_bytes, ms_step, world)
     achieved = step_bytes / (ms_step * 1e-3) / 1e9     # every launch of the step is the GEMV kernel
@@ -473,7 +507,11 @@ def run_ours(args, rank, world):
                                         "tokens per second = steps per second, summed over replicas"},
         "decode_step": decode,
         "e2e": {"value": round(replica_gbs(step_bytes, ms_e2e, world), 1), "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4),
+                "pipeline": "per step: pinned H2D of the bf16 activations (copy stream), the captured step, D2H "
+                            "of the fp32 outputs (second copy stream); two buffer sets, copies of step i "
+                            "overlapping the compute of steps i-1 and i+1",
+                "outputs_match": e2e_ok},
         "gpu_launches": args.steps * len(step_launches),
         "parity_bit_exact": parity,
         "parity_sample": "%d rows of each of %s in the timed launch, against the oracle" % (

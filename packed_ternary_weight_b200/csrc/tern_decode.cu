@@ -75,7 +75,7 @@ constexpr int kDT = 32 * kDW;            // consumer threads
 constexpr int kDBlock = kDT + 32;        // + the producer warp
 constexpr int kChunkCols = 16;           // 64-k columns per ring slot
 constexpr int kSlotBytes = kChunkCols * kPlaneColBytes;  // 8 KB
-constexpr int kKvPass = 32;              // cached positions per attention pass
+constexpr int kKvPass = 64;              // cached positions per attention pass (a whole range up to ~1,850 positions)
 constexpr int kHD = kDecHeadDim;         // 128
 constexpr int kBarNamed = 1;             // named barrier of the consumer threads
 
@@ -803,52 +803,76 @@ __global__ void __launch_bounds__(kDBlock, 1) decode_kernel(const __grid_constan
   };
 
   // ---- combine the ranges' states (after the attention's grid barrier): CTA
-  // c finishes outputs [c * HQ / G, (c + 1) * HQ / G) of the attention, one
-  // warp per output and a lane per position range: each lane loads its
-  // ranges' (maximum, sum, weighted value) in one round, folds them in order,
-  // and the lanes' states merge by a fixed butterfly
+  // c finishes outputs [c * HQ / G, (c + 1) * HQ / G) of the attention, a warp
+  // per output and a lane per position range: each lane loads its ranges'
+  // (maximum, sum, weighted value) in one round, folds them in order, and the
+  // lanes' states merge by a fixed butterfly
   auto combine_stage = [&](int layer) {
     const int o0 = (int)((long long)HQ * cta / G), o1 = (int)((long long)HQ * (cta + 1) / G);
     const float* Pa = reinterpret_cast<const float*>(p.ws + p.off_att);
     float* outp = reinterpret_cast<float*>(p.ws + p.off_attn);
     const size_t stride = (size_t)rep * (kHD + 2);
-    for (int out = o0 + warp; out < o1; out += kDW) {
-      const int h = out / kHD, d = out - h * kHD;
-      const int jj = h / rep, r = h - jj * rep;
-      const float* e0 = Pa + ((size_t)jj * ns * rep + r) * (kHD + 2);
-      float M = -INFINITY, L = 0.f, O = 0.f;
+    // two outputs per warp per trip, their loads issued together
+    for (int out0 = o0 + warp; out0 < o1; out0 += 2 * kDW) {
+      float M[2], L[2], O[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        M[u] = -INFINITY;
+        L[u] = 0.f;
+        O[u] = 0.f;
+      }
       for (int s0 = 0; s0 < ns; s0 += 32) {
         const int s2 = s0 + lane;
-        float ms = -INFINITY, ls = 0.f, os = 0.f;
-        if (s2 < ns) {
-          const float* e = e0 + s2 * stride;
-          ms = __ldcg(e);
-          ls = __ldcg(e + 1);
-          os = __ldcg(e + 2 + d);
+        float ms[2], ls[2], os[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int out = out0 + u * kDW;
+          ms[u] = -INFINITY;
+          ls[u] = 0.f;
+          os[u] = 0.f;
+          if (s2 < ns && out < o1) {
+            const int h = out / kHD, d = out - h * kHD;
+            const int jj = h / rep, r = h - jj * rep;
+            const float* e = Pa + ((size_t)jj * ns * rep + r) * (kHD + 2) + s2 * stride;
+            ms[u] = __ldcg(e);
+            ls[u] = __ldcg(e + 1);
+            os[u] = __ldcg(e + 2 + d);
+          }
         }
-        if (ls != 0.f) {
-          const float mn = fmaxf(M, ms);
-          const float a = exp2f(M - mn), b = exp2f(ms - mn);
-          L = fmaf(L, a, ls * b);
-          O = fmaf(O, a, os * b);
-          M = mn;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (ls[u] != 0.f) {
+            const float mn = fmaxf(M[u], ms[u]);
+            const float a = exp2f(M[u] - mn), b = exp2f(ms[u] - mn);
+            L[u] = fmaf(L[u], a, ls[u] * b);
+            O[u] = fmaf(O[u], a, os[u] * b);
+            M[u] = mn;
+          }
         }
       }
 #pragma unroll
       for (int o = 16; o; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, M, o);
-        const float l2 = __shfl_xor_sync(0xffffffffu, L, o);
-        const float p2 = __shfl_xor_sync(0xffffffffu, O, o);
-        const float mn = fmaxf(M, m2);
-        const float a = L != 0.f ? exp2f(M - mn) : 0.f, b = l2 != 0.f ? exp2f(m2 - mn) : 0.f;
-        L = fmaf(L, a, l2 * b);
-        O = fmaf(O, a, p2 * b);
-        M = mn;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const float m2 = __shfl_xor_sync(0xffffffffu, M[u], o);
+          const float l2 = __shfl_xor_sync(0xffffffffu, L[u], o);
+          const float p2 = __shfl_xor_sync(0xffffffffu, O[u], o);
+          const float mn = fmaxf(M[u], m2);
+          const float a = L[u] != 0.f ? exp2f(M[u] - mn) : 0.f, b = l2 != 0.f ? exp2f(m2 - mn) : 0.f;
+          L[u] = fmaf(L[u], a, l2 * b);
+          O[u] = fmaf(O[u], a, p2 * b);
+          M[u] = mn;
+        }
       }
       if (lane == 0) {
-        const float val = O / L;
-        outp[out] = val;
-        if (p.trace) p.trace[(size_t)layer * p.trace_stride + HQ + 2 * KVH * kHD + out] = val;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int out = out0 + u * kDW;
+          if (out >= o1) break;
+          const float val = O[u] / L[u];
+          outp[out] = val;
+          if (p.trace) p.trace[(size_t)layer * p.trace_stride + HQ + 2 * KVH * kHD + out] = val;
+        }
       }
     }
   };

@@ -124,8 +124,8 @@ def test_qkv_rope_cache_and_attention(tern, shape, pos, max_pos):
 
 
 def test_attention_long_context_passes(tern):
-    # one KV head: the 148 position ranges hold more than 32 cached positions each (several passes)
-    m = synth.decode_model(D=256, F=256, H=2, KVH=1, n_layers=1, pos=6000, max_pos=6001, seed=70)
+    # one KV head: the 148 position ranges hold more than 64 cached positions each (several passes)
+    m = synth.decode_model(D=256, F=256, H=2, KVH=1, n_layers=1, pos=12000, max_pos=12001, seed=70)
     s = Setup(tern, m)
     s.run(tern, m.h0, first=0, last=1)
     rec = {}
