@@ -210,34 +210,42 @@ __device__ __forceinline__ uint32_t f32_to_bf16_rn(float v) {
   return (b + 0x7FFFu + ((b >> 16) & 1u)) >> 16;
 }
 
+// `bar` counts barrier arrivals; its top bit is the abort flag, so that one
+// load tells a waiting CTA both whether the barrier has opened and whether
+// some CTA gave up.
 struct DecCtl {
-  unsigned bar, exitc, abort, pad;
+  unsigned bar, exitc, pad0, pad1;
 };
+constexpr unsigned kAbortBit = 0x80000000u;
+
+__device__ __noinline__ void raise_abort(DecCtl* ctl) {
+  atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
+  atomicOr(&ctl->bar, kAbortBit);
+}
+__device__ __forceinline__ bool aborted(const DecCtl* ctl) { return (ld_acquire_u32(&ctl->bar) & kAbortBit) != 0u; }
 
 // Grid barrier over the consumer threads of every CTA (bounded). Returns false
 // if a CTA gave up (timeout here or elsewhere).
 __device__ bool grid_sync(DecCtl* ctl, unsigned& epoch, volatile int* s_ok) {
   named_sync();
   if (threadIdx.x == 0) {
-    bool ok = ld_acquire_u32(&ctl->abort) == 0u;
-    if (ok) {
-      red_release_add(&ctl->bar, 1u);
-      const unsigned target = (epoch + 1u) * gridDim.x;
-      uint64_t t0 = 0;
-      for (uint32_t it = 0;; ++it) {
-        if (ld_acquire_u32(&ctl->bar) >= target) break;
-        if ((it & 63u) == 63u) {
-          if (t0 == 0) t0 = global_timer_ns();
-          if (ld_acquire_u32(&ctl->abort) != 0u) {
-            ok = false;
-            break;
-          }
-          if (global_timer_ns() - t0 > kWaitLimitNs) {
-            atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
-            atomicExch(&ctl->abort, 1u);
-            ok = false;
-            break;
-          }
+    bool ok = true;
+    red_release_add(&ctl->bar, 1u);
+    const unsigned target = (epoch + 1u) * gridDim.x;
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+      const unsigned v = ld_acquire_u32(&ctl->bar);
+      if (v & kAbortBit) {
+        ok = false;
+        break;
+      }
+      if (v >= target) break;
+      if ((it & 63u) == 63u) {
+        if (t0 == 0) t0 = global_timer_ns();
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          raise_abort(ctl);
+          ok = false;
+          break;
         }
       }
     }
@@ -246,11 +254,6 @@ __device__ bool grid_sync(DecCtl* ctl, unsigned& epoch, volatile int* s_ok) {
   ++epoch;
   named_sync();
   return *s_ok != 0;
-}
-
-__device__ void raise_abort(DecCtl* ctl) {
-  atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
-  atomicExch(&ctl->abort, 1u);
 }
 
 // Sum / maximum over the consumer threads in a fixed order (butterfly in the
@@ -370,6 +373,12 @@ __global__ void __launch_bounds__(kDBlock, 1) decode_kernel(const __grid_constan
     bool ok = true;
     unsigned nkv = 0;  // first passes of cached keys and values issued
     for (int si = p.first; si <= p.last && ok; ++si) {
+      // once per stage: a CTA that gave up stops the copies (a wait below that
+      // the consumers no longer answer ends at its own limit)
+      if (aborted(ctl)) {
+        ok = false;
+        break;
+      }
       const int gt = dec_gemv_of(si);
       if (gt < 0) {
         // this layer's cached keys and values, pass by pass, into the KV buffer
@@ -377,10 +386,6 @@ __global__ void __launch_bounds__(kDBlock, 1) decode_kernel(const __grid_constan
         const int ncached = kv_cached(p, cta);
         for (int base = 0; base < ncached && ok; base += kKvPass) {
           if (nkv > 0 && !mbar_wait_bounded(kvbar + 1, (nkv - 1u) & 1u)) {
-            ok = false;
-            break;
-          }
-          if (ld_acquire_u32(&ctl->abort) != 0u) {
             ok = false;
             break;
           }
@@ -405,10 +410,6 @@ __global__ void __launch_bounds__(kDBlock, 1) decode_kernel(const __grid_constan
             ok = false;
             break;
           }
-          if (ld_acquire_u32(&ctl->abort) != 0u) {
-            ok = false;
-            break;
-          }
           const uint32_t bytes = (uint32_t)nc * kPlaneColBytes;
           mbar_arrive_expect_tx(&full[slot], bytes);
           bulk_g2s(ring + (size_t)slot * kSlotBytes, tr + ((size_t)tt * S.cols + c) * kPlaneColBytes, bytes,
@@ -417,7 +418,7 @@ __global__ void __launch_bounds__(kDBlock, 1) decode_kernel(const __grid_constan
         }
       }
     }
-    if (!ok) atomicExch(&ctl->abort, 1u);
+    if (!ok) raise_abort(ctl);
     // every copy this warp issued has landed before the CTA can exit (bounded;
     // immediate on the normal path, where the consumers have used them all)
     const unsigned lo = n > (unsigned)nslot ? n - (unsigned)nslot : 0u;

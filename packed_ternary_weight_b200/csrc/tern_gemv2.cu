@@ -63,7 +63,7 @@ constexpr uint32_t kM03 = 0x03030303u;
 constexpr uint32_t kM30 = 0x30303030u;
 
 struct SmemPlan {
-  size_t bars, ring, xa, xb, xc, xraw, gsum, gmult, red, amx, misc, total;
+  size_t bars, cbar, ring, xa, xb, xc, xraw, gsum, gmult, red, amx, misc, total;
   int stage_bytes;
 };
 
@@ -82,7 +82,9 @@ __host__ __device__ inline SmemPlan smem_plan(const Gemv2Params& p, int xmode, i
   const bool bf = xmode == kXBf16;
   size_t off = 0;
   s.bars = off;
-  off = align_up(off + (size_t)p.wpc * p.nstage * 8, 128);
+  off += (size_t)p.wpc * p.nstage * 8;
+  s.cbar = off;  // K split over a cluster: [0] the splits' token maxima arrived, [1] their partial sums
+  off = align_up(off + 16, 128);
   s.ring = off;
   off += (size_t)p.wpc * p.nstage * s.stage_bytes;
   s.xa = off;  // int8 x [mt][kr], or the signed high byte of the bf16 image [kr]
@@ -175,7 +177,8 @@ __device__ __forceinline__ float bf16_abs_max8(uint4 v) {
 }
 
 // In-kernel per-token absmax quantisation (same rule as tern_quantize_act):
-// the token maxima of all K-splits are exchanged through the cluster.
+// every split sends its token maxima to every CTA of the cluster with
+// st.async, and each CTA waits for them on its own barrier.
 template <int MT>
 __device__ void stage_x_q8(const Gemv2Params& p, const Gemv2Problem& pr, const SmemPlan& sp, uint8_t* smem, int k0,
                            int kr, int gsz, bool clus, int split) {
@@ -219,21 +222,23 @@ __device__ void stage_x_q8(const Gemv2Params& p, const Gemv2Problem& pr, const S
   }
   __syncthreads();
   if (clus) {
+    uint64_t* xbar = reinterpret_cast<uint64_t*>(smem + sp.cbar);
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(xbar, (uint32_t)(p.ks * MT * 4));
     for (int i = threadIdx.x; i < p.ks * MT; i += blockDim.x) {
       const int r = i / MT, t = i - r * MT;
-      st_cluster_u32(map_cluster_rank(smem_u32(&amx[split * MT + t]), (uint32_t)r), tmax[t]);
+      st_async_u32(map_cluster_rank(smem_u32(&amx[split * MT + t]), (uint32_t)r), tmax[t],
+                   map_cluster_rank(smem_u32(xbar), (uint32_t)r));
     }
-    cluster_sync();
-  } else {
-    if (threadIdx.x < MT) amx[threadIdx.x] = __uint_as_float(tmax[threadIdx.x]);
-    __syncthreads();
+    (void)mbar_wait_bounded<true>(xbar, 0);  // on expiry the error word records a timeout
   }
-  const int nsp = clus ? p.ks : 1;
   float inv[MT];
+  const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int t = 0; t < MT; ++t) {
-    float a = 0.f;
-    for (int r = 0; r < nsp; ++r) a = fmaxf(a, amx[r * MT + t]);
+    // maxima are non-negative floats: their bit patterns order like the values
+    unsigned ab = tmax[t];
+    if (clus) ab = __reduce_max_sync(0xffffffffu, lane < p.ks ? __float_as_uint(amx[lane * MT + t]) : 0u);
+    const float a = __uint_as_float(ab);
     inv[t] = a > 0.f ? __fdiv_rn(127.0f, a) : 0.f;
     if (threadIdx.x == 0) sxs[t] = a > 0.f ? __fdiv_rn(a, 127.0f) : 0.f;
   }
@@ -320,7 +325,15 @@ __global__ void __launch_bounds__(256) gemv2_kernel(const __grid_constant__ Gemv
   auto tile_of = [&](int gi, int q) { return (gi - p.prob[q].cta_begin) * p.wpc + warp; };
 
   // ---- prologue (independent of the preceding kernel): barriers, first weight stages
-  if (clus) cluster_arrive_relaxed();  // DSMEM is used only after every CTA of the cluster runs
+  if (clus && threadIdx.x == 0) {
+    uint64_t* cbar = reinterpret_cast<uint64_t*>(smem + sp.cbar);
+    mbar_init(cbar, 1);      // the token maxima (in-kernel quantisation)
+    mbar_init(cbar + 1, 1);  // the splits' partial sums (rank 0)
+    fence_mbar_init();
+  }
+  // other CTAs store into this one's shared memory only after every CTA of the
+  // cluster runs and has initialised its barriers
+  if (clus) cluster_arrive_relaxed();
   if (lane == 0) {
     for (int s = 0; s < nst; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
@@ -611,41 +624,53 @@ __global__ void __launch_bounds__(256) gemv2_kernel(const __grid_constant__ Gemv
         mbar_wait_bounded(&bars[j % nst], (uint32_t)(j / nst) & 1u);  // error path only
     }
     if (clus) {
-      // the splits of this row group form the cluster: reduce in CTA rank 0
+      // the splits of this row group form the cluster: each sends its partial
+      // sums to CTA rank 0 with st.async, which waits for them on its own
+      // barrier, sums them in split order and writes the outputs; the other
+      // CTAs are then done
       const int rows_cta = p.wpc * kTileRows;
       const int esz = red_elem(XM, kTQ);
+      uint64_t* rbar = reinterpret_cast<uint64_t*>(smem + sp.cbar) + 1;
+      if (split == 0 && threadIdx.x == 0) {
+        // every split's partials of the active warps (the same warps in every split)
+        const int nact = max(0, min(p.wpc, pr.row_tiles - (T - warp)));
+        mbar_arrive_expect_tx(rbar, (uint32_t)(p.ks * m * nact * kTileRows * esz));
+      }
       if (active) {
+        const uint32_t rbar0 = map_cluster_rank(smem_u32(rbar), 0);
 #pragma unroll
         for (int t = 0; t < MT; ++t) {
           if (t >= m) continue;
           const size_t idx = ((size_t)split * MT + t) * rows_cta + warp * kTileRows + lane;
           const uint32_t dst = map_cluster_rank(smem_u32(smem + sp.red + idx * esz), 0);
           if (XM == kXBf16)
-            st_cluster_u32(dst, __float_as_uint(yacc));
+            st_async_u32(dst, __float_as_uint(yacc), rbar0);
           else if (kTQ)
-            st_cluster_u64(dst, (unsigned long long)acc64[t]);
+            st_async_u64(dst, (unsigned long long)acc64[t], rbar0);
           else
-            st_cluster_u32(dst, (uint32_t)accb[t]);
+            st_async_u32(dst, (uint32_t)accb[t], rbar0);
         }
       }
-      cluster_sync();
-      if (split == 0 && active) {
+      if (split == 0) {
+        (void)mbar_wait_bounded<true>(rbar, 0);  // on expiry the error word records a timeout
+        if (active) {
 #pragma unroll
-        for (int t = 0; t < MT; ++t) {
-          if (t >= m) continue;
-          long long s64 = 0;
-          int s32 = 0;
-          float sf = 0.f;
-          for (int s = 0; s < p.ks; ++s) {
-            const size_t idx = ((size_t)s * MT + t) * rows_cta + warp * kTileRows + lane;
-            if (XM == kXBf16)
-              sf += reinterpret_cast<const float*>(smem + sp.red)[idx];
-            else if (kTQ)
-              s64 += reinterpret_cast<const long long*>(smem + sp.red)[idx];
-            else
-              s32 += reinterpret_cast<const int*>(smem + sp.red)[idx];
+          for (int t = 0; t < MT; ++t) {
+            if (t >= m) continue;
+            long long s64 = 0;
+            int s32 = 0;
+            float sf = 0.f;
+            for (int s = 0; s < p.ks; ++s) {
+              const size_t idx = ((size_t)s * MT + t) * rows_cta + warp * kTileRows + lane;
+              if (XM == kXBf16)
+                sf += reinterpret_cast<const float*>(smem + sp.red)[idx];
+              else if (kTQ)
+                s64 += reinterpret_cast<const long long*>(smem + sp.red)[idx];
+              else
+                s32 += reinterpret_cast<const int*>(smem + sp.red)[idx];
+            }
+            finish(t, s64, s32, sf);
           }
-          finish(t, s64, s32, sf);
         }
       }
       return;

@@ -45,7 +45,7 @@ using gemv_common::align_up;
 using gemv_common::triple_levels;
 
 struct Smem3 {
-  size_t bars, ring, xa, xb, xc, gsum, gmult, cb, red, total;
+  size_t bars, cbar, ring, xa, xb, xc, gsum, gmult, cb, red, total;
   int stage_bytes;
 };
 
@@ -57,7 +57,9 @@ __host__ __device__ inline Smem3 smem3_plan(const Gemv2Params& p) {
   s.stage_bytes = (int)align_up((size_t)p.stage_cols * bt_col_bytes(p.planes), 128);
   size_t off = 0;
   s.bars = off;
-  off = align_up(off + (size_t)p.wpc * p.nstage * 8, 128);
+  off += (size_t)p.wpc * p.nstage * 8;
+  s.cbar = off;  // K split over a cluster: the splits' partial sums arrived (rank 0)
+  off = align_up(off + 8, 128);
   s.ring = off;
   off += (size_t)p.wpc * p.nstage * s.stage_bytes;
   s.xa = off;  // [mt][kr] each
@@ -130,6 +132,12 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
   auto tile_of = [&](int gi, int q) { return (gi - p.prob[q].cta_begin) * p.wpc + warp; };
 
   // ---- prologue: barriers, first weight stages
+  if (clus && threadIdx.x == 0) {
+    mbar_init(reinterpret_cast<uint64_t*>(smem + sp.cbar), 1);
+    fence_mbar_init();
+  }
+  // other CTAs store into this one's shared memory only after every CTA of the
+  // cluster runs and has initialised its barrier
   if (clus) cluster_arrive_relaxed();
   if (lane == 0) {
     for (int s = 0; s < nst; ++s) mbar_init(&bars[s], 1);
@@ -310,17 +318,26 @@ __global__ void __launch_bounds__(256) gemv3_kernel(const __grid_constant__ Gemv
       for (int j = ifail; j < min(nissued, ifail + nst); ++j)
         mbar_wait_bounded(&bars[j % nst], (uint32_t)(j / nst) & 1u);  // error path only
     }
-    // K is split: the splits of this row group form the cluster; reduce in rank 0
+    // K is split: the splits of this row group form the cluster. Each sends
+    // its partial sums to CTA rank 0 with st.async; rank 0 waits for them on
+    // its own barrier and sums them in split order, the others are done.
     const int rows_cta = p.wpc * kTileRows;
+    uint64_t* rbar = reinterpret_cast<uint64_t*>(smem + sp.cbar);
+    if (split == 0 && threadIdx.x == 0) {
+      // every split's partials of the active warps (the same warps in every split)
+      const int nact = max(0, min(p.wpc, pr.row_tiles - (T - warp)));
+      mbar_arrive_expect_tx(rbar, (uint32_t)(p.ks * m * nact * kTileRows * 4));
+    }
     if (active) {
+      const uint32_t rbar0 = map_cluster_rank(smem_u32(rbar), 0);
 #pragma unroll
       for (int t = 0; t < MT; ++t) {
         if (t >= m) break;
         const size_t idx = ((size_t)split * MT + t) * rows_cta + warp * kTileRows + lane;
-        st_cluster_u32(map_cluster_rank(smem_u32(smem + sp.red + idx * 4), 0), __float_as_uint(yacc[t]));
+        st_async_u32(map_cluster_rank(smem_u32(smem + sp.red + idx * 4), 0), __float_as_uint(yacc[t]), rbar0);
       }
     }
-    cluster_sync();
+    if (split == 0) (void)mbar_wait_bounded<true>(rbar, 0);  // on expiry the error word records a timeout
     if (split == 0 && active) {
 #pragma unroll
       for (int t = 0; t < MT; ++t) {

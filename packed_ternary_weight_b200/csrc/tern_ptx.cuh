@@ -70,15 +70,27 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
 // One potentially blocking test of the phase: the thread may be suspended
 // for up to about 0.5 ms waiting for the phase to complete (so a waiting warp
 // does not spin on the issue slots).
+// kCluster: acquire at cluster scope, for phases that other CTAs' st.async
+// stores complete.
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(500000u)
-      : "memory");
+  if constexpr (kCluster)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(500000u)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(500000u)
+        : "memory");
   return ok != 0;
 }
 
@@ -94,14 +106,15 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // the stage).
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
 
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait_bounded_ns(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait<kCluster>(bar, parity)) return true;
   // back off between tests so that waiting warps leave the issue slots to the
   // warps that have data; check the time limit only now and then
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     __nanosleep(it < 4 ? 32u : 128u);
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<kCluster>(bar, parity)) return true;
     if ((it & 63u) == 0u && global_timer_ns() - t0 > limit_ns) {
       atomicOr(&g_dev_error, TERN_DEVERR_TIMEOUT);
       return false;
@@ -109,8 +122,9 @@ __device__ __forceinline__ bool mbar_wait_bounded_ns(uint64_t* bar, uint32_t par
   }
 }
 
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-  return mbar_wait_bounded_ns(bar, parity, kWaitLimitNs);
+  return mbar_wait_bounded_ns<kCluster>(bar, parity, kWaitLimitNs);
 }
 
 // Programmatic dependent launch: wait until the preceding grid on the stream
@@ -148,6 +162,20 @@ __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
 }
 __device__ __forceinline__ void st_cluster_u64(uint32_t addr, unsigned long long v) {
   asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
+}
+// Store into a CTA's shared memory that completes its byte count on that CTA's
+// mbarrier (`addr` and `bar` mapped into the same CTA of the cluster): the
+// receiver learns of the data by waiting on its own barrier, with no
+// cluster-wide barrier.
+__device__ __forceinline__ void st_async_u32(uint32_t addr, uint32_t v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
+               "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async_u64(uint32_t addr, unsigned long long v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u64 [%0], %1, [%2];" ::"r"(addr), "l"(v),
+               "r"(bar)
+               : "memory");
 }
 
 // 16-byte shared-memory loads from a 32-bit shared address plus an immediate offset.

@@ -288,6 +288,10 @@ def test_bitnet_fused_quant_bit_exact(tern, shape):
 def test_fused_quant_batched_bit_exact(tern, m):
     q8_check(tern, synth.bitnet_layer(300, 1000, seed=m), m)
     q8_check(tern, synth.tq_layer(200, 1024, 2, 32, seed=m), m)
+    if m == 1:  # several tokens: BitNet and TQ2P g32 only
+        # groups of 64 and 128: a warp's 32 four-value words span two groups, or one
+        q8_check(tern, synth.tq_layer(200, 1024, 3, 64, seed=10 + m), m)
+        q8_check(tern, synth.tq_layer(150, 2048, 1, 128, seed=20 + m), m)
 
 
 def test_single_gemv_fused_quant(tern):
