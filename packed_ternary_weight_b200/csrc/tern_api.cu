@@ -183,11 +183,18 @@ bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, in
   if (xs > kMaxSlotsW) return false;
   p.xslots = xs;
   const int colb = bt3 ? kBt3ColBytes : L.planes * kPlaneColBytes;
-  // (warps, stages, stage bytes): sixteen warps with two 6 KB stages each
-  // measured best on the BitNet-2B layer set; when the activation images need
-  // the room (long K), smaller stages keep sixteen warps before fewer warps
-  static const int kShapes[][3] = {{16, 2, 6144}, {16, 2, 4096}, {16, 2, 3072}, {12, 2, 4096},
-                                   {8, 3, 4096},  {8, 2, 4096},  {4, 3, 4096},  {4, 2, 4096}};
+  // (warps, stages, stage bytes): sixteen warps with two stages each, the
+  // stages as large as shared memory allows next to the activation images.
+  // Every stage costs the warp a fixed ~115 instructions (barrier wait, copy
+  // issue, stage bookkeeping; ncu instruction counts per 16-k word at 3, 4 and
+  // 5.5 KB stages), so larger stages cut instructions per weight: on the
+  // BitNet-2B layer set (whose images leave no room for 6 KB) 5.5 KB stages
+  // took 169k SM cycles per step against 186k with 4 KB. Three stages of
+  // 3.5 KB, or twelve warps with 7.5 KB stages, were slower. Smaller stages
+  // and then fewer warps serve long K.
+  static const int kShapes[][3] = {{16, 2, 6144}, {16, 2, 5632}, {16, 2, 5120}, {16, 2, 4096},
+                                   {16, 2, 3072}, {12, 2, 4096}, {8, 3, 4096},  {8, 2, 4096},
+                                   {4, 3, 4096},  {4, 2, 4096}};
   for (const auto& sh : kShapes) {
     p.nw = sh[0];
     p.nstage = sh[1];
