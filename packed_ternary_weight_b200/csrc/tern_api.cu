@@ -121,11 +121,15 @@ Plan2 plan_gemv2(const Layout& L, const int* row_tiles, int nprob, int m, int xm
 }
 
 // Plan of the single-token kernel with one CTA per SM (gemv2w): tile ranges
-// of equal column counts per CTA (gemv2w_cta_tile), about 6 KB stages, as
-// many warps and stages in flight as shared memory allows next to the
-// resident activation images. Applies when
-// the launch has at least four tiles per SM (smaller launches are spread
-// over the SMs by K splits in the row-group kernel).
+// of equal column counts per CTA (gemv2w_cta_tile), 4-6 KB stages, as many
+// warps and stages in flight as shared memory allows next to the resident
+// activation images. Applies when the launch has at least four tiles per SM
+// (smaller launches are spread over the SMs by K splits in the row-group
+// kernel), or one tile per SM with bf16 activations: there the exact 24-bit
+// image makes the launch compute-bound, and sixteen warps on whole tiles beat
+// the K-split kernel (a dependent TQ3P / d = 3 launch of 14336x4096, 448
+// tiles: 19.6 / 29.9 us against 22.6 / 35.3 us; at 128 tiles the K split
+// stays faster).
 // With mt > 1 tokens (one problem, integer activations) a launch of half a
 // tile per SM is enough: each tile carries mt tokens' work. L is the layout of
 // the widest problem (its K sizes the activation images); prob_cols gives
@@ -145,7 +149,7 @@ bool plan_gemv2w(const Layout& L, const int* row_tiles, int nprob, int xmode, in
     cbeg[i + 1] = cbeg[i] + (long long)row_tiles[i] * (prob_cols ? prob_cols[i] : L.cols);
   }
   const int T = begin[nprob];
-  if (T < (mt > 1 ? (sms + 1) / 2 : 4 * sms)) return false;
+  if (T < (mt > 1 ? (sms + 1) / 2 : (xmode == kXBf16 ? sms : 4 * sms))) return false;
   p.mt = mt;
   // the kernel's index arithmetic is 32-bit: all columns, and a CTA's columns
   // x warps, stay below 2^31
