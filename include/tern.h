@@ -182,7 +182,9 @@ tern_status tern_gemv(const tern_desc* desc, const void* d_packed, tern_act act,
  * forms are this library's, the pages run one token at a time).
  *   d_x [m][K] (int8 or bf16 bits), d_xscale float [m] for TERN_ACT_INT8,
  *   d_y [m][N]. For TERN_ACT_INT8 the result is bit-identical to the oracle.
- *   TERN_ACT_BF16 (and so BT3) takes m = 1 only (TERN_EUNSUPPORTED otherwise).
+ *   TERN_ACT_BF16 (TQ and BT3) runs on the CUDA cores for any m: balanced
+ *   ternary reads the weights once per pass of up to eight tokens, the TQ
+ *   planes once per token.
  * For m >= 16 with the 2-bit formats and int8 (or in-kernel quantised bf16)
  * activations the product runs on the tensor cores (tcgen05 int8 MMA, up to
  * 256 tokens per launch); the fp16 group scales are split into small integer
